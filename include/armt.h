@@ -1,0 +1,216 @@
+/*
+ * armt.h -- C ABI of the B200 (sm_100a) Diagonal Batching forward for a
+ * layer-recurrent associative memory transformer (ARMT).
+ *
+ * What the library computes
+ * -------------------------
+ * A forward pass over S segments of seg_len tokens through L layers.  Node
+ * (segment s, layer l) depends only on (s, l-1) and (s-1, l), so the S x L
+ * nodes run as S + L - 1 diagonal waves; wave i holds every node with
+ * s + l = i and runs as ONE grouped layer over stacked per-layer weights
+ * ("Diagonal Batching for Recurrent Memory Transformers" skill page,
+ * "Practical Guidance" and "Architecture Overview"; Pith review of arXiv
+ * 2506.05229, "What carries the argument", "Core claim", Lemma 3.1).  The
+ * same kernels can also run one node at a time in segment-major order (the
+ * S x L baseline of the Pith review's Figure 3) for like-for-like timing.
+ *
+ * Per node the layer math is (the pages give no equations; this is the
+ * reading the library fixes, the plainest one for an ARMT on a LLaMA decoder):
+ *   X  = [emb rows of segment s ; M memory-token rows]      (layer 0 only)
+ *   X += A_l phi(X Wq_mem^T) / (z_l . phi(.) + mem_eps)        memory read
+ *   X += Attn(RMSNorm(X) g_attn)       causal, RoPE, grouped-query heads
+ *   X += MLP(RMSNorm(X) g_mlp)         SwiGLU
+ *   (A_l, z_l) <- delta-rule write from the M memory rows of X
+ *   phi = DPFP of order dpfp_nu (dimension P = 2 * d_key * dpfp_nu)
+ * Rows 0..seg_len-1 of node (s, L-1) are the hidden states of segment s.
+ *
+ * Conventions
+ * -----------
+ * - All entry points return an armt_status; nothing is thrown across the ABI.
+ * - Arguments are validated before any device work: a rejected call launches
+ *   nothing and leaves outputs untouched.
+ * - "device pointer" = memory on the context's CUDA device (cudaMalloc, or
+ *   any allocator handing out device memory, e.g. a framework tensor).
+ * - Matrices are row-major.  Weights use the nn.Linear layout [out, in].
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ * - A context is not thread-safe: calls on one context must not overlap.
+ */
+#ifndef ARMT_H_
+#define ARMT_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct armt_ctx armt_ctx;
+
+typedef enum {
+  ARMT_OK = 0,
+  ARMT_ERR_INVALID_ARG = 1,     /* null pointer, non-positive or inconsistent size */
+  ARMT_ERR_NOT_LOADED = 2,      /* armt_forward before armt_load_weights */
+  ARMT_ERR_SHAPE = 3,           /* S or seg_len above the maxima given at create */
+  ARMT_ERR_OOM = 4,             /* device allocation failed */
+  ARMT_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
+  ARMT_ERR_DEVICE_TIMEOUT = 6,  /* a kernel's bounded wait ran out (reported by armt_device_status) */
+  ARMT_ERR_UNSUPPORTED = 7      /* valid but not implemented shape (e.g. head_dim not 16..128 step 16) */
+} armt_status;
+
+typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1 } armt_dtype;
+
+typedef enum { ARMT_SCHED_DIAGONAL = 0, ARMT_SCHED_SEQUENTIAL = 1 } armt_schedule;
+
+/* Model geometry and numerics.  Uniform layer geometry is required for
+ * stacking the weights (Pith review, "Assumptions & free parameters").
+ *   dtype: weights and activations; fp32 runs SIMT fp32 kernels, bf16 runs
+ *          the tensor-core (tcgen05) path.  The associative memory state
+ *          A, z and the residual stream are fp32 in both modes.
+ *   max_seg_len, max_segments: size the workspace allocated at create. */
+typedef struct {
+  int n_layers;     /* L */
+  int d_model;      /* d */
+  int n_heads;      /* H query heads */
+  int n_kv_heads;   /* KV heads, H % KV == 0 */
+  int head_dim;     /* hd, even */
+  int d_ffn;        /* F */
+  int n_mem;        /* M memory tokens per segment */
+  int d_key;        /* memory key dimension d_k */
+  int dpfp_nu;      /* DPFP order nu */
+  float rope_theta;
+  float rms_eps;
+  float mem_eps;    /* eps in the read and write denominators */
+  armt_dtype dtype;
+  armt_schedule schedule;
+  int max_seg_len;
+  int max_segments;
+} armt_config;
+
+/* Host fp32 weights, row-major, nn.Linear layout [out, in].  The library
+ * copies them (rounding to bf16, round-to-nearest-even, in bf16 mode); the
+ * caller keeps ownership and may free them after armt_load_weights returns. */
+typedef struct {
+  const float* mem_emb;    /* [M, d]        memory-token embeddings */
+  const float* attn_norm;  /* [L, d]        RMSNorm gain before attention */
+  const float* mlp_norm;   /* [L, d]        RMSNorm gain before the MLP */
+  const float* wq;         /* [L, H*hd, d] */
+  const float* wk;         /* [L, KV*hd, d] */
+  const float* wv;         /* [L, KV*hd, d] */
+  const float* wo;         /* [L, d, H*hd] */
+  const float* w_gate;     /* [L, F, d] */
+  const float* w_up;       /* [L, F, d] */
+  const float* w_down;     /* [L, d, F] */
+  const float* wq_mem;     /* [L, d_k, d]   memory read query */
+  const float* wk_mem;     /* [L, d_k, d]   memory write key */
+  const float* wv_mem;     /* [L, d, d]     memory write value */
+} armt_weights;
+
+/* Create a context on the current CUDA device and allocate its workspace for
+ * up to cfg->max_segments segments of cfg->max_seg_len tokens.
+ * Errors: INVALID_ARG (null, non-positive or inconsistent sizes),
+ * UNSUPPORTED (shape outside the kernels' range), OOM, CUDA.  *out is set to
+ * NULL on error. */
+armt_status armt_create(const armt_config* cfg, armt_ctx** out);
+
+/* Copy all weights to the device in the stacked [L, ...] layout the grouped
+ * kernels read (RMSNorm gains folded into the following projection).  May be
+ * called again to replace the weights.  Synchronous.
+ * Errors: INVALID_ARG (null ctx/weights/any tensor pointer), OOM, CUDA. */
+armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* w);
+
+/* Choose the schedule used by later armt_forward calls. */
+armt_status armt_set_schedule(armt_ctx* ctx, armt_schedule schedule);
+
+/* Enable (default) or disable CUDA-graph capture of the whole forward. */
+armt_status armt_set_graph(armt_ctx* ctx, int enable);
+
+/* The forward pass (Pith review, "Core claim"; skill page, "Practical
+ * Guidance": per-layer memory state stays on the GPU, one synchronisation
+ * at the end).  Asynchronous on `stream`; returns after enqueueing.
+ *   emb        device [S*seg_len, d] in the context dtype (fp32 or bf16),
+ *              segment s = rows s*seg_len .. (s+1)*seg_len-1
+ *   out_hidden device [S*seg_len, d] context dtype: final-layer hidden states
+ *   out_A      device [L, d, P] fp32: per-layer associative matrix A_l after
+ *              segment S-1 (starts from 0 in every call)
+ *   out_z      device [L, P] fp32: per-layer normaliser z_l
+ * Buffers must not overlap and must stay valid until the stream reaches the
+ * end of the forward.  P = 2 * d_key * dpfp_nu.
+ * Errors: INVALID_ARG (null pointer, S or seg_len < 1), NOT_LOADED, SHAPE
+ * (S > max_segments or seg_len > max_seg_len), CUDA. */
+armt_status armt_forward(armt_ctx* ctx, const void* emb, int S, int seg_len,
+                         void* out_hidden, float* out_A, float* out_z, void* stream);
+
+/* Same forward with HOST buffers (same shapes and types as armt_forward):
+ * copies emb to the device, runs the forward and copies the results back,
+ * all on `stream`; returns after the stream has finished (synchronous).
+ * Pinned host memory gives full PCIe/C2C bandwidth; pageable memory works.
+ * The device staging buffers are allocated on the first call and kept.
+ * Errors: as armt_forward, plus OOM. */
+armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int seg_len,
+                              void* out_hidden_host, float* out_A_host, float* out_z_host,
+                              void* stream);
+
+/* Wait for `stream`, then report and clear the device-side error word that
+ * kernels set when a bounded wait runs out: ARMT_OK or
+ * ARMT_ERR_DEVICE_TIMEOUT (or ARMT_ERR_CUDA if the stream itself failed). */
+armt_status armt_device_status(armt_ctx* ctx, void* stream);
+
+/* Kernel launches one armt_forward enqueues for (S, current schedule):
+ * the count the caller can compare with a profiler's launch list. */
+armt_status armt_launch_count(armt_ctx* ctx, int S, int* out_count);
+
+/* Kernel kinds the forward launches (grouped GEMMs, attention, memory
+ * read/write, ...): armt_kernel_kinds() of them, named by
+ * armt_kernel_kind_name(k) (NULL for k out of range). */
+int armt_kernel_kinds(void);
+const char* armt_kernel_kind_name(int k);
+
+/* One forward exactly as armt_forward enqueues it but launched directly
+ * (no CUDA graph), with a CUDA event recorded on `stream` before and after
+ * every kernel.  Synchronous.  Adds each kind's device time in milliseconds
+ * to ms[k] and its launch count to launches[k]; both are HOST arrays of
+ * armt_kernel_kinds() entries owned by the caller.  Used to measure each
+ * kernel's duration and achieved fraction of peak.
+ * Errors: as armt_forward. */
+armt_status armt_profile_forward(armt_ctx* ctx, const void* emb, int S, int seg_len, void* out_hidden,
+                                 float* out_A, float* out_z, void* stream, double* ms, int* launches);
+
+/* Free everything the context owns.  NULL is accepted. */
+armt_status armt_destroy(armt_ctx* ctx);
+
+/* Static description of a status code (never NULL). */
+const char* armt_status_string(armt_status s);
+
+/* Last error message recorded on ctx (detail for the last failing call). */
+const char* armt_last_error(armt_ctx* ctx);
+
+/* ------------------------------------------------------------------------
+ * Unit entry points: one grouped kernel on caller-provided device buffers.
+ * They exist so that each kernel can be checked on its own against the
+ * oracle; the forward does not go through them.
+ * ---------------------------------------------------------------------- */
+
+/* Grouped GEMM over G groups: for g < G,
+ *   C[g] (m x n, row-major, fp32) = A[g] (m x k, row-major) * B[bidx[g]]^T
+ * with B stored [num_b, n, k] row-major (nn.Linear layout), A and B bf16
+ * (dtype ARMT_BF16: the tcgen05 tensor-core kernel) or fp32 (ARMT_FP32: SIMT).
+ * A is [G, m, k], C is [G, m, n]; bidx is a HOST array of G indices < num_b.
+ * This is the per-wave "grouped layer" product (skill page, "GroupedGEMM
+ * Operations"), each group indexing its own layer's weights.
+ * Requires k % 8 == 0 (bf16) and n % 16 == 0.  Asynchronous on stream.
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, int k,
+                              const void* A, const void* B, int num_b, const int* bidx,
+                              float* C, void* stream);
+
+/* Delta-rule memory write of one node (the write step above) on device
+ * buffers: m [M, d] fp32 memory rows, wk [d_k, d], wv [d, d] fp32,
+ * A [d, P] and z [P] fp32 updated in place.  Asynchronous on stream.
+ * Errors: INVALID_ARG, CUDA, OOM (scratch allocation). */
+armt_status armt_memory_write(int M, int d, int d_key, int nu, float eps,
+                              const float* m, const float* wk, const float* wv,
+                              float* A, float* z, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARMT_H_ */

@@ -1,0 +1,145 @@
+// Internal declarations shared by the library's translation units.
+// Nothing here is part of the C ABI (include/armt.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/armt.h"
+
+namespace armt {
+
+typedef __nv_bfloat16 bf16;
+
+// One node of the (segment, layer) grid as the kernels see it: x = segment s,
+// y = layer l, z = activation slot (s mod number-of-slots), w = flags.
+typedef int4 NodeEntry;
+
+// A contiguous run of node-table entries launched together (one wave).
+struct Wave {
+  int first;   // index of the wave's first entry in the device node table
+  int count;   // nodes in the wave
+  bool any_first_layer;
+  bool any_last_layer;
+};
+
+// Device workspace.  Activations are per slot: a segment keeps its slot for
+// all its layers, and the <= L segments live in one wave have distinct slots.
+struct Workspace {
+  int slots = 0;
+  int tp_max = 0;           // max rows per node (max_seg_len + n_mem)
+  float* h = nullptr;       // [slots][T'][d] residual stream, fp32
+  void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (act dtype)
+  float* qm = nullptr;      // [slots][T'][dk] memory-read query
+  void* phi = nullptr;      // [slots][T'][P] DPFP features (act dtype)
+  float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
+  void* qkv = nullptr;      // [slots][T'][Nqkv] (act)
+  void* attn = nullptr;     // [slots][T'][H*hd] (act)
+  void* gu = nullptr;       // [slots][T'][2F] (act)
+  void* u = nullptr;        // [slots][T'][F] (act)
+  float* kv = nullptr;      // [slots][M][dk + d]
+  float* phik = nullptr;    // [slots][M][P]
+  float* coef = nullptr;    // [slots][M] 1 / (z . phi_k + eps)
+  float* gamma = nullptr;   // [slots][M]
+  void* a_act = nullptr;    // [L][d][P] act-dtype copy of A (bf16 mode)
+  float2* rope = nullptr;   // [tp_max][hd/2] (cos, sin)
+  NodeEntry* nodes = nullptr;
+  int nodes_cap = 0;
+  unsigned* err = nullptr;  // device error word (bounded waits)
+};
+
+// Device weights in the layout the grouped kernels read.
+struct Weights {
+  bool loaded = false;
+  float* mem_emb = nullptr;  // [M][d] fp32
+  void* w_qkv = nullptr;     // [L][Nqkv][d]   attn gain folded
+  void* w_o = nullptr;       // [L][d][H*hd]
+  void* w_gu = nullptr;      // [L][2F][d]     mlp gain folded; gate rows then up rows
+  void* w_down = nullptr;    // [L][d][F]
+  void* w_qm = nullptr;      // [L][dk][d]
+  void* w_kvm = nullptr;     // [L][dk+d][d]   key rows then value rows
+};
+
+struct Dims {
+  int L, d, H, KV, hd, F, M, dk, nu, P, nqkv;
+  float theta, rms_eps, mem_eps;
+  bool bf16;
+};
+
+}  // namespace armt
+
+struct armt_ctx {
+  armt_config cfg;
+  armt::Dims dm;
+  int device = 0;
+  int sm_count = 0;
+  bool use_graph = true;
+  armt::Weights w;
+  armt::Workspace ws;
+  std::string last_error;
+  // CUDA graph of the last forward
+  cudaGraphExec_t graph_exec = nullptr;
+  cudaStream_t capture_stream = nullptr;
+  struct GraphKey {
+    int S = -1, T = -1, sched = -1;
+    const void* emb = nullptr; void* out = nullptr; float* A = nullptr; float* z = nullptr;
+  } graph_key;
+  // node table of the last (S, schedule)
+  int table_S = -1, table_sched = -1;
+  std::vector<armt::Wave> waves;
+  // host-buffer forward staging
+  void* st_emb = nullptr; void* st_out = nullptr; float* st_A = nullptr; float* st_z = nullptr;
+  size_t st_tokens = 0;
+};
+
+namespace armt {
+
+// ---- kernels launched by the scheduler (all take the wave's node pointer) ----
+
+enum GemmEpi { EPI_STORE_F32 = 0, EPI_STORE_ACT = 1, EPI_RESID = 2 };
+
+struct GemmArgs {
+  const NodeEntry* nodes;
+  int n_nodes;
+  int M, N, K;
+  const void* A; long long a_slot_stride; int lda; int a_by_layer;
+  const void* B; long long b_layer_stride; int ldb;
+  void* C; long long c_slot_stride; int ldc;
+  const float* rowscale; long long rs_slot_stride;   // optional (nullptr)
+  int epi;
+};
+
+// SIMT grouped GEMM; a_bf16/b_bf16/c_bf16 select operand storage types.
+cudaError_t launch_simt_gemm(const GemmArgs& a, bool a_bf16, bool b_bf16, bool c_bf16,
+                             cudaStream_t st);
+
+cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
+                                    const void* emb, const float* mem_emb, float* h, void* xb, cudaStream_t st);
+cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h,
+                           void* xb, float eps, cudaStream_t st);
+cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
+                             const float* z_state, void* phi, float* inv_den, cudaStream_t st);
+cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
+                        const float2* rope, cudaStream_t st);
+cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
+                                  const void* qkv, void* out, cudaStream_t st);
+cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* gu,
+                          void* u, cudaStream_t st);
+cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
+                            float* z_state, float* phik, float* coef, float* gamma, cudaStream_t st);
+cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
+                               const float* phik, const float* coef, float* A_state, void* a_act,
+                               cudaStream_t st);
+cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
+                          const float* h, void* out, cudaStream_t st);
+
+cudaError_t setup_memory_kernels(const Dims& dm);
+
+// fp32 -> act conversions used at weight load
+cudaError_t launch_convert(const float* src, void* dst, size_t n, bool to_bf16, cudaStream_t st);
+
+}  // namespace armt

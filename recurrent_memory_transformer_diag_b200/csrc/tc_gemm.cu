@@ -1,0 +1,569 @@
+// Grouped GEMM on the 5th-generation tensor cores (sm_100a: tcgen05.mma with
+// TMEM accumulators, operands staged by TMA), one launch per wave.
+//
+// Every node g of a wave multiplies its own activations A_g [M x K] by the
+// weights of its own layer B_l [N x K]^T (skill page "Diagonal Batching for
+// Recurrent Memory Transformers", "GroupedGEMM Operations": the wave's layers
+// batched in one grouped kernel; Pith review of arXiv 2506.05229, "What
+// carries the argument": stacked weights + grouped matrix multiplication).
+// The stacked weights are one 3-D tensor [L, N, K]; the layer index is the
+// outer TMA coordinate, so a tile of node g loads B with coordinate l(g).
+//
+// Kernel structure (persistent, one CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (bf16, 128-byte
+//               swizzle) per pipeline stage
+//   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
+//               K=16) and commits stage/accumulator barriers
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (thread = row),
+//               fused per-use epilogue, stores to global memory
+// Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap
+// the main loop of tile t+1.  Tiles never straddle nodes: a node's rows are
+// the middle TMA coordinate with extent M, rows past M read as zeros.
+// Every mbarrier wait is bounded (about one second); on timeout the kernel
+// sets the device error word, drains its own outstanding copies and MMAs,
+// frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "armt_internal.cuh"
+#include "tc_gemm.cuh"
+
+namespace armt {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
+constexpr int NUM_THREADS = 192;
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `parity`; false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, K-major operand, 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (SBO), LBO unused (1),
+// descriptor version 1 (sm_100), layout type 2 = SWIZZLE_128B.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;                 // LBO (16 B units)
+  d |= (uint64_t)(1024 >> 4) << 32;       // SBO (16 B units)
+  d |= (uint64_t)1 << 46;                 // version
+  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: D fp32, A/B bf16, both K-major, shape 128 x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const float* v) {
+  // 32 values = 64 bytes: four 16-byte stores (dst 16-byte aligned)
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 pk;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    reinterpret_cast<uint4*>(dst)[q] = pk;
+  }
+}
+
+template <int BN>
+struct Smem {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
+  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
+};
+
+__device__ __forceinline__ void store_f32x32(float* dst, const float* v, int valid_cols) {
+  if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid_cols) dst[i] = v[i];
+  }
+}
+
+__device__ __forceinline__ void store_act32(bf16* dst, const float* v, int valid_cols) {
+  if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+    store_bf16x32(dst, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid_cols) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+// h += v * rs on 32 columns; v receives the new residual values.
+__device__ __forceinline__ void resid_add32(float* H, float* v, float rs, int valid_cols) {
+  if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float4 o = reinterpret_cast<float4*>(H)[q];
+      o.x = fmaf(v[4 * q], rs, o.x);
+      o.y = fmaf(v[4 * q + 1], rs, o.y);
+      o.z = fmaf(v[4 * q + 2], rs, o.z);
+      o.w = fmaf(v[4 * q + 3], rs, o.w);
+      reinterpret_cast<float4*>(H)[q] = o;
+      v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      if (i < valid_cols) {
+        const float o = fmaf(v[i], rs, H[i]);
+        H[i] = o;
+        v[i] = o;
+      }
+    }
+  }
+}
+
+// Epilogue of one accumulator tile for this thread's row.  Every tcgen05.ld
+// is executed by the whole warp (warp-uniform loops); only the stores are
+// guarded by the row/column bounds.
+template <int BN, int EPI>
+__device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, int slot, int row, bool valid,
+                                             int nb) {
+  const long long rofs = (long long)row;
+  if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+    float rs = 1.f;
+    if (EPI == TC_EPI_RESID && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+#pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+      float v[32];
+      tmem_ld32(tbase + c * 32, v);
+      const int col = nb * BN + c * 32;
+      if (!valid || col >= p.N) continue;
+      const int nv = p.N - col;
+      if (EPI == TC_EPI_F32) {
+        float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+        store_f32x32(C, v, nv);
+      } else {
+        float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
+        resid_add32(H, v, rs, nv);
+        if (EPI == TC_EPI_RESID_ACT) {
+          bf16* X = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+          store_act32(X, v, nv);
+        }
+      }
+    }
+  } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
+    // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
+    const int hd = p.head_dim;
+    const int cph = hd / 32;          // chunks per head
+    const int pairs = hd / 64;        // chunk pairs per head
+#pragma unroll 1
+    for (int hh = 0; hh < BN / hd; ++hh) {
+      const int head = (nb * BN) / hd + hh;
+      const bool rot = head < p.rope_heads;
+#pragma unroll 1
+      for (int pc = 0; pc < pairs; ++pc) {
+        const int c1 = hh * cph + pc, c2 = c1 + pairs;
+        float v1[32], v2[32];
+        tmem_ld32(tbase + c1 * 32, v1);
+        tmem_ld32(tbase + c2 * 32, v2);
+        const int col1 = nb * BN + c1 * 32, col2 = nb * BN + c2 * 32;
+        if (!valid || col1 >= p.N) continue;
+        if (rot) {
+          const float2* cs = p.rope + rofs * p.rope_half + pc * 32;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 a = cs[i];
+            const float x1 = v1[i], x2 = v2[i];
+            v1[i] = x1 * a.x - x2 * a.y;
+            v2[i] = x2 * a.x + x1 * a.y;
+          }
+        }
+        bf16* C = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
+        store_act32(C + col1, v1, p.N - col1);
+        if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+      }
+    }
+  } else if constexpr (EPI == TC_EPI_SWIGLU) {
+    // tile columns [0, BN/2) = gate features f0.., [BN/2, BN) = up features f0..
+    constexpr int HALF = BN / 2;
+    const int f0 = nb * HALF;
+#pragma unroll 1
+    for (int c = 0; c < HALF / 32; ++c) {
+      float g[32], u[32];
+      tmem_ld32(tbase + c * 32, g);
+      tmem_ld32(tbase + HALF + c * 32, u);
+      const int f = f0 + c * 32;
+      if (!valid || f >= p.f_out) continue;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.f + __expf(-g[i])) * u[i];
+      bf16* C = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + f;
+      store_act32(C, g, p.f_out - f);
+    }
+  }
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const TcGemmParams p) {
+  using SM = Smem<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFFSET);
+  uint64_t* empty = full + SM::STAGES;
+  uint64_t* tfull = empty + SM::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SM::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(2 * BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int tiles_per_node = p.m_tiles * p.n_tiles;
+  const int total = p.n_nodes * tiles_per_node;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;   // bit s: stage s has an issued load not yet seen complete by the consumer
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+        const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+        const NodeEntry nd = p.nodes[node];
+        const int a_outer = p.a_by_layer ? nd.y : nd.z;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          armed &= ~(1u << stage);
+          uint8_t* sa = smem + stage * SM::STAGE_BYTES;
+          mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
+          tma_load_3d(&tmA, &full[stage], sa, kb * BK, mb * BM, a_outer);
+          tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BK, nb * BN, nd.y);
+          armed |= 1u << stage;
+          if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        atomicOr(p.err, 1u);
+        *abort_flag = 1;
+      }
+      // drain: wait (bounded) until every issued copy has landed
+      if (*abort_flag) {
+        for (int s = 0; s < SM::STAGES; ++s) {
+          if (!(armed & (1u << s))) continue;
+          const unsigned long long t0 = global_ns();
+          // the latest phase of stage s is either complete or will complete; poll both parities
+          while (!mbar_try_wait(&full[s], 0) && !mbar_try_wait(&full[s], 1)) {
+            if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t IDESC = idesc_bf16(BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * SM::STAGE_BYTES);
+          const uint32_t sb = sa + SM::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[buf]);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      }
+      if (!ok) {
+        atomicOr(p.err, 2u);
+        *abort_flag = 1;
+      }
+      // make sure no MMA is still writing TMEM before it is freed
+      mma_commit(drain);
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(drain, 0)) {
+        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const bool got = mbar_wait(&tfull[buf], acc_phase, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) atomicOr(p.err, 4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = mb * BM + row_in_tile;
+      const bool valid = row < p.M;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+      run_epilogue<BN, EPI>(p, tbase, nd.z, row, valid, nb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * BN) : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, int sm_count,
+                          cudaStream_t st) {
+  using SM = Smem<BN>;
+  const int total = p.n_nodes * p.m_tiles * p.n_tiles;
+  const int grid = total < sm_count ? total : sm_count;
+  tc_gemm_kernel<BN, EPI><<<grid, NUM_THREADS, SM::TOTAL, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+template <int BN, int EPI>
+cudaError_t configure() {
+  return cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Smem<BN>::TOTAL);
+}
+
+}  // namespace
+
+cudaError_t setup_tc_gemm() {
+  static bool done = false;
+  if (done) return cudaSuccess;
+  cudaError_t e = configure<256, TC_EPI_F32>();
+  if (e == cudaSuccess) e = configure<128, TC_EPI_F32>();
+  if (e == cudaSuccess) e = configure<64, TC_EPI_F32>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_RESID>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_RESID_ACT>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_QKV_ROPE>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_SWIGLU>();
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
+// 3-D tensor map over a bf16 array [outer][rows][inner] (inner contiguous),
+// box = box_inner x box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows, int outer, int box_inner,
+                         int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * rows * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+bool tc_gemm_supported(int m, int n, int k) {
+  (void)m;
+  return k % 8 == 0 && n % 16 == 0 && get_encode_fn() != nullptr;
+}
+
+int tc_pick_bn(int n) { return n >= 256 ? 256 : (n >= 128 ? 128 : 64); }
+
+cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
+                           cudaStream_t st) {
+  CUtensorMap ta, tb;
+  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn);
+  if (e != cudaSuccess) return e;
+  p.m_tiles = (p.M + BM - 1) / BM;
+  p.n_tiles = (p.N + bn - 1) / bn;
+  p.k_blocks = (p.K + BK - 1) / BK;
+#define ARMT_TC_CASE(BNV, E) \
+  if (bn == BNV && epi == E) return launch_kernel<BNV, E>(ta, tb, p, sm_count, st);
+  ARMT_TC_CASE(256, TC_EPI_F32)
+  ARMT_TC_CASE(128, TC_EPI_F32)
+  ARMT_TC_CASE(64, TC_EPI_F32)
+  ARMT_TC_CASE(256, TC_EPI_RESID)
+  ARMT_TC_CASE(256, TC_EPI_RESID_ACT)
+  ARMT_TC_CASE(256, TC_EPI_QKV_ROPE)
+  ARMT_TC_CASE(256, TC_EPI_SWIGLU)
+#undef ARMT_TC_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
+                                const NodeEntry* nodes, float* C, unsigned* err, cudaStream_t st) {
+  int dev = 0, sms = 148;
+  cudaError_t se = setup_tc_gemm();
+  if (se != cudaSuccess) return se;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  TcGemmOperands op;
+  op.A = A; op.a_rows = m; op.a_outer = G;
+  op.B = B; op.b_rows = n; op.b_outer = num_b;
+  TcGemmParams p{};
+  p.nodes = nodes; p.n_nodes = G; p.M = m; p.N = n; p.K = k;
+  p.C = C; p.c_slot_stride = (long long)m * n; p.ldc = n;
+  p.err = err;
+  const int bn = tc_pick_bn(n);
+  return launch_tc_gemm(op, p, TC_EPI_F32, bn, sms, st);
+}
+
+}  // namespace armt

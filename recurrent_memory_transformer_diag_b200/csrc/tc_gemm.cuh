@@ -1,0 +1,44 @@
+// Interface of the tcgen05 grouped GEMM (tc_gemm.cu).
+#pragma once
+
+#include "armt_internal.cuh"
+
+namespace armt {
+
+// Fused epilogues (thread = one accumulator row; see tc_gemm.cu).
+enum TcEpi {
+  TC_EPI_F32 = 0,        // C (fp32) = acc
+  TC_EPI_RESID = 1,      // h += acc * rowscale[row]   (rowscale optional)
+  TC_EPI_RESID_ACT = 2,  // h += acc; C (bf16) = h     (GEMM-operand copy of the new residual)
+  TC_EPI_QKV_ROPE = 3,   // C (bf16) = acc, rotate-half RoPE on heads < rope_heads
+  TC_EPI_SWIGLU = 4      // C (bf16)[f] = silu(acc[gate f]) * acc[up f]; B rows interleaved per 128
+};
+
+struct TcGemmParams {
+  const NodeEntry* nodes;
+  int n_nodes;
+  int M, N, K;              // per node: rows, B rows (output columns), reduction
+  int m_tiles, n_tiles, k_blocks;
+  int a_by_layer;           // A's outer TMA coordinate: 0 = node slot, 1 = node layer
+  void* C; long long c_slot_stride; int ldc;
+  float* h; long long h_slot_stride; int ldh;
+  const float* rowscale; long long rs_slot_stride;
+  const float2* rope; int rope_half; int rope_heads; int head_dim;
+  int f_out;                // SWIGLU: number of valid output features
+  unsigned* err;            // device error word (bounded waits)
+};
+
+struct TcGemmOperands {
+  const void* A; int a_rows; int a_outer;   // bf16 [a_outer][a_rows][K]
+  const void* B; int b_rows; int b_outer;   // bf16 [b_outer][b_rows][K]
+};
+
+cudaError_t setup_tc_gemm();
+int tc_pick_bn(int n);
+bool tc_gemm_supported(int m, int n, int k);
+cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
+                           cudaStream_t st);
+cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
+                                const NodeEntry* nodes, float* C, unsigned* err, cudaStream_t st);
+
+}  // namespace armt

@@ -9,3 +9,15 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+import pytest  # noqa: E402
+
+
+@pytest.fixture(scope="session")
+def libarmt():
+    """The in-tree libarmt.so, rebuilt first if any source is newer."""
+    from recurrent_memory_transformer_diag_b200 import build
+    build.build()
+    from recurrent_memory_transformer_diag_b200 import armt
+    return armt.lib()

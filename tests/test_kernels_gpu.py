@@ -1,0 +1,76 @@
+"""Single kernels through the unit entry points, against the oracle."""
+import numpy as np
+import pytest
+
+import oracle
+
+from .gpu_util import rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("G,m,n,k,num_b", [
+    (1, 128, 256, 64, 1),       # one tile, one k block
+    (3, 1040, 512, 2048, 5),    # ragged M (8 full tiles + 16 rows), many k blocks
+    (2, 144, 768, 688, 4),      # ragged K (10.75 k blocks)
+    (4, 200, 64, 384, 2),       # N = 64 tile width
+    (2, 77, 128, 136, 3),       # N = 128, tiny ragged M and K
+    (16, 1040, 3072, 2048, 16), # a full 1B wave of QKV shapes
+])
+def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b):
+    import torch
+    from recurrent_memory_transformer_diag_b200 import grouped_gemm
+    g = torch.Generator().manual_seed(G * 1000 + m + n + k)
+    A = torch.randn(G, m, k, generator=g).to(torch.bfloat16)
+    B = (torch.randn(num_b, n, k, generator=g) * 0.05).to(torch.bfloat16)
+    bidx = [(3 * i + 1) % num_b for i in range(G)]
+    C = torch.full((G, m, n), float("nan"), device="cuda")
+    grouped_gemm(A.cuda(), B.cuda(), bidx, C)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    An = A.float().numpy().astype(np.float64)
+    Bn = B.float().numpy().astype(np.float64)
+    for i in range(G):
+        ref = An[i] @ Bn[bidx[i]].T
+        assert rel_l2(got[i], ref) < 1e-5, (i, rel_l2(got[i], ref))
+
+
+def test_simt_grouped_gemm_fp32_matches_fp64():
+    import torch
+    from recurrent_memory_transformer_diag_b200 import grouped_gemm
+    g = torch.Generator().manual_seed(5)
+    A = torch.randn(3, 70, 172, generator=g)
+    B = torch.randn(2, 90, 172, generator=g)
+    C = torch.empty(3, 70, 90, device="cuda")
+    grouped_gemm(A.cuda(), B.cuda(), [1, 0, 1], C)
+    torch.cuda.synchronize()
+    for i, b in enumerate([1, 0, 1]):
+        ref = A[i].double().numpy() @ B[b].double().numpy().T
+        assert rel_l2(C[i].cpu().numpy(), ref) < 1e-6
+
+
+@pytest.mark.parametrize("M,d,dk,nu", [(4, 64, 16, 2), (16, 256, 64, 3), (16, 2048, 64, 3), (16, 3072, 128, 3)])
+def test_memory_write_matches_oracle(M, d, dk, nu):
+    import torch
+    from recurrent_memory_transformer_diag_b200 import memory_write
+    rng = np.random.default_rng(M + d)
+    P = 2 * dk * nu
+    m = rng.standard_normal((M, d)).astype(np.float32)
+    wk = (0.02 * rng.standard_normal((dk, d))).astype(np.float32)
+    wv = (0.02 * rng.standard_normal((d, d))).astype(np.float32)
+    # a non-trivial prior state: two earlier writes
+    A0 = np.zeros((d, P))
+    z0 = np.zeros(P)
+    for _ in range(2):
+        prev = rng.standard_normal((M, d)).astype(np.float32)
+        A0, z0 = oracle.mem_write(prev, wk, wv, A0, z0, nu, 1e-5)
+    A0 = A0.astype(np.float32)
+    z0 = z0.astype(np.float32)
+    Ar, zr = oracle.mem_write(m, wk, wv, A0, z0, nu, 1e-5)
+    At = torch.from_numpy(A0).cuda()
+    zt = torch.from_numpy(z0).cuda()
+    memory_write(torch.from_numpy(m).cuda(), torch.from_numpy(wk).cuda(), torch.from_numpy(wv).cuda(),
+                 At, zt, nu, 1e-5)
+    torch.cuda.synchronize()
+    assert rel_l2(At.cpu().numpy(), Ar) < 1e-5
+    assert rel_l2(zt.cpu().numpy(), zr) < 1e-5
