@@ -146,7 +146,7 @@ void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeE
 const char* const KIND_NAMES[] = {
     "init", "gemm_qmem", "tc_qmem", "dpfp_read", "gemm_read", "tc_read", "norm_attn", "gemm_qkv",
     "rope", "tc_qkv_rope", "attention", "gemm_o", "tc_o", "norm_mlp", "gemm_gateup", "swiglu",
-    "tc_gateup_swiglu", "gemm_down", "tc_down", "gemm_kvmem", "memw_phi", "memw_update", "output"};
+    "tc_gateup_swiglu", "gemm_down", "tc_down", "gemm_kvmem", "tc_kvmem", "memw_phi", "memw_update", "output"};
 constexpr int N_KINDS = (int)(sizeof(KIND_NAMES) / sizeof(KIND_NAMES[0]));
 
 int kind_index(const char* name) {
@@ -341,7 +341,10 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.rope = ws.rope; p.rope_half = dm.hd / 2; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
     return launch_tc_gemm(op, p, TC_EPI_QKV_ROPE, 256, sms, st);
   });
-  L("attention", [&] { return launch_attention_simt(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
+  L("attention", [&] {
+    return attention_mma_supported(dm) ? launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st)
+                                       : launch_attention_simt(dm, nodes, n, Tp, ws.qkv, ws.attn, st);
+  });
   L("tc_o", [&] {
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
@@ -365,16 +368,15 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
 
-  // ---- memory write from the M memory rows of the layer output (fp32 rows)
-  {
-    GemmArgs g{};
-    g.nodes = nodes; g.n_nodes = n; g.M = dm.M; g.N = dm.dk + dm.d; g.K = dm.d;
-    g.A = ws.h + (long long)T * dm.d; g.a_slot_stride = hs; g.lda = dm.d;
-    g.B = w.w_kvm; g.b_layer_stride = (long long)(dm.dk + dm.d) * dm.d; g.ldb = dm.d;
-    g.C = ws.kv; g.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); g.ldc = dm.dk + dm.d;
-    g.epi = EPI_STORE_F32;
-    L("gemm_kvmem", [&] { return launch_simt_gemm(g, false, true, false, st); });
-  }
+  // ---- memory write: [k | v] = m [Wk_mem; Wv_mem]^T for the M memory rows
+  // (rows T..T'-1 of the bf16 copy of the layer output the down GEMM wrote)
+  L("tc_kvmem", [&] {
+    TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, dm.dk + dm.d, dm.L};
+    op.a_pitch = Tp;
+    TcGemmParams p; base(p, dm.M, dm.dk + dm.d, dm.d);
+    p.C = ws.kv; p.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); p.ldc = dm.dk + dm.d;
+    return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, st);
+  });
   L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.coef, ws.gamma, st); });
   L("memw_update", [&] { return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.coef, A, ws.a_act, st); });
 
@@ -550,6 +552,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   }
   if (e == cudaSuccess) e = setup_memory_kernels(dm);
   if (e == cudaSuccess && dm.bf16) e = setup_tc_gemm();
+  if (e == cudaSuccess && dm.bf16) e = setup_attention_mma();
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ctx->capture_stream, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     armt_status s = cuda_fail(nullptr, e, "create");

@@ -139,6 +139,12 @@ cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, 
 
 cudaError_t setup_memory_kernels(const Dims& dm);
 
+// bf16 tensor-core attention (mma.sync); head_dim 64 or 128
+bool attention_mma_supported(const Dims& dm);
+cudaError_t setup_attention_mma();
+cudaError_t launch_attention_mma(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* qkv, void* out,
+                                 cudaStream_t st);
+
 // fp32 -> act conversions used at weight load
 cudaError_t launch_convert(const float* src, void* dst, size_t n, bool to_bf16, cudaStream_t st);
 

@@ -95,8 +95,11 @@ cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const
   return cudaGetLastError();
 }
 
+constexpr int MEMW_ROWS_PER_BLOCK = 64;
+
 // A_state: [L][d][P] fp32 in place; a_act: optional bf16 copy [L][d][P].
-// grid (ceil(d / 8), nodes), 8 warps, one A row per warp per iteration.
+// grid (ceil(d / ROWS_PER_BLOCK), nodes), 8 warps, one A row per warp per
+// iteration; phi is staged once per block.
 template <int MAXC>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
@@ -111,47 +114,49 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   for (int e = threadIdx.x; e < M; e += blockDim.x) cf[e] = coef[(long long)slot * M + e];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = blockIdx.x * 8 + warp;
-  if (i >= d) return;
-  float* Arow = A_state + ((long long)layer * d + i) * P;
-  float a[MAXC];
-#pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int p = lane + 32 * c;
-    a[c] = p < P ? Arow[p] : 0.f;
-  }
-  float* dl = delta + warp * M;
-  for (int j = 0; j < M; ++j) {
-    const float* pj = ph + j * P;
-    float dot = 0.f;
-#pragma unroll
+  const int i_end = min(d, (blockIdx.x + 1) * MEMW_ROWS_PER_BLOCK);
+  for (int i = blockIdx.x * MEMW_ROWS_PER_BLOCK + warp; i < i_end; i += 8) {
+    float* Arow = A_state + ((long long)layer * d + i) * P;
+    float a[MAXC];
+  #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
-      if (p < P) dot = fmaf(a[c], pj[p], dot);
+      a[c] = p < P ? Arow[p] : 0.f;
     }
-    dot = warp_sum_m(dot);
-    if (lane == 0) {
-      const float v = kv[((long long)slot * M + j) * (dk + d) + dk + i];
-      dl[j] = v - dot * cf[j];
+    float* dl = delta + warp * M;
+    for (int j = 0; j < M; ++j) {
+      const float* pj = ph + j * P;
+      float dot = 0.f;
+  #pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int p = lane + 32 * c;
+        if (p < P) dot = fmaf(a[c], pj[p], dot);
+      }
+      dot = warp_sum_m(dot);
+      if (lane == 0) {
+        const float v = kv[((long long)slot * M + j) * (dk + d) + dk + i];
+        dl[j] = v - dot * cf[j];
+      }
     }
-  }
-  __syncwarp();
-#pragma unroll
-  for (int c = 0; c < MAXC; ++c) {
-    const int p = lane + 32 * c;
-    if (p < P) {
-      float acc = a[c];
-      for (int j = 0; j < M; ++j) acc = fmaf(dl[j], ph[j * P + p], acc);
-      Arow[p] = acc;
-      if (a_act) a_act[((long long)layer * d + i) * P + p] = __float2bfloat16_rn(acc);
+    __syncwarp();
+  #pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int p = lane + 32 * c;
+      if (p < P) {
+        float acc = a[c];
+        for (int j = 0; j < M; ++j) acc = fmaf(dl[j], ph[j * P + p], acc);
+        Arow[p] = acc;
+        if (a_act) a_act[((long long)layer * d + i) * P + p] = __float2bfloat16_rn(acc);
+      }
     }
+    __syncwarp();
   }
 }
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                                const float* phik, const float* coef, float* A_state, void* a_act,
                                cudaStream_t st) {
-  dim3 grid((dm.d + 7) / 8, n);
+  dim3 grid((dm.d + MEMW_ROWS_PER_BLOCK - 1) / MEMW_ROWS_PER_BLOCK, n);
   const size_t sh = ((size_t)dm.M * dm.P + dm.M + 8 * dm.M) * sizeof(float);
   const int chunks = (dm.P + 31) / 32;
 #define ARMT_MEMW_CASE(C)                                                                        \

@@ -491,6 +491,7 @@ cudaError_t configure() {
 cudaError_t setup_tc_gemm() {
   static bool done = false;
   if (done) return cudaSuccess;
+  if (!get_encode_fn()) return cudaErrorNotSupported;
   cudaError_t e = configure<256, TC_EPI_F32>();
   if (e == cudaSuccess) e = configure<128, TC_EPI_F32>();
   if (e == cudaSuccess) e = configure<64, TC_EPI_F32>();
@@ -502,14 +503,16 @@ cudaError_t setup_tc_gemm() {
   return e;
 }
 
-// 3-D tensor map over a bf16 array [outer][rows][inner] (inner contiguous),
-// box = box_inner x box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+// 3-D tensor map over a bf16 array [outer][rows][inner] (inner contiguous;
+// consecutive outer indices pitch_rows rows apart), box = box_inner x
+// box_rows x 1, 128-byte swizzle, zero fill out of bounds.
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows, int outer, int box_inner,
-                         int box_rows) {
+                         int box_rows, int pitch_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
   if (!enc) return cudaErrorNotSupported;
+  if (pitch_rows <= 0) pitch_rows = rows;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
-  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * rows * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * pitch_rows * 2};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -528,9 +531,9 @@ int tc_pick_bn(int n) { return n >= 256 ? 256 : (n >= 128 ? 128 : 64); }
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st) {
   CUtensorMap ta, tb;
-  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM);
+  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM, op.a_pitch);
   if (e != cudaSuccess) return e;
-  e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn);
+  e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn, 0);
   if (e != cudaSuccess) return e;
   p.m_tiles = (p.M + BM - 1) / BM;
   p.n_tiles = (p.N + bn - 1) / bn;

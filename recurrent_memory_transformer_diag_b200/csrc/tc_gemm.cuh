@@ -29,8 +29,9 @@ struct TcGemmParams {
 };
 
 struct TcGemmOperands {
-  const void* A; int a_rows; int a_outer;   // bf16 [a_outer][a_rows][K]
+  const void* A; int a_rows; int a_outer;   // bf16 [a_outer][a_rows][K] (rows a_pitch apart per outer step)
   const void* B; int b_rows; int b_outer;   // bf16 [b_outer][b_rows][K]
+  int a_pitch = 0;                          // rows between outer steps of A (0 = a_rows)
 };
 
 cudaError_t setup_tc_gemm();

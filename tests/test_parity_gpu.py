@@ -162,5 +162,9 @@ def test_launch_count_diagonal_vs_sequential(small):
     ns = m.launch_count(S)
     m.close()
     assert nd < ns
-    per_node_max = ns / (S * L)
-    assert nd <= (S + L - 1) * per_node_max
+    # per wave: the same kernel sequence, plus the layer-0 input kernel when
+    # the wave holds a layer-0 node and the output kernel when it holds a
+    # last-layer node (S of each in both schedules)
+    per_wave = (ns - 2 * S) // (S * L)
+    assert ns == S * L * per_wave + 2 * S
+    assert nd == (S + L - 1) * per_wave + 2 * S
