@@ -248,11 +248,13 @@ def run_ours(args, cfg, S):
         barrier(world)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.nvtx.range_push(f"timed_{schedule}")
         e0.record(stream)
         for _ in range(n_steps):
             m.forward(emb, S, T, out, A, z)
         e1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
         barrier(world)
         m.device_status()
         return e0.elapsed_time(e1) / n_steps

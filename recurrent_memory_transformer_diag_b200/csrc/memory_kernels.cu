@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   for (int i = blockIdx.x * MEMW_ROWS_PER_BLOCK + warp; i < i_end; i += 8) {
     float* Arow = A_state + ((long long)layer * d + i) * P;
     float a[MAXC];
-  #pragma unroll
+#pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       a[c] = p < P ? Arow[p] : 0.f;
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
     for (int j = 0; j < M; ++j) {
       const float* pj = ph + j * P;
       float dot = 0.f;
-  #pragma unroll
+#pragma unroll
       for (int c = 0; c < MAXC; ++c) {
         const int p = lane + 32 * c;
         if (p < P) dot = fmaf(a[c], pj[p], dot);
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
       }
     }
     __syncwarp();
-  #pragma unroll
+#pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       if (p < P) {
