@@ -55,15 +55,22 @@ typedef enum {
   ARMT_ERR_UNSUPPORTED = 7      /* valid but not implemented shape (e.g. head_dim not 16..128 step 16) */
 } armt_status;
 
-typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1 } armt_dtype;
+/* ARMT_FP32: fp32 weights and activations, SIMT kernels.
+ * ARMT_BF16: weights rounded to bf16 (round to nearest even) on load; the
+ *   tensor-core path stores these bf16 values in fp16 (exact for every value
+ *   of magnitude >= 2^-17) and keeps the GEMM activations in fp16, which the
+ *   tcgen05 tensor cores multiply at the bf16 rate with 3 more mantissa bits;
+ *   accumulation, residual stream and memory state are fp32; embeddings in
+ *   and hidden states out are bf16.
+ * ARMT_F16: fp16 operands; accepted by armt_grouped_gemm only. */
+typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1, ARMT_F16 = 2 } armt_dtype;
 
 typedef enum { ARMT_SCHED_DIAGONAL = 0, ARMT_SCHED_SEQUENTIAL = 1 } armt_schedule;
 
 /* Model geometry and numerics.  Uniform layer geometry is required for
  * stacking the weights (Pith review, "Assumptions & free parameters").
- *   dtype: weights and activations; fp32 runs SIMT fp32 kernels, bf16 runs
- *          the tensor-core (tcgen05) path.  The associative memory state
- *          A, z and the residual stream are fp32 in both modes.
+ *   dtype: ARMT_FP32 or ARMT_BF16 (see armt_dtype).  The associative
+ *          memory state A, z and the residual stream are fp32 in both modes.
  *   max_seg_len, max_segments: size the workspace allocated at create. */
 typedef struct {
   int n_layers;     /* L */
@@ -190,8 +197,9 @@ const char* armt_last_error(armt_ctx* ctx);
 
 /* Grouped GEMM over G groups: for g < G,
  *   C[g] (m x n, row-major, fp32) = A[g] (m x k, row-major) * B[bidx[g]]^T
- * with B stored [num_b, n, k] row-major (nn.Linear layout), A and B bf16
- * (dtype ARMT_BF16: the tcgen05 tensor-core kernel) or fp32 (ARMT_FP32: SIMT).
+ * with B stored [num_b, n, k] row-major (nn.Linear layout), A and B both bf16
+ * (ARMT_BF16) or both fp16 (ARMT_F16) on the tcgen05 tensor-core kernel, or
+ * fp32 (ARMT_FP32) on the SIMT kernel.
  * A is [G, m, k], C is [G, m, n]; bidx is a HOST array of G indices < num_b.
  * This is the per-wave "grouped layer" product (skill page, "GroupedGEMM
  * Operations"), each group indexing its own layer's weights.

@@ -19,7 +19,7 @@ from .inputs import ArmtConfig
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libarmt.so")
 
-ARMT_FP32, ARMT_BF16 = 0, 1
+ARMT_FP32, ARMT_BF16, ARMT_F16 = 0, 1, 2
 SCHED = {"diagonal": 0, "sequential": 1}
 
 STATUS = {
@@ -207,9 +207,9 @@ class Armt:
 
 
 def grouped_gemm(A, B, bidx, C, stream=None):
-    """C[g] = A[g] @ B[bidx[g]]^T on device tensors; bf16 -> tcgen05 kernel, fp32 -> SIMT."""
+    """C[g] = A[g] @ B[bidx[g]]^T on device tensors; bf16/fp16 -> tcgen05 kernel, fp32 -> SIMT."""
     import torch
-    dtype = ARMT_BF16 if A.dtype == torch.bfloat16 else ARMT_FP32
+    dtype = {torch.bfloat16: ARMT_BF16, torch.float16: ARMT_F16}.get(A.dtype, ARMT_FP32)
     G, m, k = A.shape
     num_b, n, _ = B.shape
     idx = (ctypes.c_int * G)(*[int(i) for i in bidx])

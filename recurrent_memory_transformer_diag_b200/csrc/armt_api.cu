@@ -103,6 +103,9 @@ armt_status validate_config(const armt_config* c, const char** why) {
   if (c->dtype == ARMT_BF16 && (c->d_model % 8 || c->d_ffn % 8 || (c->n_heads * c->head_dim) % 8 || P % 8)) {
     *why = "bf16 mode needs d_model, d_ffn, H*hd and phi dimension multiples of 8"; return ARMT_ERR_UNSUPPORTED;
   }
+  if (c->dtype == ARMT_BF16 && c->head_dim != 64 && c->head_dim != 128) {
+    *why = "bf16 mode needs head_dim 64 or 128"; return ARMT_ERR_UNSUPPORTED;
+  }
   return ARMT_OK;
 }
 
@@ -190,7 +193,8 @@ struct Launcher {
   }
 };
 
-// Enqueue every kernel of one wave.  T = seg_len, Tp = T + M rows per node.
+// fp32 path: enqueue every kernel of one wave (SIMT kernels, fp32 throughout).
+// T = seg_len, Tp = T + M rows per node.
 void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
                   cudaStream_t st, Launcher& L) {
   const Dims& dm = ctx->dm;
@@ -199,9 +203,8 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   const int Tp = T + dm.M;
   const int n = wv.count;
   const NodeEntry* nodes = ws.nodes + wv.first;
-  const bool bf = dm.bf16;
   const long long hs = (long long)Tp * dm.d;
-  void* a_read = bf ? ws.a_act : (void*)A;
+  void* a_read = A;
 
   if (wv.any_first_layer)
     L("init", [&] { return launch_init_first_layer(dm, nodes, n, T, Tp, emb, w.mem_emb, ws.h, nullptr, st); });
@@ -214,7 +217,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_qm; g.b_layer_stride = (long long)dm.dk * dm.d; g.ldb = dm.d;
     g.C = ws.qm; g.c_slot_stride = (long long)Tp * dm.dk; g.ldc = dm.dk;
     g.epi = EPI_STORE_F32;
-    L("gemm_qmem", [&] { return launch_simt_gemm(g, false, bf, false, st); });
+    L("gemm_qmem", [&] { return launch_simt_gemm(g, st); });
   }
   L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
   {
@@ -225,7 +228,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.C = ws.h; g.c_slot_stride = hs; g.ldc = dm.d;
     g.rowscale = ws.inv_den; g.rs_slot_stride = Tp;
     g.epi = EPI_RESID;
-    L("gemm_read", [&] { return launch_simt_gemm(g, bf, bf, false, st); });
+    L("gemm_read", [&] { return launch_simt_gemm(g, st); });
   }
 
   // ---- attention block
@@ -237,7 +240,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_qkv; g.b_layer_stride = (long long)dm.nqkv * dm.d; g.ldb = dm.d;
     g.C = ws.qkv; g.c_slot_stride = (long long)Tp * dm.nqkv; g.ldc = dm.nqkv;
     g.epi = EPI_STORE_ACT;
-    L("gemm_qkv", [&] { return launch_simt_gemm(g, bf, bf, bf, st); });
+    L("gemm_qkv", [&] { return launch_simt_gemm(g, st); });
   }
   L("rope", [&] { return launch_rope(dm, nodes, n, Tp, ws.qkv, ws.rope, st); });
   L("attention", [&] { return launch_attention_simt(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
@@ -248,7 +251,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_o; g.b_layer_stride = (long long)dm.d * dm.H * dm.hd; g.ldb = dm.H * dm.hd;
     g.C = ws.h; g.c_slot_stride = hs; g.ldc = dm.d;
     g.epi = EPI_RESID;
-    L("gemm_o", [&] { return launch_simt_gemm(g, bf, bf, false, st); });
+    L("gemm_o", [&] { return launch_simt_gemm(g, st); });
   }
 
   // ---- MLP block
@@ -260,7 +263,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_gu; g.b_layer_stride = 2LL * dm.F * dm.d; g.ldb = dm.d;
     g.C = ws.gu; g.c_slot_stride = 2LL * Tp * dm.F; g.ldc = 2 * dm.F;
     g.epi = EPI_STORE_ACT;
-    L("gemm_gateup", [&] { return launch_simt_gemm(g, bf, bf, bf, st); });
+    L("gemm_gateup", [&] { return launch_simt_gemm(g, st); });
   }
   L("swiglu", [&] { return launch_swiglu(dm, nodes, n, Tp, ws.gu, ws.u, st); });
   {
@@ -270,7 +273,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_down; g.b_layer_stride = (long long)dm.d * dm.F; g.ldb = dm.F;
     g.C = ws.h; g.c_slot_stride = hs; g.ldc = dm.d;
     g.epi = EPI_RESID;
-    L("gemm_down", [&] { return launch_simt_gemm(g, bf, bf, false, st); });
+    L("gemm_down", [&] { return launch_simt_gemm(g, st); });
   }
 
   // ---- memory write from the M memory rows of the layer output
@@ -281,20 +284,25 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.B = w.w_kvm; g.b_layer_stride = (long long)(dm.dk + dm.d) * dm.d; g.ldb = dm.d;
     g.C = ws.kv; g.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); g.ldc = dm.dk + dm.d;
     g.epi = EPI_STORE_F32;
-    L("gemm_kvmem", [&] { return launch_simt_gemm(g, false, bf, false, st); });
+    L("gemm_kvmem", [&] { return launch_simt_gemm(g, st); });
   }
   L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.coef, ws.gamma, st); });
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.coef, A, bf ? ws.a_act : nullptr, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.coef, A, nullptr, st);
   });
 
   if (wv.any_last_layer)
     L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
 }
 
-// bf16 path: the dense products run on the tcgen05 grouped GEMM with fused
-// epilogues; the row-wise steps (norm, DPFP, attention, memory write) are the
-// same kernels as the fp32 path.
+// Tensor-core path (bf16 mode): the dense products run on the tcgen05 grouped
+// GEMM with fused epilogues, attention on tensor cores.  Weights hold the
+// bf16-rounded values in fp16 containers and the GEMM activations are fp16
+// (same tensor-core rate as bf16, 3 more mantissa bits: rounding the
+// normalised activations to bf16 alone costs ~1 % relative error over 16
+// layers); the memory-read product phi A^T keeps bf16 operands because A
+// spans a wide range of magnitudes.  Residual stream, accumulation and the
+// memory state are fp32.
 void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
                      cudaStream_t st, Launcher& L) {
   const Dims& dm = ctx->dm;
@@ -314,7 +322,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   };
 
   if (wv.any_first_layer)
-    L("init", [&] { return launch_init_first_layer(dm, nodes, n, T, Tp, emb, w.mem_emb, ws.h, ws.xb, st); });
+    L("init", [&] { return launch_init_first_layer(dm, nodes, n, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st); });
 
   // ---- memory read
   L("tc_qmem", [&] {
@@ -327,6 +335,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   L("tc_read", [&] {
     TcGemmOperands op{ws.phi, Tp, slots, ws.a_act, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.P);
+    p.ab_bf16 = 1;
     p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
     p.rowscale = ws.inv_den; p.rs_slot_stride = Tp;
     return launch_tc_gemm(op, p, TC_EPI_RESID, 256, sms, st);
@@ -341,10 +350,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.rope = ws.rope; p.rope_half = dm.hd / 2; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
     return launch_tc_gemm(op, p, TC_EPI_QKV_ROPE, 256, sms, st);
   });
-  L("attention", [&] {
-    return attention_mma_supported(dm) ? launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st)
-                                       : launch_attention_simt(dm, nodes, n, Tp, ws.qkv, ws.attn, st);
-  });
+  L("attention", [&] { return launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
   L("tc_o", [&] {
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
@@ -369,7 +375,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   });
 
   // ---- memory write: [k | v] = m [Wk_mem; Wv_mem]^T for the M memory rows
-  // (rows T..T'-1 of the bf16 copy of the layer output the down GEMM wrote)
+  // (rows T..T'-1 of the fp16 copy of the layer output the down GEMM wrote)
   L("tc_kvmem", [&] {
     TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, dm.dk + dm.d, dm.L};
     op.a_pitch = Tp;
@@ -625,7 +631,8 @@ extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) 
     if (e != cudaSuccess) return;
     e = cudaMemcpy(stage, host.data(), n_elems * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
-      e = launch_convert(stage, (char*)dst_base + (size_t)l * layer_elems * as, n_elems, dm.bf16, st);
+      e = launch_convert(stage, (char*)dst_base + (size_t)l * layer_elems * as, n_elems,
+                         dm.bf16 ? CONVERT_BF16_AS_F16 : CONVERT_COPY_F32, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   };
   // rows of W scaled by the RMSNorm gain on the input dimension: (x*g) W^T = x (W diag g)^T

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <string>
@@ -14,6 +15,7 @@
 namespace armt {
 
 typedef __nv_bfloat16 bf16;
+typedef __half f16;
 
 // One node of the (segment, layer) grid as the kernels see it: x = segment s,
 // y = layer l, z = activation slot (s mod number-of-slots), w = flags.
@@ -33,26 +35,28 @@ struct Workspace {
   int slots = 0;
   int tp_max = 0;           // max rows per node (max_seg_len + n_mem)
   float* h = nullptr;       // [slots][T'][d] residual stream, fp32
-  void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (act dtype)
+  void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (fp32, or fp16 on the tensor-core path)
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
-  void* phi = nullptr;      // [slots][T'][P] DPFP features (act dtype)
+  void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or bf16 on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
-  void* qkv = nullptr;      // [slots][T'][Nqkv] (act)
-  void* attn = nullptr;     // [slots][T'][H*hd] (act)
-  void* gu = nullptr;       // [slots][T'][2F] (act)
-  void* u = nullptr;        // [slots][T'][F] (act)
+  void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
+  void* attn = nullptr;     // [slots][T'][H*hd]  (fp32 / fp16)
+  void* gu = nullptr;       // [slots][T'][2F]    (fp32 path only)
+  void* u = nullptr;        // [slots][T'][F]     (fp32 / fp16)
   float* kv = nullptr;      // [slots][M][dk + d]
   float* phik = nullptr;    // [slots][M][P]
   float* coef = nullptr;    // [slots][M] 1 / (z . phi_k + eps)
   float* gamma = nullptr;   // [slots][M]
-  void* a_act = nullptr;    // [L][d][P] act-dtype copy of A (bf16 mode)
+  void* a_act = nullptr;    // [L][d][P] bf16 copy of A (tensor-core path: the read GEMM operand)
   float2* rope = nullptr;   // [tp_max][hd/2] (cos, sin)
   NodeEntry* nodes = nullptr;
   int nodes_cap = 0;
   unsigned* err = nullptr;  // device error word (bounded waits)
 };
 
-// Device weights in the layout the grouped kernels read.
+// Device weights in the layout the grouped kernels read: fp32 on the fp32
+// path; on the tensor-core path the bf16-rounded values stored as fp16 (fp16
+// holds every bf16 value of magnitude >= 2^-17 exactly).
 struct Weights {
   bool loaded = false;
   float* mem_emb = nullptr;  // [M][d] fp32
@@ -113,12 +117,11 @@ struct GemmArgs {
   int epi;
 };
 
-// SIMT grouped GEMM; a_bf16/b_bf16/c_bf16 select operand storage types.
-cudaError_t launch_simt_gemm(const GemmArgs& a, bool a_bf16, bool b_bf16, bool c_bf16,
-                             cudaStream_t st);
+// SIMT grouped GEMM, fp32 operands (fp32 path, unit entry points).
+cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
-                                    const void* emb, const float* mem_emb, float* h, void* xb, cudaStream_t st);
+                                    const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st);
 cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h,
                            void* xb, float eps, cudaStream_t st);
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
@@ -145,7 +148,8 @@ cudaError_t setup_attention_mma();
 cudaError_t launch_attention_mma(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* qkv, void* out,
                                  cudaStream_t st);
 
-// fp32 -> act conversions used at weight load
-cudaError_t launch_convert(const float* src, void* dst, size_t n, bool to_bf16, cudaStream_t st);
+// weight conversions at load: fp32 copy, or bf16 rounding (RNE) stored as fp16
+enum ConvertMode { CONVERT_COPY_F32 = 0, CONVERT_BF16_AS_F16 = 1 };
+cudaError_t launch_convert(const float* src, void* dst, size_t n, int mode, cudaStream_t st);
 
 }  // namespace armt

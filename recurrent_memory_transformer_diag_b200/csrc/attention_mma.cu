@@ -1,5 +1,6 @@
-// Batched causal attention over the nodes of a wave, bf16 tensor cores
-// (warp-level mma.sync m16n8k16, fp32 accumulation, online softmax).
+// Batched causal attention over the nodes of a wave on tensor cores
+// (warp-level mma.sync m16n8k16, fp16 operands, fp32 accumulation, online
+// softmax).
 //
 // The wave's nodes are treated as a batch: one CTA per (q tile, query head,
 // node), every node attending only over the T' rows of its own segment plus
@@ -42,18 +43,18 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
 
 __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// element offset of (row, 16-byte chunk) in a swizzled [rows][HD] bf16 tile
+// element offset of (row, 16-byte chunk) in a swizzled [rows][HD] 16-bit tile
 template <int HD>
 __device__ __forceinline__ int swz(int row, int chunk) {
   return row * HD + ((chunk ^ (row & 7)) << 3);
@@ -61,8 +62,8 @@ __device__ __forceinline__ int swz(int row, int chunk) {
 
 template <int HD, int WARPS>
 __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEntry* nodes, int Tp, int H, int KV,
-                                                                   int nqkv, const bf16* __restrict__ qkv,
-                                                                   bf16* __restrict__ out, float scale_log2) {
+                                                                   int nqkv, const f16* __restrict__ qkv,
+                                                                   f16* __restrict__ out, float scale_log2) {
   constexpr int BM = 16 * WARPS;
   constexpr int BN = 64;
   constexpr int CH = HD / 8;            // 16-byte chunks per row
@@ -71,9 +72,9 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
   constexpr int NT = BN / 8;            // 8-wide key tiles of S
   constexpr int NTHREADS = WARPS * 32;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  bf16* sQ = reinterpret_cast<bf16*>(smem_raw);
-  bf16* sK = sQ + BM * HD;              // [2][BN][HD]
-  bf16* sV = sK + 2 * BN * HD;          // [2][BN][HD]
+  f16* sQ = reinterpret_cast<f16*>(smem_raw);
+  f16* sK = sQ + BM * HD;              // [2][BN][HD]
+  f16* sV = sK + 2 * BN * HD;          // [2][BN][HD]
 
   const NodeEntry nd = nodes[blockIdx.z];
   const int h = blockIdx.y;
@@ -81,10 +82,10 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
   const int qt = gridDim.x - 1 - blockIdx.x;      // longest rows first
   const int q0 = qt * BM;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bf16* base = qkv + (long long)nd.z * Tp * nqkv;
-  const bf16* Qg = base + h * HD;
-  const bf16* Kg = base + (H + g) * HD;
-  const bf16* Vg = base + (H + KV + g) * HD;
+  const f16* base = qkv + (long long)nd.z * Tp * nqkv;
+  const f16* Qg = base + h * HD;
+  const f16* Kg = base + (H + g) * HD;
+  const f16* Vg = base + (H + KV + g) * HD;
 
   for (int idx = tid; idx < BM * CH; idx += NTHREADS) {
     const int r = idx / CH, c = idx - r * CH;
@@ -92,8 +93,8 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
     cp_async16(sQ + swz<HD>(r, c), Qg + (long long)min(gr, Tp - 1) * nqkv + c * 8, gr < Tp);
   }
   auto load_kv = [&](int j, int buf) {
-    bf16* dk = sK + buf * BN * HD;
-    bf16* dv = sV + buf * BN * HD;
+    f16* dk = sK + buf * BN * HD;
+    f16* dv = sV + buf * BN * HD;
     for (int idx = tid; idx < BN * CH; idx += NTHREADS) {
       const int r = idx / CH, c = idx - r * CH;
       const int gr = j * BN + r;
@@ -130,8 +131,8 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
     cp_async_commit();
     const int k0 = j * BN;
     if (k0 <= warp_last) {
-      const bf16* cK = sK + (j & 1) * BN * HD;
-      const bf16* cV = sV + (j & 1) * BN * HD;
+      const f16* cK = sK + (j & 1) * BN * HD;
+      const f16* cV = sV + (j & 1) * BN * HD;
       float s[NT][4];
 #pragma unroll
       for (int i = 0; i < NT; ++i) s[i][0] = s[i][1] = s[i][2] = s[i][3] = 0.f;
@@ -194,10 +195,10 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk) {
         uint32_t a[4];
-        a[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-        a[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-        a[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-        a[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+        a[0] = pack_f16(s[2 * kk][0], s[2 * kk][1]);
+        a[1] = pack_f16(s[2 * kk][2], s[2 * kk][3]);
+        a[2] = pack_f16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+        a[3] = pack_f16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
 #pragma unroll
         for (int dp = 0; dp < DT / 2; ++dp) {
           const int key = kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
@@ -224,11 +225,11 @@ __global__ void __launch_bounds__(WARPS * 32) attention_mma_kernel(const NodeEnt
   for (int dt = 0; dt < DT; ++dt) {
     const int col = dt * 8 + 2 * (lane & 3);
     const int c = col >> 3, w = col & 7;
-    *reinterpret_cast<uint32_t*>(sQ + swz<HD>(r0, c) + w) = pack_bf16(o[dt][0] * inv0, o[dt][1] * inv0);
-    *reinterpret_cast<uint32_t*>(sQ + swz<HD>(r0 + 8, c) + w) = pack_bf16(o[dt][2] * inv1, o[dt][3] * inv1);
+    *reinterpret_cast<uint32_t*>(sQ + swz<HD>(r0, c) + w) = pack_f16(o[dt][0] * inv0, o[dt][1] * inv0);
+    *reinterpret_cast<uint32_t*>(sQ + swz<HD>(r0 + 8, c) + w) = pack_f16(o[dt][2] * inv1, o[dt][3] * inv1);
   }
   __syncwarp();
-  bf16* og = out + ((long long)nd.z * Tp) * (H * HD) + h * HD;
+  f16* og = out + ((long long)nd.z * Tp) * (H * HD) + h * HD;
   for (int idx = lane; idx < 16 * CH; idx += 32) {
     const int r = idx / CH, c = idx - r * CH;
     const int row = warp * 16 + r;
@@ -243,11 +244,11 @@ template <int HD, int WARPS>
 cudaError_t launch_hd(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* qkv, void* out,
                       cudaStream_t st) {
   constexpr int BM = 16 * WARPS;
-  const size_t smem = (size_t)(BM * HD + 4 * 64 * HD) * sizeof(bf16);
+  const size_t smem = (size_t)(BM * HD + 4 * 64 * HD) * sizeof(f16);
   dim3 grid((Tp + BM - 1) / BM, dm.H, n);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   attention_mma_kernel<HD, WARPS><<<grid, WARPS * 32, smem, st>>>(nodes, Tp, dm.H, dm.KV, dm.nqkv,
-                                                                  (const bf16*)qkv, (bf16*)out, scale_log2);
+                                                                  (const f16*)qkv, (f16*)out, scale_log2);
   return cudaGetLastError();
 }
 

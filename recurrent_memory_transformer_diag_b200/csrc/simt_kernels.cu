@@ -1,5 +1,5 @@
-// SIMT kernels of the forward: the fp32 path end to end, and the
-// element-wise / row-wise steps of the bf16 path.
+// SIMT kernels of the forward: the fp32 path end to end, and the row-wise
+// steps (layer-0 input, RMSNorm, DPFP features, output) of the tensor-core path.
 //
 // Every kernel takes the wave's node entries (segment, layer, slot) and
 // handles all nodes of the wave in one launch (blockIdx.z or blockIdx.y =
@@ -14,6 +14,8 @@ __device__ __forceinline__ float ld(const float* p, size_t i) { return p[i]; }
 __device__ __forceinline__ float ld(const bf16* p, size_t i) { return __bfloat162float(p[i]); }
 __device__ __forceinline__ void st(float* p, size_t i, float v) { p[i] = v; }
 __device__ __forceinline__ void st(bf16* p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+__device__ __forceinline__ float ld(const f16* p, size_t i) { return __half2float(p[i]); }
+__device__ __forceinline__ void st(f16* p, size_t i, float v) { p[i] = __float2half_rn(v); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -86,18 +88,10 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(GemmArgs g) {
   }
 }
 
-cudaError_t launch_simt_gemm(const GemmArgs& a, bool a_bf16, bool b_bf16, bool c_bf16, cudaStream_t st) {
+cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st) {
   if (a.n_nodes <= 0) return cudaSuccess;
   dim3 grid((a.N + 63) / 64, (a.M + 63) / 64, a.n_nodes);
-  if (a.epi == EPI_RESID || a.epi == EPI_STORE_F32) c_bf16 = false;
-#define ARMT_GEMM_CASE(TA, TB, TC) simt_gemm_kernel<TA, TB, TC><<<grid, 256, 0, st>>>(a)
-  if (!a_bf16 && !b_bf16 && !c_bf16) ARMT_GEMM_CASE(float, float, float);
-  else if (!a_bf16 && b_bf16 && !c_bf16) ARMT_GEMM_CASE(float, bf16, float);
-  else if (a_bf16 && b_bf16 && !c_bf16) ARMT_GEMM_CASE(bf16, bf16, float);
-  else if (a_bf16 && b_bf16 && c_bf16) ARMT_GEMM_CASE(bf16, bf16, bf16);
-  else if (!a_bf16 && b_bf16 && c_bf16) ARMT_GEMM_CASE(float, bf16, bf16);
-  else return cudaErrorInvalidValue;
-#undef ARMT_GEMM_CASE
+  simt_gemm_kernel<float, float, float><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
@@ -107,7 +101,7 @@ cudaError_t launch_simt_gemm(const GemmArgs& a, bool a_bf16, bool b_bf16, bool c
 // ---------------------------------------------------------------------------
 template <typename TE>
 __global__ void init_first_layer_kernel(const NodeEntry* nodes, int T, int Tp, int d,
-                                        const TE* emb, const float* mem_emb, float* h, bf16* xb) {
+                                        const TE* emb, const float* mem_emb, float* h, f16* xb) {
   const NodeEntry nd = nodes[blockIdx.y];
   if (nd.y != 0) return;
   const int t = blockIdx.x;
@@ -116,16 +110,15 @@ __global__ void init_first_layer_kernel(const NodeEntry* nodes, int T, int Tp, i
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     const float v = t < T ? ld(emb, ((long long)nd.x * T + t) * d + c) : mem_emb[(long long)(t - T) * d + c];
     dst[c] = v;
-    if (xb) xb[o + c] = __float2bfloat16_rn(v);
+    if (xb) xb[o + c] = __float2half_rn(v);
   }
 }
 
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
-                                    const void* emb, const float* mem_emb, float* h, void* xb, cudaStream_t st) {
+                                    const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st) {
   dim3 grid(Tp, n);
   if (dm.bf16)
-    init_first_layer_kernel<bf16><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const bf16*)emb, mem_emb, h,
-                                                        (bf16*)xb);
+    init_first_layer_kernel<bf16><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const bf16*)emb, mem_emb, h, xb);
   else
     init_first_layer_kernel<float><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const float*)emb, mem_emb, h,
                                                          nullptr);
@@ -154,7 +147,7 @@ __global__ void rmsnorm_kernel(const NodeEntry* nodes, int Tp, int d, const floa
 cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h,
                            void* xb, float eps, cudaStream_t st) {
   dim3 grid((Tp + 7) / 8, n);
-  if (dm.bf16) rmsnorm_kernel<bf16><<<grid, 256, 0, st>>>(nodes, Tp, dm.d, h, (bf16*)xb, eps);
+  if (dm.bf16) rmsnorm_kernel<f16><<<grid, 256, 0, st>>>(nodes, Tp, dm.d, h, (f16*)xb, eps);
   else rmsnorm_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.d, h, (float*)xb, eps);
   return cudaGetLastError();
 }
@@ -237,8 +230,8 @@ __global__ void rope_kernel(const NodeEntry* nodes, int Tp, int nheads_qk, int h
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
                         const float2* rope, cudaStream_t st) {
   dim3 grid(Tp, n);
-  if (dm.bf16) rope_kernel<bf16><<<grid, 256, 0, st>>>(nodes, Tp, dm.H + dm.KV, dm.hd, dm.nqkv, (bf16*)qkv, rope);
-  else rope_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.H + dm.KV, dm.hd, dm.nqkv, (float*)qkv, rope);
+  if (dm.bf16) return cudaErrorInvalidValue;   // the tensor-core path fuses RoPE into the QKV GEMM
+  rope_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.H + dm.KV, dm.hd, dm.nqkv, (float*)qkv, rope);
   return cudaGetLastError();
 }
 
@@ -321,8 +314,8 @@ static cudaError_t attention_dispatch(const Dims& dm, const NodeEntry* nodes, in
 
 cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
                                   const void* qkv, void* out, cudaStream_t st) {
-  return dm.bf16 ? attention_dispatch<bf16>(dm, nodes, n, Tp, qkv, out, st)
-                 : attention_dispatch<float>(dm, nodes, n, Tp, qkv, out, st);
+  if (dm.bf16) return cudaErrorInvalidValue;   // the tensor-core path has its own attention kernel
+  return attention_dispatch<float>(dm, nodes, n, Tp, qkv, out, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -345,8 +338,8 @@ __global__ void swiglu_kernel(const NodeEntry* nodes, int Tp, int F, const T* gu
 cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* gu,
                           void* u, cudaStream_t st) {
   dim3 grid(256, n);
-  if (dm.bf16) swiglu_kernel<bf16><<<grid, 256, 0, st>>>(nodes, Tp, dm.F, (const bf16*)gu, (bf16*)u);
-  else swiglu_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.F, (const float*)gu, (float*)u);
+  if (dm.bf16) return cudaErrorInvalidValue;   // fused into the gate/up GEMM on the tensor-core path
+  swiglu_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.F, (const float*)gu, (float*)u);
   return cudaGetLastError();
 }
 
@@ -372,14 +365,15 @@ cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, 
   return cudaGetLastError();
 }
 
-__global__ void convert_kernel(const float* src, bf16* dst, size_t n) {
+// fp32 -> bf16 (round to nearest even) -> fp16 container
+__global__ void convert_bf16_as_f16_kernel(const float* src, f16* dst, size_t n) {
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
-    dst[i] = __float2bfloat16_rn(src[i]);
+    dst[i] = __float2half_rn(__bfloat162float(__float2bfloat16_rn(src[i])));
 }
 
-cudaError_t launch_convert(const float* src, void* dst, size_t n, bool to_bf16, cudaStream_t st) {
-  if (!to_bf16) return cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
-  convert_kernel<<<1184, 256, 0, st>>>(src, (bf16*)dst, n);
+cudaError_t launch_convert(const float* src, void* dst, size_t n, int mode, cudaStream_t st) {
+  if (mode == CONVERT_COPY_F32) return cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
+  convert_bf16_as_f16_kernel<<<1184, 256, 0, st>>>(src, (f16*)dst, n);
   return cudaGetLastError();
 }
 

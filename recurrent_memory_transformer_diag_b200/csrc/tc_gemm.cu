@@ -9,8 +9,11 @@
 // The stacked weights are one 3-D tensor [L, N, K]; the layer index is the
 // outer TMA coordinate, so a tile of node g loads B with coordinate l(g).
 //
+// Operands are 16-bit, both fp16 or both bf16 (a runtime instruction-
+// descriptor field).
+//
 // Kernel structure (persistent, one CTA per SM, 192 threads):
-//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (bf16, 128-byte
+//   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (16-bit, 128-byte
 //               swizzle) per pipeline stage
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
 //               K=16) and commits stage/accumulator barriers
@@ -108,9 +111,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: D fp32, A/B bf16, both K-major, shape 128 x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor: D fp32, A/B both fp16 (format 0) or both bf16
+// (format 1), both K-major, shape 128 x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int n, int ab_bf16) {
+  return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
 }
 
 __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
@@ -147,7 +152,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void store_bf16x32(bf16* dst, const float* v) {
+__device__ __forceinline__ void store_f16x32(f16* dst, const float* v) {
   // 32 values = 64 bytes: four 16-byte stores (dst 16-byte aligned)
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -155,8 +160,8 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float* v) {
     uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&b2);
+      __half2 h2 = __floats2half2_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h2);
     }
     reinterpret_cast<uint4*>(dst)[q] = pk;
   }
@@ -184,13 +189,13 @@ __device__ __forceinline__ void store_f32x32(float* dst, const float* v, int val
   }
 }
 
-__device__ __forceinline__ void store_act32(bf16* dst, const float* v, int valid_cols) {
+__device__ __forceinline__ void store_act32(f16* dst, const float* v, int valid_cols) {
   if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-    store_bf16x32(dst, v);
+    store_f16x32(dst, v);
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-      if (i < valid_cols) dst[i] = __float2bfloat16_rn(v[i]);
+      if (i < valid_cols) dst[i] = __float2half_rn(v[i]);
   }
 }
 
@@ -243,7 +248,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
         resid_add32(H, v, rs, nv);
         if (EPI == TC_EPI_RESID_ACT) {
-          bf16* X = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+          f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
           store_act32(X, v, nv);
         }
       }
@@ -275,7 +280,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
             v2[i] = x2 * a.x + x1 * a.y;
           }
         }
-        bf16* C = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
+        f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
         store_act32(C + col1, v1, p.N - col1);
         if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
       }
@@ -293,7 +298,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       if (!valid || f >= p.f_out) continue;
 #pragma unroll
       for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.f + __expf(-g[i])) * u[i];
-      bf16* C = reinterpret_cast<bf16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + f;
+      f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + f;
       store_act32(C, g, p.f_out - f);
     }
   }
@@ -384,7 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t IDESC = idesc_bf16(BN);
+      const uint32_t IDESC = idesc_f16(BN, p.ab_bf16);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -503,11 +508,11 @@ cudaError_t setup_tc_gemm() {
   return e;
 }
 
-// 3-D tensor map over a bf16 array [outer][rows][inner] (inner contiguous;
+// 3-D tensor map over a 16-bit array [outer][rows][inner] (inner contiguous;
 // consecutive outer indices pitch_rows rows apart), box = box_inner x
 // box_rows x 1, 128-byte swizzle, zero fill out of bounds.
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows, int outer, int box_inner,
-                         int box_rows, int pitch_rows) {
+                         int box_rows, int pitch_rows, bool is_bf16) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
   if (!enc) return cudaErrorNotSupported;
   if (pitch_rows <= 0) pitch_rows = rows;
@@ -515,7 +520,7 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows
   cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * pitch_rows * 2};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = enc(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -531,9 +536,9 @@ int tc_pick_bn(int n) { return n >= 256 ? 256 : (n >= 128 ? 128 : 64); }
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st) {
   CUtensorMap ta, tb;
-  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM, op.a_pitch);
+  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM, op.a_pitch, p.ab_bf16 != 0);
   if (e != cudaSuccess) return e;
-  e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn, 0);
+  e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn, 0, p.ab_bf16 != 0);
   if (e != cudaSuccess) return e;
   p.m_tiles = (p.M + BM - 1) / BM;
   p.n_tiles = (p.N + bn - 1) / bn;
@@ -552,7 +557,7 @@ cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, in
 }
 
 cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
-                                const NodeEntry* nodes, float* C, unsigned* err, cudaStream_t st) {
+                                const NodeEntry* nodes, float* C, unsigned* err, int ab_bf16, cudaStream_t st) {
   int dev = 0, sms = 148;
   cudaError_t se = setup_tc_gemm();
   if (se != cudaSuccess) return se;
@@ -565,6 +570,7 @@ cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const
   p.nodes = nodes; p.n_nodes = G; p.M = m; p.N = n; p.K = k;
   p.C = C; p.c_slot_stride = (long long)m * n; p.ldc = n;
   p.err = err;
+  p.ab_bf16 = ab_bf16;
   const int bn = tc_pick_bn(n);
   return launch_tc_gemm(op, p, TC_EPI_F32, bn, sms, st);
 }

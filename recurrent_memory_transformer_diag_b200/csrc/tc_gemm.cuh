@@ -9,9 +9,9 @@ namespace armt {
 enum TcEpi {
   TC_EPI_F32 = 0,        // C (fp32) = acc
   TC_EPI_RESID = 1,      // h += acc * rowscale[row]   (rowscale optional)
-  TC_EPI_RESID_ACT = 2,  // h += acc; C (bf16) = h     (GEMM-operand copy of the new residual)
-  TC_EPI_QKV_ROPE = 3,   // C (bf16) = acc, rotate-half RoPE on heads < rope_heads
-  TC_EPI_SWIGLU = 4      // C (bf16)[f] = silu(acc[gate f]) * acc[up f]; B rows interleaved per 128
+  TC_EPI_RESID_ACT = 2,  // h += acc; C (fp16) = h     (GEMM-operand copy of the new residual)
+  TC_EPI_QKV_ROPE = 3,   // C (fp16) = acc, rotate-half RoPE on heads < rope_heads
+  TC_EPI_SWIGLU = 4      // C (fp16)[f] = silu(acc[gate f]) * acc[up f]; B rows interleaved per 128
 };
 
 struct TcGemmParams {
@@ -20,6 +20,7 @@ struct TcGemmParams {
   int M, N, K;              // per node: rows, B rows (output columns), reduction
   int m_tiles, n_tiles, k_blocks;
   int a_by_layer;           // A's outer TMA coordinate: 0 = node slot, 1 = node layer
+  int ab_bf16;              // operand type: 0 = fp16, 1 = bf16 (both operands alike)
   void* C; long long c_slot_stride; int ldc;
   float* h; long long h_slot_stride; int ldh;
   const float* rowscale; long long rs_slot_stride;
@@ -29,8 +30,8 @@ struct TcGemmParams {
 };
 
 struct TcGemmOperands {
-  const void* A; int a_rows; int a_outer;   // bf16 [a_outer][a_rows][K] (rows a_pitch apart per outer step)
-  const void* B; int b_rows; int b_outer;   // bf16 [b_outer][b_rows][K]
+  const void* A; int a_rows; int a_outer;   // 16-bit [a_outer][a_rows][K] (rows a_pitch apart per outer step)
+  const void* B; int b_rows; int b_outer;   // 16-bit [b_outer][b_rows][K]
   int a_pitch = 0;                          // rows between outer steps of A (0 = a_rows)
 };
 
@@ -40,6 +41,6 @@ bool tc_gemm_supported(int m, int n, int k);
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st);
 cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
-                                const NodeEntry* nodes, float* C, unsigned* err, cudaStream_t st);
+                                const NodeEntry* nodes, float* C, unsigned* err, int ab_bf16, cudaStream_t st);
 
 }  // namespace armt

@@ -21,13 +21,13 @@ armt_status to_status(cudaError_t e) {
 extern "C" armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, int k, const void* A,
                                          const void* B, int num_b, const int* bidx, float* C, void* stream) {
   if (G < 1 || m < 1 || n < 1 || k < 1 || num_b < 1 || !A || !B || !bidx || !C) return ARMT_ERR_INVALID_ARG;
-  if (dtype != ARMT_FP32 && dtype != ARMT_BF16) return ARMT_ERR_INVALID_ARG;
+  if (dtype != ARMT_FP32 && dtype != ARMT_BF16 && dtype != ARMT_F16) return ARMT_ERR_INVALID_ARG;
   std::vector<NodeEntry> tab(G);
   for (int g = 0; g < G; ++g) {
     if (bidx[g] < 0 || bidx[g] >= num_b) return ARMT_ERR_INVALID_ARG;
     tab[g] = make_int4(g, bidx[g], g, 0);
   }
-  if (dtype == ARMT_BF16 && !tc_gemm_supported(m, n, k)) return ARMT_ERR_UNSUPPORTED;
+  if (dtype != ARMT_FP32 && !tc_gemm_supported(m, n, k)) return ARMT_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   NodeEntry* dnodes = nullptr;
   cudaError_t e = cudaMallocAsync((void**)&dnodes, G * sizeof(NodeEntry) + 16, st);
@@ -37,8 +37,8 @@ extern "C" armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, 
   e = cudaMemcpyAsync(dnodes, tab.data(), G * sizeof(NodeEntry), cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemsetAsync(derr, 0, sizeof(unsigned), st);
   if (e == cudaSuccess) {
-    if (dtype == ARMT_BF16) {
-      e = launch_tc_gemm_unit(G, m, n, k, A, B, num_b, dnodes, C, derr, st);
+    if (dtype != ARMT_FP32) {
+      e = launch_tc_gemm_unit(G, m, n, k, A, B, num_b, dnodes, C, derr, dtype == ARMT_BF16 ? 1 : 0, st);
     } else {
       GemmArgs g{};
       g.nodes = dnodes; g.n_nodes = G; g.M = m; g.N = n; g.K = k;
@@ -46,7 +46,7 @@ extern "C" armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, 
       g.B = B; g.b_layer_stride = (long long)n * k; g.ldb = k;
       g.C = C; g.c_slot_stride = (long long)m * n; g.ldc = n;
       g.epi = EPI_STORE_F32;
-      e = launch_simt_gemm(g, false, false, false, st);
+      e = launch_simt_gemm(g, st);
     }
   }
   if (e == cudaSuccess) e = cudaMemcpyAsync(&herr, derr, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
@@ -92,7 +92,7 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
     g.B = w_kv; g.b_layer_stride = 0; g.ldb = d;
     g.C = kv; g.c_slot_stride = 0; g.ldc = d_key + d;
     g.epi = EPI_STORE_F32;
-    e = launch_simt_gemm(g, false, false, false, st);
+    e = launch_simt_gemm(g, st);
   }
   if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, coef, gamma, st);
   if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, coef, A, nullptr, st);

@@ -9,6 +9,7 @@ from .gpu_util import rel_l2
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("G,m,n,k,num_b", [
     (1, 128, 256, 64, 1),       # one tile, one k block
     (3, 1040, 512, 2048, 5),    # ragged M (8 full tiles + 16 rows), many k blocks
@@ -17,12 +18,13 @@ pytestmark = pytest.mark.gpu
     (2, 77, 128, 136, 3),       # N = 128, tiny ragged M and K
     (16, 1040, 3072, 2048, 16), # a full 1B wave of QKV shapes
 ])
-def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b):
+def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b, dtype):
     import torch
     from recurrent_memory_transformer_diag_b200 import grouped_gemm
     g = torch.Generator().manual_seed(G * 1000 + m + n + k)
-    A = torch.randn(G, m, k, generator=g).to(torch.bfloat16)
-    B = (torch.randn(num_b, n, k, generator=g) * 0.05).to(torch.bfloat16)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    A = torch.randn(G, m, k, generator=g).to(tdt)
+    B = (torch.randn(num_b, n, k, generator=g) * 0.05).to(tdt)
     bidx = [(3 * i + 1) % num_b for i in range(G)]
     C = torch.full((G, m, n), float("nan"), device="cuda")
     grouped_gemm(A.cuda(), B.cuda(), bidx, C)
