@@ -25,6 +25,8 @@ def _compare(cfg, got, ref, tol):
     for l in range(cfg.n_layers):
         errs[f"A[{l}]"] = rel_l2(A[l], Ar[l])
         errs[f"z[{l}]"] = rel_l2(z[l], zr[l])
+    worst = max(errs, key=errs.get)
+    print(f"\n{cfg.name}: rel-L2 hidden {errs['hidden']:.3e}, worst {worst} {errs[worst]:.3e} (tol {tol})")
     bad = {k: v for k, v in errs.items() if not v <= tol}
     assert not bad, f"rel-L2 above {tol}: {bad}"
     return errs

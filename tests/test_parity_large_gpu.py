@@ -30,6 +30,8 @@ def _prefix_parity(name, S=2):
     for l in range(cfg.n_layers):
         errs[f"A[{l}]"] = rel_l2(got[1][l], ref[1][l])
         errs[f"z[{l}]"] = rel_l2(got[2][l], ref[2][l])
+    worst = max(errs, key=errs.get)
+    print(f"\n{name} S={S}: rel-L2 hidden {errs['hidden']:.3e}, worst {worst} {errs[worst]:.3e}")
     bad = {k: v for k, v in errs.items() if not v <= 1e-2}
     assert not bad, bad
     return cfg, w, got
