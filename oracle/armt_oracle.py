@@ -37,12 +37,21 @@ both cited in the Pith review's reference list):
    positions 0..T'-1, restarting every segment), causal softmax attention
    over the T' rows of this node only, scale 1/sqrt(hd), query head h using
    kv head floor(h * KV / H), and MLP = (silu(x Wg^T) * (x Wu^T)) Wd^T.
-4. Memory write, after the layer, from m = rows T..T'-1 of the layer output:
-   k = m Wk_mem^T, v = m Wv_mem^T, phi_j = DPFP(k_j);
-   vbar_j = A phi_j / (z . phi_j + eps);
-   gamma_j = clamp(1 - (z . phi_j) / (|phi_j|^2 + eps), 0, 1);
-   A <- A + sum_j (v_j - vbar_j) phi_j^T;  z <- z + sum_j gamma_j phi_j,
-   every j using the state before this write.
+4. Memory write, after the layer, from the M memory rows of the layer
+   output (rows T..T'-1), each RMS-normalised without gain (m = RMSNorm(row)):
+   k = m Wk_mem^T, v = m Wv_mem^T, phi_j = DPFP(k_j), and the delta rule
+   applied to the rows one after another (j = 0..M-1), each seeing the state
+   the previous rows left:
+     vbar_j  = A phi_j / (z . phi_j + eps)
+     gamma_j = clamp(1 - (z . phi_j) / (|phi_j|^2 + eps), 0, 1)
+     A <- A + (v_j - vbar_j) phi_j^T;   z <- z + gamma_j phi_j
+   The memory is updated once per segment (after the segment's layer), the
+   M rows in order: the delta rule is a sequential recurrence (ref. 38
+   parallelises exactly that recurrence).  Applying all M rows to the
+   pre-write state at once, or writing un-normalised rows, makes this
+   random-init model diverge geometrically over the segments (fp64: hidden
+   RMS x2 and |A| x10 per segment at the 1B shape), so no finite-precision
+   forward over 128 segments could be compared with it.
 5. DPFP_nu(x): r = [relu(x); relu(-x)] (length 2 d_k);
    phi[(n-1) 2 d_k + j] = r_j * r_{(j-n) mod 2 d_k}, n = 1..nu  (P = 2 d_k nu).
 6. Output: rows 0..T-1 of node (s, L-1) are the final hidden states of
@@ -121,14 +130,20 @@ def mem_read(x: np.ndarray, wq_mem: np.ndarray, A: np.ndarray, z: np.ndarray,
 
 def mem_write(m: np.ndarray, wk_mem: np.ndarray, wv_mem: np.ndarray, A: np.ndarray,
               z: np.ndarray, nu: int, eps: float) -> Tuple[np.ndarray, np.ndarray]:
-    """Delta-rule update of (A, z) from memory rows m [M, d]; returns new (A, z)."""
+    """Delta-rule update of (A, z) from memory rows m [M, d], row after row;
+    returns the new (A, z)."""
     k = m @ wk_mem.T                              # [M, dk]
     v = m @ wv_mem.T                              # [M, d]
     phi = dpfp(k, nu)                             # [M, P]
-    zphi = phi @ z                                # [M]
-    vbar = (phi @ A.T) / (zphi + eps)[:, None]    # [M, d]
-    gamma = np.clip(1.0 - zphi / (np.sum(phi * phi, axis=-1) + eps), 0.0, 1.0)
-    return A + (v - vbar).T @ phi, z + gamma @ phi
+    A = A.copy()
+    z = z.copy()
+    for j in range(m.shape[0]):
+        zphi = phi[j] @ z
+        vbar = (A @ phi[j]) / (zphi + eps)
+        gamma = min(max(1.0 - zphi / (phi[j] @ phi[j] + eps), 0.0), 1.0)
+        A += np.outer(v[j] - vbar, phi[j])
+        z += gamma * phi[j]
+    return A, z
 
 
 def decoder_layer(x: np.ndarray, w: Dict[str, np.ndarray], l: int, cfg) -> np.ndarray:
@@ -158,8 +173,8 @@ def node_forward(x: np.ndarray, w: Dict[str, np.ndarray], l: int, A: np.ndarray,
         x = x + mem_read(x, w["wq_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
     x = decoder_layer(x, w, l, cfg)
     if memory:
-        A, z = mem_write(x[cfg.seg_len:], w["wk_mem"][l], w["wv_mem"][l], A, z,
-                         cfg.dpfp_nu, cfg.mem_eps)
+        m = rms_norm(x[cfg.seg_len:], np.ones(x.shape[1]), cfg.rms_eps)
+        A, z = mem_write(m, w["wk_mem"][l], w["wv_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
     return x, A, z
 
 

@@ -6,7 +6,8 @@ each step differently: RoPE as complex multiplication, attention as explicit
 per-query loops, DPFP with explicit index arithmetic, the delta rule one
 scalar at a time.  The readings it follows are the same ones the oracle
 states (pre-norm LLaMA layer; ARMT read before and delta-rule write after the
-layer; memory tokens appended to every segment).
+layer, the write taking the RMS-normalised memory rows one after another;
+memory tokens appended to every segment).
 """
 import cmath
 import math
@@ -116,18 +117,16 @@ def forward(cfg, weights, emb, memory=True):
                         x[t][i] += sum(A[l][i][p] * phi[p] for p in range(P)) / den
             x = _layer(x, W, l, cfg)
             if memory:
-                mem = x[T:T + M]
+                mem = _rmsnorm(x[T:T + M], [1.0] * d, cfg.rms_eps)
                 kk = _linear(mem, W["wk_mem"][l])
                 vv = _linear(mem, W["wv_mem"][l])
-                A_old = [row[:] for row in A[l]]
-                z_old = z[l][:]
-                for j in range(M):
+                for j in range(M):              # one memory row after another
                     phi = _dpfp(kk[j], cfg.dpfp_nu)
-                    zphi = sum(z_old[p] * phi[p] for p in range(P))
+                    zphi = sum(z[l][p] * phi[p] for p in range(P))
                     nrm = sum(p * p for p in phi)
                     gamma = min(max(1.0 - zphi / (nrm + eps), 0.0), 1.0)
                     for i in range(d):
-                        vbar = sum(A_old[i][p] * phi[p] for p in range(P)) / (zphi + eps)
+                        vbar = sum(A[l][i][p] * phi[p] for p in range(P)) / (zphi + eps)
                         for p in range(P):
                             A[l][i][p] += (vv[j][i] - vbar) * phi[p]
                     for p in range(P):

@@ -110,27 +110,47 @@ def test_rewrite_same_key_replaces_value():
     np.testing.assert_allclose(r[0], wv2 @ k[0], rtol=1e-4)
 
 
-def test_batched_write_uses_pre_update_state():
-    """Two rows with the same key in ONE write both see A=0, z=0, so the update
-    is doubled (a one-at-a-time write would store the value only once)."""
+def test_write_rows_apply_one_after_another():
+    """The same key twice in one write: the second row sees the first row's
+    state (vbar = v |phi|^2/(|phi|^2+eps), gamma = eps/(|phi|^2+eps)), so the
+    value is stored once, not twice (closed form below)."""
     dk, nu, eps = 2, 2, 1e-5
     k = np.array([[0.3, -0.9], [0.3, -0.9]])
     P = 2 * dk * nu
     A, z = oracle.mem_write(k, np.eye(dk), np.eye(dk), np.zeros((dk, P)), np.zeros(P), nu, eps)
     phi = oracle.dpfp(k[0], nu)
-    np.testing.assert_allclose(A, 2 * np.outer(k[0], phi), rtol=1e-14)
-    np.testing.assert_allclose(z, 2 * phi, rtol=1e-14)
+    n2 = phi @ phi
+    c = n2 / (n2 + eps)
+    np.testing.assert_allclose(A, (2.0 - c) * np.outer(k[0], phi), rtol=1e-13)
+    np.testing.assert_allclose(z, (1.0 + eps / (n2 + eps)) * phi, rtol=1e-13)
+
+
+def test_one_write_of_two_rows_equals_two_writes():
+    """Sequential reading: writing rows [m1, m2] at once equals writing m1,
+    then m2 (the same operations in the same order, up to the matrix
+    products' summation order)."""
+    rng = np.random.default_rng(11)
+    d, dk, nu, eps = 6, 3, 2, 1e-5
+    P = 2 * dk * nu
+    m = rng.standard_normal((2, d))
+    wk, wv = rng.standard_normal((dk, d)), rng.standard_normal((d, d))
+    A0, z0 = rng.standard_normal((d, P)) * 0.1, np.abs(rng.standard_normal(P))
+    A, z = oracle.mem_write(m, wk, wv, A0, z0, nu, eps)
+    A1, z1 = oracle.mem_write(m[:1], wk, wv, A0, z0, nu, eps)
+    A2, z2 = oracle.mem_write(m[1:], wk, wv, A1, z1, nu, eps)
+    np.testing.assert_allclose(A, A2, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(z, z2, rtol=1e-12, atol=1e-14)
 
 
 def test_gamma_clamped_at_zero():
-    """After z = 2 phi, a third write of the same key has 1 - z.phi/|phi|^2 ~ -1:
-    clamped to 0, z stays as it was."""
+    """With z = 2 phi(k) already, writing k gives 1 - z.phi/|phi|^2 ~ -1:
+    gamma is clamped to 0 and z stays as it was."""
     dk, nu, eps = 2, 2, 1e-5
-    k = np.array([[0.3, -0.9], [0.3, -0.9]])
+    k = np.array([[0.3, -0.9]])
     P = 2 * dk * nu
-    A, z = oracle.mem_write(k, np.eye(dk), np.eye(dk), np.zeros((dk, P)), np.zeros(P), nu, eps)
-    _, z3 = oracle.mem_write(k[:1], np.eye(dk), np.eye(dk), A, z, nu, eps)
-    np.testing.assert_array_equal(z3, z)
+    z0 = 2 * oracle.dpfp(k[0], nu)
+    _, z = oracle.mem_write(k, np.eye(dk), np.eye(dk), np.zeros((dk, P)), z0, nu, eps)
+    np.testing.assert_array_equal(z, z0)
 
 
 def test_orthogonal_keys_retrieved_independently():
@@ -363,8 +383,8 @@ def test_planted_write_rows_are_caught(monkeypatch):
             x = x + ao.mem_read(x, w["wq_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
         x = ao.decoder_layer(x, w, l, cfg)
         if memory:   # wrong rows: the first M instead of the memory tokens
-            A, z = ao.mem_write(x[:cfg.n_mem], w["wk_mem"][l], w["wv_mem"][l], A, z,
-                                cfg.dpfp_nu, cfg.mem_eps)
+            m = ao.rms_norm(x[:cfg.n_mem], np.ones(x.shape[1]), cfg.rms_eps)
+            A, z = ao.mem_write(m, w["wk_mem"][l], w["wv_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
         return x, A, z
     monkeypatch.setattr(ao, "node_forward", bad_node)
     assert _fails(test_oracle_matches_pure_python_bruteforce)
@@ -387,9 +407,39 @@ def test_planted_gamma_sign_is_caught(monkeypatch):
         k = m @ wk.T
         v = m @ wv.T
         phi = ao.dpfp(k, nu)
-        zphi = phi @ z
-        vbar = (phi @ A.T) / (zphi + eps)[:, None]
-        gamma = np.clip(1.0 + zphi / (np.sum(phi * phi, axis=-1) + eps), 0.0, 1.0)
-        return A + (v - vbar).T @ phi, z + gamma @ phi
+        A, z = A.copy(), z.copy()
+        for j in range(m.shape[0]):
+            zphi = phi[j] @ z
+            vbar = (A @ phi[j]) / (zphi + eps)
+            gamma = min(max(1.0 + zphi / (phi[j] @ phi[j] + eps), 0.0), 1.0)
+            A += np.outer(v[j] - vbar, phi[j])
+            z += gamma * phi[j]
+        return A, z
     _run_pins(monkeypatch, "mem_write", bad_write)
     assert _fails(test_rewrite_same_key_replaces_value)
+
+
+def test_planted_batched_write_is_caught(monkeypatch):
+    def batched_write(m, wk, wv, A, z, nu, eps):
+        k = m @ wk.T
+        v = m @ wv.T
+        phi = ao.dpfp(k, nu)
+        zphi = phi @ z
+        vbar = (phi @ A.T) / (zphi + eps)[:, None]
+        gamma = np.clip(1.0 - zphi / (np.sum(phi * phi, axis=-1) + eps), 0.0, 1.0)
+        return A + (v - vbar).T @ phi, z + gamma @ phi
+    _run_pins(monkeypatch, "mem_write", batched_write)
+    assert _fails(test_write_rows_apply_one_after_another)
+    assert _fails(test_oracle_matches_pure_python_bruteforce)
+
+
+def test_planted_missing_write_norm_is_caught(monkeypatch):
+    def node_no_norm(x, w, l, A, z, cfg, memory=True):
+        if memory:
+            x = x + ao.mem_read(x, w["wq_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
+        x = ao.decoder_layer(x, w, l, cfg)
+        if memory:
+            A, z = ao.mem_write(x[cfg.seg_len:], w["wk_mem"][l], w["wv_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
+        return x, A, z
+    monkeypatch.setattr(ao, "node_forward", node_no_norm)
+    assert _fails(test_oracle_matches_pure_python_bruteforce)
