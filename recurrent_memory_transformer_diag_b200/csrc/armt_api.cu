@@ -70,7 +70,7 @@ void free_weights(Weights& w) {
 void free_workspace(Workspace& ws) {
   dfree(ws.h); dfree(ws.xb); dfree(ws.qm); dfree(ws.phi); dfree(ws.inv_den); dfree(ws.qkv);
   dfree(ws.attn); dfree(ws.gu); dfree(ws.u); dfree(ws.kv); dfree(ws.phik); dfree(ws.coef);
-  dfree(ws.gamma); dfree(ws.a_act); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err);
+  dfree(ws.gamma); dfree(ws.a_act); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err); dfree(ws.rsq); dfree(ws.gram);
   ws = Workspace();
 }
 
@@ -97,7 +97,7 @@ armt_status validate_config(const armt_config* c, const char** why) {
   const long long P = 2LL * c->d_key * c->dpfp_nu;
   if (P > 1024) { *why = "phi dimension 2*d_key*nu must be <= 1024"; return ARMT_ERR_UNSUPPORTED; }
   if (c->n_mem > 64) { *why = "n_mem must be <= 64"; return ARMT_ERR_UNSUPPORTED; }
-  if ((long long)c->n_mem * P * 4 + 9LL * c->n_mem * 4 > 200 * 1024) {
+  if (((long long)c->n_mem * P + (long long)c->n_mem * c->n_mem + 9LL * c->n_mem) * 4 > 200 * 1024) {
     *why = "n_mem * phi dimension too large for the write kernel"; return ARMT_ERR_UNSUPPORTED;
   }
   if (c->dtype == ARMT_BF16 && (c->d_model % 8 || c->d_ffn % 8 || (c->n_heads * c->head_dim) % 8 || P % 8)) {
@@ -149,7 +149,8 @@ void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeE
 const char* const KIND_NAMES[] = {
     "init", "gemm_qmem", "tc_qmem", "dpfp_read", "gemm_read", "tc_read", "norm_attn", "gemm_qkv",
     "rope", "tc_qkv_rope", "attention", "gemm_o", "tc_o", "norm_mlp", "gemm_gateup", "swiglu",
-    "tc_gateup_swiglu", "gemm_down", "tc_down", "gemm_kvmem", "tc_kvmem", "memw_phi", "memw_update", "output"};
+    "tc_gateup_swiglu", "gemm_down", "tc_down", "norm_mem", "gemm_kvmem", "tc_kvmem", "memw_phi", "memw_update",
+    "output"};
 constexpr int N_KINDS = (int)(sizeof(KIND_NAMES) / sizeof(KIND_NAMES[0]));
 
 int kind_index(const char* name) {
@@ -232,7 +233,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   }
 
   // ---- attention block
-  L("norm_attn", [&] { return launch_rmsnorm(dm, nodes, n, Tp, ws.h, ws.xb, dm.rms_eps, st); });
+  L("norm_attn", [&] { return launch_rmsnorm(dm, nodes, n, Tp, 0, Tp, ws.h, ws.xb, dm.rms_eps, st); });
   {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = Tp; g.N = dm.nqkv; g.K = dm.d;
@@ -255,7 +256,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   }
 
   // ---- MLP block
-  L("norm_mlp", [&] { return launch_rmsnorm(dm, nodes, n, Tp, ws.h, ws.xb, dm.rms_eps, st); });
+  L("norm_mlp", [&] { return launch_rmsnorm(dm, nodes, n, Tp, 0, Tp, ws.h, ws.xb, dm.rms_eps, st); });
   {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = Tp; g.N = 2 * dm.F; g.K = dm.d;
@@ -276,19 +277,20 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     L("gemm_down", [&] { return launch_simt_gemm(g, st); });
   }
 
-  // ---- memory write from the M memory rows of the layer output
+  // ---- memory write from the RMS-normalised M memory rows of the layer output
+  L("norm_mem", [&] { return launch_rmsnorm(dm, nodes, n, Tp, T, dm.M, ws.h, ws.xb, dm.rms_eps, st); });
   {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = dm.M; g.N = dm.dk + dm.d; g.K = dm.d;
-    g.A = ws.h + (long long)T * dm.d; g.a_slot_stride = hs; g.lda = dm.d;
+    g.A = (const float*)ws.xb + (long long)T * dm.d; g.a_slot_stride = hs; g.lda = dm.d;
     g.B = w.w_kvm; g.b_layer_stride = (long long)(dm.dk + dm.d) * dm.d; g.ldb = dm.d;
     g.C = ws.kv; g.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); g.ldc = dm.dk + dm.d;
     g.epi = EPI_STORE_F32;
     L("gemm_kvmem", [&] { return launch_simt_gemm(g, st); });
   }
-  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.coef, ws.gamma, st); });
+  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.coef, A, nullptr, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, nullptr, st);
   });
 
   if (wv.any_last_layer)
@@ -319,6 +321,12 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   auto base = [&](TcGemmParams& p, int M, int N, int K) {
     p = TcGemmParams{};
     p.nodes = nodes; p.n_nodes = n; p.M = M; p.N = N; p.K = K; p.err = ws.err;
+    p.out_layer = -1;
+  };
+  const int rsq_parts = (dm.d + 255) / 256;
+  auto norm_partials = [&](TcGemmParams& p) {
+    p.rsq = ws.rsq; p.rsq_slot_stride = (long long)Tp * rsq_parts; p.rsq_parts = rsq_parts;
+    p.norm_dim = dm.d; p.norm_eps = dm.rms_eps;
   };
 
   if (wv.any_first_layer)
@@ -333,21 +341,24 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   });
   L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
   L("tc_read", [&] {
+    // h += phi A^T / (z.phi + eps); new h -> fp16 operand copy + norm partials
     TcGemmOperands op{ws.phi, Tp, slots, ws.a_act, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.P);
     p.ab_bf16 = 1;
     p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
     p.rowscale = ws.inv_den; p.rs_slot_stride = Tp;
-    return launch_tc_gemm(op, p, TC_EPI_RESID, 256, sms, st);
+    p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
+    norm_partials(p);
+    return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
 
-  // ---- attention block
-  L("norm_attn", [&] { return launch_rmsnorm(dm, nodes, n, Tp, ws.h, ws.xb, dm.rms_eps, st); });
+  // ---- attention block (RMSNorm folded: row scale applied in the QKV epilogue)
   L("tc_qkv_rope", [&] {
     TcGemmOperands op{ws.xb, Tp, slots, w.w_qkv, dm.nqkv, dm.L};
     TcGemmParams p; base(p, Tp, dm.nqkv, dm.d);
     p.C = ws.qkv; p.c_slot_stride = (long long)Tp * dm.nqkv; p.ldc = dm.nqkv;
     p.rope = ws.rope; p.rope_half = dm.hd / 2; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
+    norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_QKV_ROPE, 256, sms, st);
   });
   L("attention", [&] { return launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
@@ -355,39 +366,48 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
     p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
-    return launch_tc_gemm(op, p, TC_EPI_RESID, 256, sms, st);
+    p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
+    norm_partials(p);
+    return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
 
-  // ---- MLP block
-  L("norm_mlp", [&] { return launch_rmsnorm(dm, nodes, n, Tp, ws.h, ws.xb, dm.rms_eps, st); });
+  // ---- MLP block (RMSNorm folded into the gate/up epilogue)
   L("tc_gateup_swiglu", [&] {
     TcGemmOperands op{ws.xb, Tp, slots, w.w_gu, 2 * f_pad, dm.L};
     TcGemmParams p; base(p, Tp, 2 * f_pad, dm.d);
     p.C = ws.u; p.c_slot_stride = (long long)Tp * dm.F; p.ldc = dm.F; p.f_out = dm.F;
+    norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_SWIGLU, 256, sms, st);
   });
   L("tc_down", [&] {
+    // h += u W_d^T; new h -> fp16 copy (next layer's memory-read query and
+    // this node's memory-write rows); last layer: rows < T -> out_hidden
     TcGemmOperands op{ws.u, Tp, slots, w.w_down, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.F);
     p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
+    p.out = out; p.out_layer = dm.L - 1; p.seg_len = T;
+    norm_partials(p);   // for the memory-write rows
     return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
 
-  // ---- memory write: [k | v] = m [Wk_mem; Wv_mem]^T for the M memory rows
-  // (rows T..T'-1 of the fp16 copy of the layer output the down GEMM wrote)
+  // ---- memory write: [k | v] = RMSNorm(m) [Wk_mem; Wv_mem]^T for the M memory
+  // rows (rows T..T'-1 of the fp16 copy of the layer output the down GEMM
+  // wrote; the RMS row scale comes from the down GEMM's partial sums)
   L("tc_kvmem", [&] {
     TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, dm.dk + dm.d, dm.L};
     op.a_pitch = Tp;
     TcGemmParams p; base(p, dm.M, dm.dk + dm.d, dm.d);
     p.C = ws.kv; p.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); p.ldc = dm.dk + dm.d;
+    norm_partials(p);
+    p.rsq_row0 = T;
     return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, st);
   });
-  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.coef, ws.gamma, st); });
-  L("memw_update", [&] { return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.coef, A, ws.a_act, st); });
+  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
+  L("memw_update", [&] {
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, ws.a_act, st);
+  });
 
-  if (wv.any_last_layer)
-    L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
 }
 
 armt_status ensure_table(armt_ctx* ctx, int S, cudaStream_t st) {
@@ -532,6 +552,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   A(&ws.qm, rows * dm.dk * 4);
   A(&ws.phi, rows * dm.P * as);
   A(&ws.inv_den, rows * 4);
+  if (dm.bf16) A(&ws.rsq, rows * ((dm.d + 255) / 256) * 4);
   A(&ws.qkv, rows * dm.nqkv * as);
   A(&ws.attn, rows * dm.H * dm.hd * as);
   if (!dm.bf16) A(&ws.gu, rows * 2 * dm.F * as);
@@ -539,6 +560,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   A(&ws.kv, (size_t)ws.slots * dm.M * (dm.dk + dm.d) * 4);
   A(&ws.phik, (size_t)ws.slots * dm.M * dm.P * 4);
   A(&ws.coef, (size_t)ws.slots * dm.M * 4);
+  A(&ws.gram, (size_t)ws.slots * dm.M * dm.M * 4);
   A(&ws.gamma, (size_t)ws.slots * dm.M * 4);
   if (dm.bf16) A(&ws.a_act, (size_t)dm.L * dm.d * dm.P * as);
   A(&ws.rope, (size_t)ws.tp_max * (dm.hd / 2) * sizeof(float2));

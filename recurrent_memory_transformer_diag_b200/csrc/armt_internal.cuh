@@ -39,13 +39,15 @@ struct Workspace {
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
   void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or bf16 on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
+  float* rsq = nullptr;     // [slots][T'][ceil(d/256)] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
   void* attn = nullptr;     // [slots][T'][H*hd]  (fp32 / fp16)
   void* gu = nullptr;       // [slots][T'][2F]    (fp32 path only)
   void* u = nullptr;        // [slots][T'][F]     (fp32 / fp16)
   float* kv = nullptr;      // [slots][M][dk + d]
   float* phik = nullptr;    // [slots][M][P]
-  float* coef = nullptr;    // [slots][M] 1 / (z . phi_k + eps)
+  float* gram = nullptr;    // [slots][M][M] phi_j . phi_j'
+  float* coef = nullptr;    // [slots][M] 1 / (z_j . phi_j + eps)
   float* gamma = nullptr;   // [slots][M]
   void* a_act = nullptr;    // [L][d][P] bf16 copy of A (tensor-core path: the read GEMM operand)
   float2* rope = nullptr;   // [tp_max][hd/2] (cos, sin)
@@ -122,8 +124,9 @@ cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                                     const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st);
-cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h,
-                           void* xb, float eps, cudaStream_t st);
+// RMSNorm (no gain) of rows row0 .. row0+nrows-1 of every node's slot.
+cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int row0, int nrows,
+                           const float* h, void* xb, float eps, cudaStream_t st);
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
                              const float* z_state, void* phi, float* inv_den, cudaStream_t st);
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
@@ -133,10 +136,11 @@ cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n,
 cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* gu,
                           void* u, cudaStream_t st);
 cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                            float* z_state, float* phik, float* coef, float* gamma, cudaStream_t st);
+                            float* z_state, float* phik, float* gram, float* coef, float* gamma,
+                            cudaStream_t st);
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                               const float* phik, const float* coef, float* A_state, void* a_act,
-                               cudaStream_t st);
+                               const float* phik, const float* gram, const float* coef, float* A_state,
+                               void* a_act, cudaStream_t st);
 cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                           const float* h, void* out, cudaStream_t st);
 

@@ -130,11 +130,13 @@ cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int 
 // One warp per row.
 // ---------------------------------------------------------------------------
 template <typename TX>
-__global__ void rmsnorm_kernel(const NodeEntry* nodes, int Tp, int d, const float* h, TX* xb, float eps) {
+__global__ void rmsnorm_kernel(const NodeEntry* nodes, int Tp, int row0, int nrows, int d, const float* h, TX* xb,
+                               float eps) {
   const NodeEntry nd = nodes[blockIdx.y];
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int rr = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= Tp) return;
+  if (rr >= nrows) return;
+  const int row = row0 + rr;
   const long long off = ((long long)nd.z * Tp + row) * d;
   const float* src = h + off;
   float ss = 0.f;
@@ -144,11 +146,11 @@ __global__ void rmsnorm_kernel(const NodeEntry* nodes, int Tp, int d, const floa
   for (int c = lane; c < d; c += 32) st(xb, off + c, src[c] * r);
 }
 
-cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h,
-                           void* xb, float eps, cudaStream_t st) {
-  dim3 grid((Tp + 7) / 8, n);
-  if (dm.bf16) rmsnorm_kernel<f16><<<grid, 256, 0, st>>>(nodes, Tp, dm.d, h, (f16*)xb, eps);
-  else rmsnorm_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.d, h, (float*)xb, eps);
+cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int row0, int nrows,
+                           const float* h, void* xb, float eps, cudaStream_t st) {
+  dim3 grid((nrows + 7) / 8, n);
+  if (dm.bf16) rmsnorm_kernel<f16><<<grid, 256, 0, st>>>(nodes, Tp, row0, nrows, dm.d, h, (f16*)xb, eps);
+  else rmsnorm_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, row0, nrows, dm.d, h, (float*)xb, eps);
   return cudaGetLastError();
 }
 

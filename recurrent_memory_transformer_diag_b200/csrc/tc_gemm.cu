@@ -199,6 +199,26 @@ __device__ __forceinline__ void store_act32(f16* dst, const float* v, int valid_
   }
 }
 
+__device__ __forceinline__ void store_bf16_32(bf16* dst, const float* v, int valid_cols) {
+  if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint4 pk;
+      uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      reinterpret_cast<uint4*>(dst)[q] = pk;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < valid_cols) dst[i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
 // h += v * rs on 32 columns; v receives the new residual values.
 __device__ __forceinline__ void resid_add32(float* H, float* v, float rs, int valid_cols) {
   if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) {
@@ -227,13 +247,25 @@ __device__ __forceinline__ void resid_add32(float* H, float* v, float rs, int va
 // Epilogue of one accumulator tile for this thread's row.  Every tcgen05.ld
 // is executed by the whole warp (warp-uniform loops); only the stores are
 // guarded by the row/column bounds.
+// RMSNorm row scale from the per-tile partial sums of squares.
+__device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot, int row) {
+  const float* part = p.rsq + (long long)slot * p.rsq_slot_stride + (long long)row * p.rsq_parts;
+  float ss = 0.f;
+  for (int i = 0; i < p.rsq_parts; ++i) ss += part[i];
+  return rsqrtf(ss / (float)p.norm_dim + p.norm_eps);
+}
+
 template <int BN, int EPI>
-__device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, int slot, int row, bool valid,
-                                             int nb) {
+__device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
+                                             bool valid, int nb) {
+  const int slot = nd.z;
   const long long rofs = (long long)row;
   if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
     float rs = 1.f;
-    if (EPI == TC_EPI_RESID && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+    if (EPI != TC_EPI_F32 && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
+    if (EPI == TC_EPI_F32 && p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
+    float ss = 0.f;
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       float v[32];
@@ -243,21 +275,36 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       const int nv = p.N - col;
       if (EPI == TC_EPI_F32) {
         float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+        if (p.rsq) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= rs;
+        }
         store_f32x32(C, v, nv);
       } else {
         float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
         resid_add32(H, v, rs, nv);
+        if (p.rsq) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
+        }
         if (EPI == TC_EPI_RESID_ACT) {
           f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
           store_act32(X, v, nv);
+          if (to_out) {
+            bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
+            store_bf16_32(O, v, nv);
+          }
         }
       }
     }
+    if (EPI != TC_EPI_F32 && p.rsq && valid)
+      p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + nb] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
     const int hd = p.head_dim;
     const int cph = hd / 32;          // chunks per head
     const int pairs = hd / 64;        // chunk pairs per head
+    const float rs = (p.rsq && valid) ? norm_row_scale(p, slot, row) : 1.f;
 #pragma unroll 1
     for (int hh = 0; hh < BN / hd; ++hh) {
       const int head = (nb * BN) / hd + hh;
@@ -275,9 +322,15 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float2 a = cs[i];
-            const float x1 = v1[i], x2 = v2[i];
+            const float x1 = v1[i] * rs, x2 = v2[i] * rs;
             v1[i] = x1 * a.x - x2 * a.y;
             v2[i] = x2 * a.x + x1 * a.y;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v1[i] *= rs;
+            v2[i] *= rs;
           }
         }
         f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
@@ -289,6 +342,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
     // tile columns [0, BN/2) = gate features f0.., [BN/2, BN) = up features f0..
     constexpr int HALF = BN / 2;
     const int f0 = nb * HALF;
+    const float rs = (p.rsq && valid) ? norm_row_scale(p, slot, row) : 1.f;
 #pragma unroll 1
     for (int c = 0; c < HALF / 32; ++c) {
       float g[32], u[32];
@@ -297,7 +351,10 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       const int f = f0 + c * 32;
       if (!valid || f >= p.f_out) continue;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) g[i] = g[i] / (1.f + __expf(-g[i])) * u[i];
+      for (int i = 0; i < 32; ++i) {
+        const float gi = g[i] * rs;
+        g[i] = gi / (1.f + __expf(-gi)) * (u[i] * rs);
+      }
       f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + f;
       store_act32(C, g, p.f_out - f);
     }
@@ -447,7 +504,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = mb * BM + row_in_tile;
       const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd.z, row, valid, nb);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);

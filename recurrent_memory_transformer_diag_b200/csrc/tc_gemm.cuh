@@ -7,9 +7,10 @@ namespace armt {
 
 // Fused epilogues (thread = one accumulator row; see tc_gemm.cu).
 enum TcEpi {
-  TC_EPI_F32 = 0,        // C (fp32) = acc
+  TC_EPI_F32 = 0,        // C (fp32) = acc (times the RMSNorm row scale when rsq is set)
   TC_EPI_RESID = 1,      // h += acc * rowscale[row]   (rowscale optional)
-  TC_EPI_RESID_ACT = 2,  // h += acc; C (fp16) = h     (GEMM-operand copy of the new residual)
+  TC_EPI_RESID_ACT = 2,  // as RESID, and C (fp16) = new h (the next GEMM's operand); optional
+                         // norm partials (rsq) and bf16 copy of rows < seg_len to `out`
   TC_EPI_QKV_ROPE = 3,   // C (fp16) = acc, rotate-half RoPE on heads < rope_heads
   TC_EPI_SWIGLU = 4      // C (fp16)[f] = silu(acc[gate f]) * acc[up f]; B rows interleaved per 128
 };
@@ -26,6 +27,14 @@ struct TcGemmParams {
   const float* rowscale; long long rs_slot_stride;
   const float2* rope; int rope_half; int rope_heads; int head_dim;
   int f_out;                // SWIGLU: number of valid output features
+  // RMSNorm folded into the GEMMs.  Residual epilogues write, per row and per
+  // n-tile, the partial sum of squares of the new residual over the tile's
+  // columns (rsq[slot][row][tile], rsq_parts entries per row); QKV and gate/up
+  // epilogues scale their rows by rsqrt(sum of the partials / norm_dim + eps).
+  float* rsq; long long rsq_slot_stride; int rsq_parts; int norm_dim; float norm_eps;
+  int rsq_row0;             // F32 epilogue: output row r is normalised with the partials of row rsq_row0 + r
+  // final hidden states (down-projection epilogue of last-layer nodes)
+  void* out; int out_layer; int seg_len;
   unsigned* err;            // device error word (bounded waits)
 };
 

@@ -65,12 +65,12 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
   Dims dm{};
   dm.L = 1; dm.d = d; dm.M = M; dm.dk = d_key; dm.nu = nu; dm.P = 2 * d_key * nu; dm.mem_eps = eps;
   dm.bf16 = false;
-  if ((size_t)dm.M * dm.P * 4 + 9 * dm.M * 4 > 200 * 1024) return ARMT_ERR_UNSUPPORTED;
+  if (((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + 9 * dm.M) * 4 > 200 * 1024) return ARMT_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = setup_memory_kernels(dm);
   if (e != cudaSuccess) return to_status(e);
   const size_t n_w = (size_t)(d_key + d) * d, n_kv = (size_t)M * (d_key + d), n_ph = (size_t)M * dm.P;
-  const size_t bytes = (n_w + n_kv + n_ph + 2 * (size_t)M) * sizeof(float) + sizeof(NodeEntry);
+  const size_t bytes = (n_w + n_kv + n_ph + 2 * (size_t)M + (size_t)M * M) * sizeof(float) + sizeof(NodeEntry);
   char* scratch = nullptr;
   e = cudaMallocAsync((void**)&scratch, bytes, st);
   if (e != cudaSuccess) return to_status(e);
@@ -80,6 +80,7 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
   float* phik = kv + n_kv;
   float* coef = phik + n_ph;
   float* gamma = coef + M;
+  float* gram = gamma + M;
   static const NodeEntry one = {0, 0, 0, 0};
   e = cudaMemcpyAsync(node, &one, sizeof(NodeEntry), cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w_kv, wk, (size_t)d_key * d * 4, cudaMemcpyDeviceToDevice, st);
@@ -94,8 +95,8 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
     g.epi = EPI_STORE_F32;
     e = launch_simt_gemm(g, st);
   }
-  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, coef, gamma, st);
-  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, coef, A, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, st);
+  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, A, nullptr, st);
   cudaError_t e2 = cudaFreeAsync(scratch, st);
   if (e == cudaSuccess) e = e2;
   return to_status(e);
