@@ -52,16 +52,17 @@ typedef enum {
   ARMT_ERR_OOM = 4,             /* device allocation failed */
   ARMT_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
   ARMT_ERR_DEVICE_TIMEOUT = 6,  /* a kernel's bounded wait ran out (reported by armt_device_status) */
-  ARMT_ERR_UNSUPPORTED = 7      /* valid but not implemented shape (e.g. head_dim not 16..128 step 16) */
+  ARMT_ERR_UNSUPPORTED = 7,     /* valid but not implemented shape (e.g. head_dim not 16..128 step 16) */
+  ARMT_ERR_NUMERIC_RANGE = 8    /* an fp16 operand copy overflowed (reported by armt_device_status) */
 } armt_status;
 
 /* ARMT_FP32: fp32 weights and activations, SIMT kernels.
  * ARMT_BF16: weights rounded to bf16 (round to nearest even) on load; the
  *   tensor-core path stores these bf16 values in fp16 (exact for every value
- *   of magnitude >= 2^-17) and keeps the GEMM activations in fp16, which the
- *   tcgen05 tensor cores multiply at the bf16 rate with 3 more mantissa bits;
- *   accumulation, residual stream and memory state are fp32; embeddings in
- *   and hidden states out are bf16.
+ *   of magnitude >= 2^-17) and keeps the GEMM/attention activations and the
+ *   memory-read operands in fp16, which the tcgen05 tensor cores multiply at
+ *   the bf16 rate with 3 more mantissa bits; accumulation, residual stream
+ *   and memory state are fp32; embeddings in and hidden states out are bf16.
  * ARMT_F16: fp16 operands; accepted by armt_grouped_gemm only. */
 typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1, ARMT_F16 = 2 } armt_dtype;
 
@@ -156,8 +157,9 @@ armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int se
                               void* stream);
 
 /* Wait for `stream`, then report and clear the device-side error word that
- * kernels set when a bounded wait runs out: ARMT_OK or
- * ARMT_ERR_DEVICE_TIMEOUT (or ARMT_ERR_CUDA if the stream itself failed). */
+ * kernels set when a bounded wait runs out (ARMT_ERR_DEVICE_TIMEOUT) or an
+ * fp16 operand copy overflows (ARMT_ERR_NUMERIC_RANGE); ARMT_OK otherwise
+ * (ARMT_ERR_CUDA if the stream itself failed). */
 armt_status armt_device_status(armt_ctx* ctx, void* stream);
 
 /* Kernel launches one armt_forward enqueues for (S, current schedule):

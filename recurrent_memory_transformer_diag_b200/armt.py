@@ -25,6 +25,7 @@ SCHED = {"diagonal": 0, "sequential": 1}
 STATUS = {
     0: "ARMT_OK", 1: "ARMT_ERR_INVALID_ARG", 2: "ARMT_ERR_NOT_LOADED", 3: "ARMT_ERR_SHAPE",
     4: "ARMT_ERR_OOM", 5: "ARMT_ERR_CUDA", 6: "ARMT_ERR_DEVICE_TIMEOUT", 7: "ARMT_ERR_UNSUPPORTED",
+    8: "ARMT_ERR_NUMERIC_RANGE",
 }
 
 # Every symbol the header declares (checked by the CPU tests).

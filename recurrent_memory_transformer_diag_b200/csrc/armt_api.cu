@@ -220,7 +220,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.epi = EPI_STORE_F32;
     L("gemm_qmem", [&] { return launch_simt_gemm(g, st); });
   }
-  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
+  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, ws.err, st); });
   {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = Tp; g.N = dm.d; g.K = dm.P;
@@ -290,7 +290,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   }
   L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, nullptr, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, nullptr, nullptr, st);
   });
 
   if (wv.any_last_layer)
@@ -302,9 +302,9 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
 // bf16-rounded values in fp16 containers and the GEMM activations are fp16
 // (same tensor-core rate as bf16, 3 more mantissa bits: rounding the
 // normalised activations to bf16 alone costs ~1 % relative error over 16
-// layers); the memory-read product phi A^T keeps bf16 operands because A
-// spans a wide range of magnitudes.  Residual stream, accumulation and the
-// memory state are fp32.
+// layers), as are the memory-read operands phi and the copy of A.  A value
+// past the fp16 range sets ERR_FP16_RANGE in the error word.  Residual
+// stream, accumulation and the memory state are fp32.
 void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
                      cudaStream_t st, Launcher& L) {
   const Dims& dm = ctx->dm;
@@ -339,12 +339,11 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.C = ws.qm; p.c_slot_stride = (long long)Tp * dm.dk; p.ldc = dm.dk;
     return launch_tc_gemm(op, p, TC_EPI_F32, tc_pick_bn(dm.dk), sms, st);
   });
-  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
+  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, ws.err, st); });
   L("tc_read", [&] {
     // h += phi A^T / (z.phi + eps); new h -> fp16 operand copy + norm partials
     TcGemmOperands op{ws.phi, Tp, slots, ws.a_act, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.P);
-    p.ab_bf16 = 1;
     p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
     p.rowscale = ws.inv_den; p.rs_slot_stride = Tp;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
@@ -405,7 +404,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   });
   L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, ws.a_act, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, ws.a_act, ws.err, st);
   });
 
 }
@@ -509,6 +508,7 @@ extern "C" const char* armt_status_string(armt_status s) {
     case ARMT_ERR_CUDA: return "CUDA error";
     case ARMT_ERR_DEVICE_TIMEOUT: return "device-side bounded wait timed out";
     case ARMT_ERR_UNSUPPORTED: return "unsupported shape";
+    case ARMT_ERR_NUMERIC_RANGE: return "a value exceeded the fp16 range of an operand copy";
   }
   return "unknown status";
 }
@@ -750,7 +750,8 @@ extern "C" armt_status armt_device_status(armt_ctx* ctx, void* stream) {
   ARMT_TRY(cudaMemcpy(&flag, ctx->ws.err, sizeof(unsigned), cudaMemcpyDeviceToHost), "read error word");
   if (flag) {
     ARMT_TRY(cudaMemset(ctx->ws.err, 0, sizeof(unsigned)), "clear error word");
-    return fail(ctx, ARMT_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait timed out");
+    if (flag & ERR_WAIT_TIMEOUT_MASK) return fail(ctx, ARMT_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait timed out");
+    return fail(ctx, ARMT_ERR_NUMERIC_RANGE, "an fp16 operand copy exceeded the fp16 range");
   }
   return ARMT_OK;
 }

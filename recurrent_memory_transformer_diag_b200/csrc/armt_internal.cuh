@@ -17,6 +17,10 @@ namespace armt {
 typedef __nv_bfloat16 bf16;
 typedef __half f16;
 
+// Bits of the device error word (Workspace::err).
+constexpr unsigned ERR_WAIT_TIMEOUT_MASK = 7u;   // bits 0..2: a bounded mbarrier wait ran out
+constexpr unsigned ERR_FP16_RANGE = 8u;          // an fp16 operand copy exceeded the fp16 range
+
 // One node of the (segment, layer) grid as the kernels see it: x = segment s,
 // y = layer l, z = activation slot (s mod number-of-slots), w = flags.
 typedef int4 NodeEntry;
@@ -37,7 +41,7 @@ struct Workspace {
   float* h = nullptr;       // [slots][T'][d] residual stream, fp32
   void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (fp32, or fp16 on the tensor-core path)
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
-  void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or bf16 on the tensor-core path)
+  void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or fp16 on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
   float* rsq = nullptr;     // [slots][T'][ceil(d/256)] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
@@ -49,7 +53,7 @@ struct Workspace {
   float* gram = nullptr;    // [slots][M][M] phi_j . phi_j'
   float* coef = nullptr;    // [slots][M] 1 / (z_j . phi_j + eps)
   float* gamma = nullptr;   // [slots][M]
-  void* a_act = nullptr;    // [L][d][P] bf16 copy of A (tensor-core path: the read GEMM operand)
+  void* a_act = nullptr;    // [L][d][P] fp16 copy of A (tensor-core path: the read GEMM operand)
   float2* rope = nullptr;   // [tp_max][hd/2] (cos, sin)
   NodeEntry* nodes = nullptr;
   int nodes_cap = 0;
@@ -128,7 +132,7 @@ cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int 
 cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int row0, int nrows,
                            const float* h, void* xb, float eps, cudaStream_t st);
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
-                             const float* z_state, void* phi, float* inv_den, cudaStream_t st);
+                             const float* z_state, void* phi, float* inv_den, unsigned* err, cudaStream_t st);
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
                         const float2* rope, cudaStream_t st);
 cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
@@ -140,7 +144,7 @@ cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const
                             cudaStream_t st);
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                                const float* phik, const float* gram, const float* coef, float* A_state,
-                               void* a_act, cudaStream_t st);
+                               void* a_act, unsigned* err, cudaStream_t st);
 cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                           const float* h, void* out, cudaStream_t st);
 

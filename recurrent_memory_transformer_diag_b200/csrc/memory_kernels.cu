@@ -116,14 +116,15 @@ cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const
 
 constexpr int MEMW_ROWS_PER_BLOCK = 64;
 
-// A_state: [L][d][P] fp32 in place; a_act: optional bf16 copy [L][d][P].
+// A_state: [L][d][P] fp32 in place; a_act: optional fp16 copy [L][d][P] (a
+// value past the fp16 range sets the error word).
 // grid (ceil(d / MEMW_ROWS_PER_BLOCK), nodes), 8 warps, one A row per warp per
 // iteration; phi, G and coef are staged once per block.
 template <int MAXC>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
                                                           const float* gram, const float* coef, float* A_state,
-                                                          bf16* a_act) {
+                                                          f16* a_act, unsigned* err) {
   extern __shared__ float sh[];
   float* ph = sh;                    // [M][P]
   float* G = ph + M * P;             // [M][M]
@@ -137,6 +138,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* dl = dots + warp * M;
+  bool over = false;
   const int i_end = min(d, (blockIdx.x + 1) * MEMW_ROWS_PER_BLOCK);
   for (int i = blockIdx.x * MEMW_ROWS_PER_BLOCK + warp; i < i_end; i += 8) {
     float* Arow = A_state + ((long long)layer * d + i) * P;
@@ -175,11 +177,15 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
         float acc = a[c];
         for (int j = 0; j < M; ++j) acc = fmaf(dl[j], ph[j * P + p], acc);
         Arow[p] = acc;
-        if (a_act) a_act[((long long)layer * d + i) * P + p] = __float2bfloat16_rn(acc);
+        if (a_act) {
+          a_act[((long long)layer * d + i) * P + p] = __float2half_rn(acc);
+          over |= fabsf(acc) > 65504.f;
+        }
       }
     }
     __syncwarp();
   }
+  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
 static size_t memw_update_smem(const Dims& dm) {
@@ -188,13 +194,13 @@ static size_t memw_update_smem(const Dims& dm) {
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                                const float* phik, const float* gram, const float* coef, float* A_state,
-                               void* a_act, cudaStream_t st) {
+                               void* a_act, unsigned* err, cudaStream_t st) {
   dim3 grid((dm.d + MEMW_ROWS_PER_BLOCK - 1) / MEMW_ROWS_PER_BLOCK, n);
   const size_t sh = memw_update_smem(dm);
   const int chunks = (dm.P + 31) / 32;
 #define ARMT_MEMW_CASE(C)                                                                              \
   memw_update_kernel<C><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
-                                               A_state, (bf16*)a_act);
+                                               A_state, (f16*)a_act, err);
   if (chunks <= 4) ARMT_MEMW_CASE(4)
   else if (chunks <= 12) ARMT_MEMW_CASE(12)
   else if (chunks <= 24) ARMT_MEMW_CASE(24)

@@ -155,8 +155,9 @@ cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp
 }
 
 // ---------------------------------------------------------------------------
-// Memory read, feature step: phi = DPFP_nu(q) per row, stored in the act
-// dtype, and inv_den = 1 / (z_l . phi + eps) computed from the stored
+// Memory read, feature step: phi = DPFP_nu(q) per row, stored as fp32 (fp32
+// path) or fp16 (tensor-core path; a value past the fp16 range sets the
+// error word), and inv_den = 1 / (z_l . phi + eps) computed from the stored
 // (rounded) features so that numerator and denominator see the same phi.
 // DPFP: r = [relu(q); relu(-q)], phi[(n-1) 2dk + j] = r_j r_{(j-n) mod 2dk}.
 // One warp per row.
@@ -164,7 +165,7 @@ cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp
 template <typename TP>
 __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu, int P,
                                  const float* qm, const float* z_state, TP* phi, float* inv_den,
-                                 float eps) {
+                                 float eps, unsigned* err) {
   extern __shared__ float r_sh[];   // [8 warps][2 dk]
   const NodeEntry nd = nodes[blockIdx.y];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -183,27 +184,31 @@ __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu,
   const float* z = z_state + (long long)nd.y * P;
   TP* out = phi + roff * P;
   float dot = 0.f;
+  bool over = false;
   for (int p = lane; p < P; p += 32) {
     const int n = p / n2 + 1, j = p - (n - 1) * n2;
     int jj = (j - n) % n2;
     if (jj < 0) jj += n2;
-    st(out, p, r[j] * r[jj]);
+    const float f = r[j] * r[jj];
+    over |= f > 65504.f;
+    st(out, p, f);
     dot = fmaf(ld(out, p), z[p], dot);
   }
   dot = warp_sum(dot);
   if (lane == 0) inv_den[roff] = 1.f / (dot + eps);
+  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
-                             const float* z_state, void* phi, float* inv_den, cudaStream_t st) {
+                             const float* z_state, void* phi, float* inv_den, unsigned* err, cudaStream_t st) {
   dim3 grid((Tp + 7) / 8, n);
   const size_t sh = 8 * 2 * dm.dk * sizeof(float);
   if (dm.bf16)
-    dpfp_read_kernel<bf16><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
-                                                  (bf16*)phi, inv_den, dm.mem_eps);
+    dpfp_read_kernel<f16><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
+                                                 (f16*)phi, inv_den, dm.mem_eps, err);
   else
     dpfp_read_kernel<float><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
-                                                   (float*)phi, inv_den, dm.mem_eps);
+                                                   (float*)phi, inv_den, dm.mem_eps, nullptr);
   return cudaGetLastError();
 }
 

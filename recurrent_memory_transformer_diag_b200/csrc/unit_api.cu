@@ -96,7 +96,7 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
     e = launch_simt_gemm(g, st);
   }
   if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, st);
-  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, A, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, A, nullptr, nullptr, st);
   cudaError_t e2 = cudaFreeAsync(scratch, st);
   if (e == cudaSuccess) e = e2;
   return to_status(e);

@@ -28,7 +28,7 @@ def test_library_exports_every_declared_symbol(libarmt):
 
 
 def test_status_strings(libarmt):
-    for code in range(8):
+    for code in range(9):
         s = libarmt.armt_status_string(code)
         assert s and s != b"unknown status"
     assert libarmt.armt_status_string(99) == b"unknown status"

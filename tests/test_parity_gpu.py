@@ -164,9 +164,12 @@ def test_launch_count_diagonal_vs_sequential(small):
     ns = m.launch_count(S)
     m.close()
     assert nd < ns
-    # per wave: the same kernel sequence, plus the layer-0 input kernel when
-    # the wave holds a layer-0 node and the output kernel when it holds a
-    # last-layer node (S of each in both schedules)
-    per_wave = (ns - 2 * S) // (S * L)
-    assert ns == S * L * per_wave + 2 * S
-    assert nd == (S + L - 1) * per_wave + 2 * S
+    # every wave launches the same kernel sequence (b kernels), plus extra
+    # kernels in the S waves that hold a layer-0 node (and, where the output
+    # is not fused, the S waves that hold a last-layer node): the same extras
+    # in both schedules, so ns - nd = (S*L - (S+L-1)) * b
+    b, rem = divmod(ns - nd, S * L - (S + L - 1))
+    assert rem == 0 and b > 0
+    extra = nd - (S + L - 1) * b
+    assert extra in (S, 2 * S)
+    assert ns == S * L * b + extra
