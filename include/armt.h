@@ -219,6 +219,28 @@ armt_status armt_memory_write(int M, int d, int d_key, int nu, float eps,
                               const float* m, const float* wk, const float* wv,
                               float* A, float* z, void* stream);
 
+/* The same delta-rule memory write as armt_memory_write, for callers that
+ * cannot allocate device memory at call time (a host framework that has
+ * reserved the device memory for its own allocator, a real-time loop with a
+ * memory budget fixed at start-up, a plug-in whose host forbids device
+ * allocation after initialisation).  The paper has no counterpart: this is
+ * a deployment variant of the library's own write kernel.
+ *
+ * It allocates nothing: its scratch is a fixed 1 MiB array in the library's
+ * device image (held by every device that loads the library, until the
+ * process exits), enough for 4 + M*(d_key + d) + M*P + M*M + 2*M floats
+ * (P = 2*d_key*nu), e.g. M = 16 rows at d = 3072, d_key = 128, nu = 3.
+ * Larger sizes return ARMT_ERR_SHAPE without launching anything.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array, so calls whose work overlaps on the GPU
+ * (other streams, other host threads) race: order them on one stream.
+ * Arguments, layouts and errors otherwise as armt_memory_write. */
+armt_status armt_memory_write_static(int M, int d, int d_key, int nu, float eps,
+                                     const float* m, const float* wk, const float* wv,
+                                     float* A, float* z, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ EXPORTS = (
     "armt_create", "armt_load_weights", "armt_set_schedule", "armt_set_graph", "armt_forward",
     "armt_forward_host", "armt_device_status", "armt_launch_count", "armt_destroy",
     "armt_status_string", "armt_last_error", "armt_grouped_gemm", "armt_memory_write",
-    "armt_kernel_kinds", "armt_kernel_kind_name", "armt_profile_forward",
+    "armt_kernel_kinds", "armt_kernel_kind_name", "armt_profile_forward", "armt_memory_write_static",
 )
 
 
@@ -89,6 +89,7 @@ def lib() -> ctypes.CDLL:
     L.armt_grouped_gemm.argtypes = [c_int, c_int, c_int, c_int, c_int, vp, vp, c_int,
                                     ctypes.POINTER(c_int), vp, vp]
     L.armt_memory_write.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
+    L.armt_memory_write_static.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
     L.armt_kernel_kinds.argtypes = []
     L.armt_kernel_kind_name.argtypes = [c_int]
     L.armt_kernel_kind_name.restype = ctypes.c_char_p
@@ -216,6 +217,15 @@ def grouped_gemm(A, B, bidx, C, stream=None):
     idx = (ctypes.c_int * G)(*[int(i) for i in bidx])
     _check(lib().armt_grouped_gemm(dtype, G, m, n, k, _ptr(A), _ptr(B), num_b, idx, _ptr(C),
                                    _stream_handle(stream)), "armt_grouped_gemm")
+
+
+def memory_write_static(m, wk, wv, A, z, nu: int, eps: float, stream=None):
+    """armt_memory_write_static: the same write with the library's fixed
+    device scratch, for callers that cannot allocate device memory."""
+    M, d = m.shape
+    dk = wk.shape[0]
+    _check(lib().armt_memory_write_static(M, d, dk, nu, eps, _ptr(m), _ptr(wk), _ptr(wv), _ptr(A), _ptr(z),
+                                          _stream_handle(stream)), "armt_memory_write_static")
 
 
 def memory_write(m, wk, wv, A, z, nu: int, eps: float, stream=None):
