@@ -303,6 +303,8 @@ def run_ours(args, cfg, S):
     d_flops_launch = flops.get(dominant, 0) / max(dcnt, 1)
     achieved = d_flops_launch / (dms / dcnt / 1e3) / 1e12
     traffic = read_traffic(dominant)
+    if traffic is not None:
+        traffic = round(traffic * n_nodes / dcnt)   # bytes per node x nodes per launch (average over launches)
     roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1), "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": round(achieved / peak_tf, 4),
                 "peak_note": f"dense bf16 sustained {peak_note}",
@@ -363,8 +365,10 @@ def run_ours(args, cfg, S):
 
 
 def read_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
-    was taken on the current kernel source (its hash is recorded there)."""
+    """DRAM bytes per node of `kernel` from the committed ncu summary
+    (profiles/traffic.txt: dram__bytes_read.sum + dram__bytes_write.sum of one
+    captured full wave, divided by its nodes), if it was taken on the current
+    kernel source (the source hash is recorded there); else None."""
     import hashlib
     summ = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "recurrent_memory_transformer_diag_b200", "csrc", "tc_gemm.cu")
