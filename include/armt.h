@@ -80,7 +80,7 @@ typedef struct {
   int n_kv_heads;   /* KV heads, H % KV == 0 */
   int head_dim;     /* hd, even */
   int d_ffn;        /* F */
-  int n_mem;        /* M memory tokens per segment */
+  int n_mem;        /* M memory tokens per segment, 1..32 */
   int d_key;        /* memory key dimension d_k */
   int dpfp_nu;      /* DPFP order nu */
   float rope_theta;
@@ -212,7 +212,8 @@ armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, int k,
                               float* C, void* stream);
 
 /* Delta-rule memory write of one node (the write step above) on device
- * buffers: m [M, d] fp32 memory rows, wk [d_k, d], wv [d, d] fp32,
+ * buffers: m [M, d] fp32 memory rows (M <= 32; rows written in order, each
+ * seeing the state the previous rows left), wk [d_k, d], wv [d, d] fp32,
  * A [d, P] and z [P] fp32 updated in place.  Asynchronous on stream.
  * Errors: INVALID_ARG, CUDA, OOM (scratch allocation). */
 armt_status armt_memory_write(int M, int d, int d_key, int nu, float eps,

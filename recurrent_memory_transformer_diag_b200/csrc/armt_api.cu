@@ -96,7 +96,7 @@ armt_status validate_config(const armt_config* c, const char** why) {
   }
   const long long P = 2LL * c->d_key * c->dpfp_nu;
   if (P > 1024) { *why = "phi dimension 2*d_key*nu must be <= 1024"; return ARMT_ERR_UNSUPPORTED; }
-  if (c->n_mem > 64) { *why = "n_mem must be <= 64"; return ARMT_ERR_UNSUPPORTED; }
+  if (c->n_mem > 32) { *why = "n_mem must be <= 32"; return ARMT_ERR_UNSUPPORTED; }
   if (((long long)c->n_mem * P + (long long)c->n_mem * c->n_mem + 9LL * c->n_mem) * 4 > 200 * 1024) {
     *why = "n_mem * phi dimension too large for the write kernel"; return ARMT_ERR_UNSUPPORTED;
   }
@@ -323,7 +323,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.nodes = nodes; p.n_nodes = n; p.M = M; p.N = N; p.K = K; p.err = ws.err;
     p.out_layer = -1;
   };
-  const int rsq_parts = (dm.d + 255) / 256;
+  const int rsq_parts = 2 * ((dm.d + 255) / 256);   // one partial per half of a 256-column tile
   auto norm_partials = [&](TcGemmParams& p) {
     p.rsq = ws.rsq; p.rsq_slot_stride = (long long)Tp * rsq_parts; p.rsq_parts = rsq_parts;
     p.norm_dim = dm.d; p.norm_eps = dm.rms_eps;
@@ -552,7 +552,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   A(&ws.qm, rows * dm.dk * 4);
   A(&ws.phi, rows * dm.P * as);
   A(&ws.inv_den, rows * 4);
-  if (dm.bf16) A(&ws.rsq, rows * ((dm.d + 255) / 256) * 4);
+  if (dm.bf16) A(&ws.rsq, rows * 2 * ((dm.d + 255) / 256) * 4);
   A(&ws.qkv, rows * dm.nqkv * as);
   A(&ws.attn, rows * dm.H * dm.hd * as);
   if (!dm.bf16) A(&ws.gu, rows * 2 * dm.F * as);

@@ -43,7 +43,7 @@ struct Workspace {
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
   void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or fp16 on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
-  float* rsq = nullptr;     // [slots][T'][ceil(d/256)] RMSNorm partial sums (tensor-core path)
+  float* rsq = nullptr;     // [slots][T'][2 ceil(d/256)] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
   void* attn = nullptr;     // [slots][T'][H*hd]  (fp32 / fp16)
   void* gu = nullptr;       // [slots][T'][2F]    (fp32 path only)

@@ -120,6 +120,7 @@ constexpr int MEMW_ROWS_PER_BLOCK = 64;
 // value past the fp16 range sets the error word).
 // grid (ceil(d / MEMW_ROWS_PER_BLOCK), nodes), 8 warps, one A row per warp per
 // iteration; phi, G and coef are staged once per block.
+// M <= 32: lane j carries memory row j through the recurrence.
 template <int MAXC>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
@@ -148,6 +149,8 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
       const int p = lane + 32 * c;
       a[c] = p < P ? Arow[p] : 0.f;
     }
+    // lane j (< M <= 32) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
+    float s = 0.f;
     for (int j = 0; j < M; ++j) {
       const float* pj = ph + j * P;
       float dot = 0.f;
@@ -157,17 +160,15 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
         if (p < P) dot = fmaf(a[c], pj[p], dot);
       }
       dot = warp_sum_m(dot);
-      if (lane == 0) dl[j] = dot;
+      if (lane == j) s = dot;
     }
-    __syncwarp();
-    if (lane == 0) {
-      // delta_j = v_j[i] - (a . phi_j + sum_{j'<j} delta_j' G[j'][j]) * coef_j
-      for (int j = 0; j < M; ++j) {
-        float s = dl[j];
-        for (int jp = 0; jp < j; ++jp) s = fmaf(dl[jp], G[jp * M + j], s);
-        const float v = kv[((long long)slot * M + j) * (dk + d) + dk + i];
-        dl[j] = v - s * cf[j];
-      }
+    const float vj = lane < M ? kv[((long long)slot * M + lane) * (dk + d) + dk + i] : 0.f;
+    const float cj = lane < M ? cf[lane] : 0.f;
+    for (int j = 0; j < M; ++j) {
+      // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
+      const float dj = __shfl_sync(0xffffffffu, vj - s * cj, j);
+      if (lane == j) dl[j] = dj;
+      if (lane > j && lane < M) s = fmaf(dj, G[j * M + lane], s);
     }
     __syncwarp();
 #pragma unroll

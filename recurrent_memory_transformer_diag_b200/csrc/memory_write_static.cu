@@ -66,7 +66,7 @@ extern "C" armt_status armt_memory_write_static(int M, int d, int d_key, int nu,
                                                 void* stream) {
   if (M < 1 || d < 1 || d_key < 1 || nu < 1 || !(eps > 0.f) || !m || !wk || !wv || !A || !z)
     return ARMT_ERR_INVALID_ARG;
-  if (M > 64 || nu > 2 * d_key || 2 * d_key * nu > 1024) return ARMT_ERR_UNSUPPORTED;
+  if (M > 32 || nu > 2 * d_key || 2 * d_key * nu > 1024) return ARMT_ERR_UNSUPPORTED;
   Dims dm{};
   dm.L = 1; dm.d = d; dm.M = M; dm.dk = d_key; dm.nu = nu; dm.P = 2 * d_key * nu; dm.mem_eps = eps;
   dm.bf16 = false;

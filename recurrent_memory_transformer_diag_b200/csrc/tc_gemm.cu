@@ -12,13 +12,14 @@
 // Operands are 16-bit, both fp16 or both bf16 (a runtime instruction-
 // descriptor field).
 //
-// Kernel structure (persistent, one CTA per SM, 192 threads):
+// Kernel structure (persistent, one CTA per SM, 320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (16-bit, 128-byte
 //               swizzle) per pipeline stage
 //   warp 1      allocates TMEM; one lane issues tcgen05.mma (M=128, N=BN,
 //               K=16) and commits stage/accumulator barriers
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (thread = row),
-//               fused per-use epilogue, stores to global memory
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator rows (thread = row;
+//               warps w and w+4 share TMEM lanes 32*(w%4).. and split the
+//               tile's columns in halves), fused epilogue, global stores
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap
 // the main loop of tile t+1.  Tiles never straddle nodes: a node's rows are
 // the middle TMA coordinate with extent M, rows past M read as zeros.
@@ -37,7 +38,8 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;           // two warps per TMEM lane quarter, each half of the columns
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
 constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -257,7 +259,7 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
 
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb) {
+                                             bool valid, int nb, int half) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
   if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
@@ -267,7 +269,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
     if (EPI == TC_EPI_F32 && p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
     float ss = 0.f;
 #pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
+    for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
       const int col = nb * BN + c * 32;
@@ -298,15 +300,16 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       }
     }
     if (EPI != TC_EPI_F32 && p.rsq && valid)
-      p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + nb] = ss;
+      p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + 2 * nb + half] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
     const int hd = p.head_dim;
     const int cph = hd / 32;          // chunks per head
     const int pairs = hd / 64;        // chunk pairs per head
     const float rs = (p.rsq && valid) ? norm_row_scale(p, slot, row) : 1.f;
+    const int heads_half = BN / hd / 2;
 #pragma unroll 1
-    for (int hh = 0; hh < BN / hd; ++hh) {
+    for (int hh = half * heads_half; hh < (half + 1) * heads_half; ++hh) {
       const int head = (nb * BN) / hd + hh;
       const bool rot = head < p.rope_heads;
 #pragma unroll 1
@@ -344,7 +347,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
     const int f0 = nb * HALF;
     const float rs = (p.rsq && valid) ? norm_row_scale(p, slot, row) : 1.f;
 #pragma unroll 1
-    for (int c = 0; c < HALF / 32; ++c) {
+    for (int c = half * (HALF / 64); c < (half + 1) * (HALF / 64); ++c) {
       float g[32], u[32];
       tmem_ld32(tbase + c * 32, g);
       tmem_ld32(tbase + HALF + c * 32, u);
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);
+      mbar_init(&tempty[b], EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -485,8 +488,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int half = (warp - 2) >> 2;        // which half of the tile's columns
     const int row_in_tile = quarter * 32 + lane;
     int buf = 0;
     uint32_t acc_phase = 0;
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = mb * BM + row_in_tile;
       const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);

@@ -28,9 +28,10 @@ struct TcGemmParams {
   const float2* rope; int rope_half; int rope_heads; int head_dim;
   int f_out;                // SWIGLU: number of valid output features
   // RMSNorm folded into the GEMMs.  Residual epilogues write, per row and per
-  // n-tile, the partial sum of squares of the new residual over the tile's
-  // columns (rsq[slot][row][tile], rsq_parts entries per row); QKV and gate/up
-  // epilogues scale their rows by rsqrt(sum of the partials / norm_dim + eps).
+  // half n-tile, the partial sum of squares of the new residual over those
+  // columns (rsq[slot][row][2 * tile + half], rsq_parts entries per row); QKV,
+  // gate/up and kv-mem epilogues scale their rows by
+  // rsqrt(sum of the partials / norm_dim + eps).
   float* rsq; long long rsq_slot_stride; int rsq_parts; int norm_dim; float norm_eps;
   int rsq_row0;             // F32 epilogue: output row r is normalised with the partials of row rsq_row0 + r
   // final hidden states (down-projection epilogue of last-layer nodes)

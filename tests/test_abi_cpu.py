@@ -45,7 +45,7 @@ def _cfg(**kw):
     ("n_layers", 0, 1), ("d_model", -1, 1), ("n_mem", 0, 1), ("max_segments", 0, 1),
     ("n_kv_heads", 3, 1), ("head_dim", 15, 1), ("dtype", 7, 1), ("schedule", 5, 1),
     ("mem_eps", 0.0, 1), ("rope_theta", -1.0, 1), ("dpfp_nu", 40, 1),
-    ("head_dim", 48, 7), ("n_mem", 100, 7), ("d_key", 600, 7),
+    ("head_dim", 48, 7), ("n_mem", 40, 7), ("d_key", 600, 7),
 ])
 def test_create_rejects_bad_config_before_device(libarmt, field, value, status):
     c = _cfg(**{field: value})

@@ -55,7 +55,7 @@ def test_static_write_matches_allocating_write_on_two_calls(M, d, dk, nu):
 def test_static_write_rejects_sizes_beyond_its_scratch():
     import torch
     from recurrent_memory_transformer_diag_b200 import ArmtError, memory_write_static
-    M, d, dk, nu = 64, 8192, 64, 3          # M*(dk+d) alone exceeds the 1 MiB array
+    M, d, dk, nu = 32, 16384, 64, 3         # M*(dk+d) alone exceeds the 1 MiB array
     m = torch.zeros(M, d, device="cuda")
     wk = torch.zeros(dk, d, device="cuda")
     wv = torch.zeros(8, 8, device="cuda")   # never read: the call is rejected first
