@@ -70,7 +70,7 @@ void free_weights(Weights& w) {
 void free_workspace(Workspace& ws) {
   dfree(ws.h); dfree(ws.xb); dfree(ws.qm); dfree(ws.phi); dfree(ws.inv_den); dfree(ws.qkv);
   dfree(ws.attn); dfree(ws.gu); dfree(ws.u); dfree(ws.kv); dfree(ws.phik); dfree(ws.coef);
-  dfree(ws.gamma); dfree(ws.a_act); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err); dfree(ws.rsq); dfree(ws.gram);
+  dfree(ws.gamma); dfree(ws.a_act); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err); dfree(ws.rsq); dfree(ws.gram); dfree(ws.vt);
   ws = Workspace();
 }
 
@@ -357,10 +357,16 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     TcGemmParams p; base(p, Tp, dm.nqkv, dm.d);
     p.C = ws.qkv; p.c_slot_stride = (long long)Tp * dm.nqkv; p.ldc = dm.nqkv;
     p.rope = ws.rope; p.rope_half = dm.hd / 2; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
+    if (ws.vt) {
+      p.vt = (f16*)ws.vt; p.vt_pitch = attention_tc_vt_pitch(Tp); p.n_vheads = dm.KV;
+    }
     norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_QKV_ROPE, 256, sms, st);
   });
-  L("attention", [&] { return launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
+  L("attention", [&] {
+    return ws.vt ? launch_attention_tc(dm, nodes, n, Tp, slots, ws.qkv, ws.vt, ws.attn, ws.err, st)
+                 : launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st);
+  });
   L("tc_o", [&] {
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
@@ -555,6 +561,8 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   if (dm.bf16) A(&ws.rsq, rows * 2 * ((dm.d + 255) / 256) * 4);
   A(&ws.qkv, rows * dm.nqkv * as);
   A(&ws.attn, rows * dm.H * dm.hd * as);
+  if (dm.bf16 && attention_tc_supported(dm))
+    A(&ws.vt, (size_t)ws.slots * dm.KV * dm.hd * attention_tc_vt_pitch(ws.tp_max) * 2);
   if (!dm.bf16) A(&ws.gu, rows * 2 * dm.F * as);
   A(&ws.u, rows * dm.F * as);
   A(&ws.kv, (size_t)ws.slots * dm.M * (dm.dk + dm.d) * 4);
@@ -581,6 +589,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   if (e == cudaSuccess) e = setup_memory_kernels(dm);
   if (e == cudaSuccess && dm.bf16) e = setup_tc_gemm();
   if (e == cudaSuccess && dm.bf16) e = setup_attention_mma();
+  if (e == cudaSuccess && dm.bf16 && attention_tc_supported(dm)) e = setup_attention_tc();
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ctx->capture_stream, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
     armt_status s = cuda_fail(nullptr, e, "create");

@@ -18,8 +18,8 @@ typedef __nv_bfloat16 bf16;
 typedef __half f16;
 
 // Bits of the device error word (Workspace::err).
-constexpr unsigned ERR_WAIT_TIMEOUT_MASK = 7u;   // bits 0..2: a bounded mbarrier wait ran out
-constexpr unsigned ERR_FP16_RANGE = 8u;          // an fp16 operand copy exceeded the fp16 range
+constexpr unsigned ERR_WAIT_TIMEOUT_MASK = 0x77u; // bits 0-2 (GEMM), 4-6 (attention): a bounded wait ran out
+constexpr unsigned ERR_FP16_RANGE = 8u;           // an fp16 operand copy exceeded the fp16 range
 
 // One node of the (segment, layer) grid as the kernels see it: x = segment s,
 // y = layer l, z = activation slot (s mod number-of-slots), w = flags.
@@ -46,6 +46,7 @@ struct Workspace {
   float* rsq = nullptr;     // [slots][T'][2 ceil(d/256)] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
   void* attn = nullptr;     // [slots][T'][H*hd]  (fp32 / fp16)
+  void* vt = nullptr;       // [slots][KV][hd][pitch] fp16 V^T for the tcgen05 attention
   void* gu = nullptr;       // [slots][T'][2F]    (fp32 path only)
   void* u = nullptr;        // [slots][T'][F]     (fp32 / fp16)
   float* kv = nullptr;      // [slots][M][dk + d]
@@ -150,7 +151,14 @@ cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, 
 
 cudaError_t setup_memory_kernels(const Dims& dm);
 
-// bf16 tensor-core attention (mma.sync); head_dim 64 or 128
+// tcgen05 attention (head_dim 64): reads V^T [slot][KV][hd][vt_pitch]
+bool attention_tc_supported(const Dims& dm);
+int attention_tc_vt_pitch(int Tp);
+cudaError_t setup_attention_tc();
+cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int slots, const void* qkv,
+                                const void* vt, void* out, unsigned* err, cudaStream_t st);
+
+// warp-level tensor-core attention (mma.sync); head_dim 64 or 128
 bool attention_mma_supported(const Dims& dm);
 cudaError_t setup_attention_mma();
 cudaError_t launch_attention_mma(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* qkv, void* out,

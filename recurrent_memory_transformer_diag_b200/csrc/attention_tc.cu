@@ -1,0 +1,404 @@
+// Batched causal attention on the 5th-generation tensor cores (tcgen05,
+// TMEM accumulators, TMA-fed operands), head_dim 64.
+//
+// The wave's nodes are a batch: a CTA handles one 128-row query tile of one
+// node for the H/KV query heads that share a kv head, so the node's keys and
+// values for that kv head stream through one CTA (Pith review of arXiv
+// 2506.05229, Figure 5: diagonal batching treats the groups as a batch for
+// attention).  Each node attends only over the T' rows of its own segment
+// plus memory tokens, causally.
+//
+// Per step (query head h, key tile j of 128 keys):
+//   MMA  S = Q K_j^T        (M=128 queries, N=128 keys, K=64)  -> TMEM S[j%2]
+//   softmax (warps 2..5, one thread per query row): row max, p = exp2(s - m),
+//        P (fp16) -> shared memory in the K-major swizzled operand layout
+//   MMA  O_j = P V_j        (M=128, N=64 dims, K=128 keys)      -> TMEM O[j%2]
+//   softmax warps: o = o * exp2(m_old - m_new) + O_j in registers
+// S of step t+1 is issued before O of step t, so the tensor core works on the
+// next tile while the softmax warps work on this one.  V is read as V^T
+// (written transposed by the QKV epilogue) so that every operand is K-major.
+// All mbarrier waits are bounded; on timeout the kernel sets the error word,
+// drains its copies and MMAs, frees TMEM and exits.
+#include "armt_internal.cuh"
+#include "tcgen05_ptx.cuh"
+
+namespace armt {
+
+namespace {
+
+using namespace tc;
+
+constexpr int HD = 64;
+constexpr int BQ = 128;                 // query rows per tile
+constexpr int BKEY = 128;               // keys per tile
+constexpr int NUM_THREADS = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
+constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
+constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
+constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB (two 64-key blocks of 8 KB)
+constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
+constexpr int OFF_Q = 0;                          // 2 buffers
+constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // 2 stages
+constexpr int OFF_VT = OFF_K + 2 * K_BYTES;       // 2 stages
+constexpr int OFF_P = OFF_VT + 2 * VT_BYTES;      // 2 buffers
+constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
+constexpr int TMEM_COLS = 512;                    // S[2] at 0, 128; O[2] at 256, 320
+
+struct AttnParams {
+  const NodeEntry* nodes;
+  int Tp;            // rows per node
+  int H, KV, nqkv;
+  int q_tiles;
+  float scale_log2;  // log2(e) / sqrt(hd)
+  f16* out;          // [slot][Tp][H*hd]
+  unsigned* err;
+};
+
+// P rows: K-major operand, 128 keys = two 64-key blocks, 128-byte swizzle.
+__device__ __forceinline__ void store_p_chunk(uint8_t* pbuf, int row, int c, const float* p) {
+  // chunk c = keys c*32 .. c*32+31 -> block c/2, 16-byte chunks (c%2)*4 .. +3
+  uint8_t* blk = pbuf + (c >> 1) * (BQ * 128) + row * 128;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int chunk = ((c & 1) << 2) + q;
+    uint4 pk;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h2 = __floats2half2_rn(p[q * 8 + 2 * i], p[q * 8 + 2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(blk + ((chunk ^ (row & 7)) << 4)) = pk;
+  }
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_constant__ CUtensorMap tm_vt,
+                        const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* q_full = bar;          // [2]
+  uint64_t* q_empty = bar + 2;     // [2]
+  uint64_t* kv_full = bar + 4;     // [2]
+  uint64_t* kv_empty = bar + 6;    // [2]
+  uint64_t* s_full = bar + 8;      // [2]
+  uint64_t* s_empty = bar + 10;    // [2]
+  uint64_t* p_full = bar + 12;     // [2]
+  uint64_t* p_empty = bar + 14;    // [2]
+  uint64_t* o_full = bar + 16;     // [2]
+  uint64_t* o_empty = bar + 18;    // [2]
+  uint64_t* drain = bar + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const NodeEntry nd = p.nodes[blockIdx.z];
+  const int g = blockIdx.y;                         // kv head
+  const int grp = p.H / p.KV;                       // query heads per kv head
+  const int qt = p.q_tiles - 1 - blockIdx.x;        // longest tiles first
+  const int q0 = qt * BQ;
+  const int ntiles = (min(p.Tp, q0 + BQ) + BKEY - 1) / BKEY;   // key tiles 0..qt
+  const int nsteps = grp * ntiles;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+      mbar_init(&kv_full[b], 1);
+      mbar_init(&kv_empty[b], 1);
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 4);
+      mbar_init(&p_full[b], 4);
+      mbar_init(&p_empty[b], 1);
+      mbar_init(&o_full[b], 1);
+      mbar_init(&o_empty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      bool ok = true;
+      uint32_t armed = 0;   // bits 0-1: Q buffers, 2-3: KV stages with loads in flight
+      for (int t = 0; t < nsteps && ok; ++t) {
+        const int hh = t / ntiles, j = t - hh * ntiles;
+        const int h = g * grp + hh;
+        if (j == 0) {
+          const int qb = hh & 1;
+          if (!mbar_wait(&q_empty[qb], ((hh >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&q_full[qb], Q_BYTES);
+          tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, h * HD, q0, nd.z);
+          armed |= 1u << qb;
+        }
+        const int st = t & 1;
+        if (!mbar_wait(&kv_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
+        tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
+        uint8_t* vt = smem + OFF_VT + st * VT_BYTES;
+        const int vt_outer = nd.z * p.KV + g;
+        tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
+        tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BYTES / 2, j * BKEY + 64, 0, vt_outer);
+        armed |= 4u << st;
+      }
+      if (!ok) {
+        atomicOr(p.err, 16u);
+        *abort_flag = 1;
+      }
+      if (*abort_flag) {   // let every issued copy land before the CTA exits
+        for (int b = 0; b < 2; ++b) {
+          const unsigned long long t0 = global_ns();
+          if (armed & (1u << b))
+            while (!mbar_try_wait(&q_full[b], 0) && !mbar_try_wait(&q_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
+          if (armed & (4u << b))
+            while (!mbar_try_wait(&kv_full[b], 0) && !mbar_try_wait(&kv_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
+      const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x 64 x 16
+      bool ok = true;
+      auto issue_s = [&](int t) -> bool {
+        const int hh = t / ntiles, j = t - hh * ntiles;
+        const int st = t & 1, qb = hh & 1;
+        if (j == 0 && !mbar_wait(&q_full[qb], (hh >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[st], (t >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&s_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
+        const uint32_t ka = smem_u32(smem + OFF_K + st * K_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          mma_f16(tmem_base + st * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+        mma_commit(&s_full[st]);
+        if (j == ntiles - 1) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
+        return true;
+      };
+      if (nsteps > 0) ok = issue_s(0);
+      for (int t = 0; t < nsteps && ok; ++t) {
+        if (t + 1 < nsteps && !issue_s(t + 1)) { ok = false; break; }
+        const int st = t & 1;
+        if (!mbar_wait(&p_full[st], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&o_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t pa = smem_u32(smem + OFF_P + st * P_BYTES);
+        const uint32_t va = smem_u32(smem + OFF_VT + st * VT_BYTES);
+#pragma unroll
+        for (int kb = 0; kb < BKEY / 64; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem_base + 2 * BKEY + st * HD, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
+                    sw128_desc(va + kb * (HD * 128) + kk * 32), idesc_o, (kb > 0 || kk > 0));
+        mma_commit(&o_full[st]);
+        mma_commit(&p_empty[st]);
+        mma_commit(&kv_empty[st]);
+      }
+      if (!ok) {
+        atomicOr(p.err, 32u);
+        *abort_flag = 1;
+      }
+      mma_commit(drain);
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(drain, 0)) {
+        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+      }
+    }
+  } else {
+    // ---------------- softmax / accumulation (warps 2..5, thread = query row) ----------------
+    const int quarter = warp & 3;
+    const int rloc = quarter * 32 + lane;
+    const int row = q0 + rloc;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    float m = -INFINITY, l = 0.f, corr_pend = 0.f, l_prev = 0.f;
+    float o[HD];
+#pragma unroll
+    for (int i = 0; i < HD; ++i) o[i] = 0.f;
+    bool ok = true;
+    // o <- o * corr + O_t (step t of the head in o), then release the O buffer
+    auto accumulate = [&](int t, float corr) -> bool {
+      const int st = t & 1;
+      const bool got = mbar_wait(&o_full[st], (t >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + lane_off + 2 * BKEY + st * HD + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], corr, v[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_empty[st]);
+      return true;
+    };
+    auto finalize = [&](int hh, float lsum) {
+      const int h = g * grp + hh;
+      if (row < p.Tp) {
+        const float inv = 1.f / lsum;
+        f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
+#pragma unroll
+        for (int q = 0; q < HD / 8; ++q) {
+          uint4 pk;
+          uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __half2 h2 = __floats2half2_rn(o[q * 8 + 2 * i] * inv, o[q * 8 + 2 * i + 1] * inv);
+            w[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          reinterpret_cast<uint4*>(dst)[q] = pk;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < HD; ++i) o[i] = 0.f;
+    };
+    for (int t = 0; t < nsteps && ok; ++t) {
+      const int hh = t / ntiles, j = t - hh * ntiles;
+      const int st = t & 1;
+      if (j == 0) {   // new head: its running max and sum start over
+        l_prev = l;
+        m = -INFINITY;
+        l = 0.f;
+      }
+      bool got = mbar_wait(&s_full[st], (t >> 1) & 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = tmem_base + lane_off + st * BKEY;
+      const bool diag = j == ntiles - 1;
+      const int k0 = j * BKEY;
+      // pass 1: row max of the scaled, masked scores
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < BKEY / 32; ++c) {
+        float v[32];
+        tmem_ld32(sbase + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool masked = diag && (k0 + c * 32 + i > row);
+          mx = fmaxf(mx, masked ? -INFINITY : v[i] * p.scale_log2);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float corr = exp2f(m - m_new);
+      got = mbar_wait(&p_empty[st], ((t >> 1) & 1) ^ 1, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      // pass 2: probabilities -> P (fp16, swizzled K-major rows of the O = P V operand)
+      uint8_t* pbuf = smem + OFF_P + st * P_BYTES;
+      float sum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < BKEY / 32; ++c) {
+        float v[32];
+        tmem_ld32(sbase + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool masked = diag && (k0 + c * 32 + i > row);
+          const float e = masked ? 0.f : exp2f(v[i] * p.scale_log2 - m_new);
+          v[i] = e;
+          sum += e;
+        }
+        store_p_chunk(pbuf, rloc, c, v);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_empty[st]);
+        mbar_arrive(&p_full[st]);
+      }
+      l = l * corr + sum;
+      m = m_new;
+      // accumulate the previous step's O (computed while this softmax ran)
+      if (t > 0) {
+        if (!accumulate(t - 1, corr_pend)) { ok = false; break; }
+        if (j == 0) finalize(hh - 1, l_prev);
+      }
+      corr_pend = corr;
+    }
+    if (ok && nsteps > 0) {
+      if (accumulate(nsteps - 1, corr_pend)) finalize(grp - 1, l);
+      else ok = false;
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.err, 64u);
+      *abort_flag = 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// 3-D tensor map over fp16 [outer][rows][inner], box = box_inner x box_rows,
+// rows pitch_rows apart per outer step, 128-byte swizzle, zero fill.
+cudaError_t make_map(CUtensorMap* map, const void* base, int inner, int rows, int outer, long long row_pitch_elems,
+                     long long outer_pitch_elems, int box_inner, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)row_pitch_elems * 2, (cuuint64_t)outer_pitch_elems * 2};
+  cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool attention_tc_supported(const Dims& dm) { return dm.bf16 && dm.hd == HD; }
+
+int attention_tc_vt_pitch(int Tp) { return (Tp + 7) / 8 * 8; }
+
+cudaError_t setup_attention_tc() {
+  if (!get_tensor_map_encoder()) return cudaErrorNotSupported;
+  return cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+}
+
+cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int slots, const void* qkv,
+                                const void* vt, void* out, unsigned* err, cudaStream_t st) {
+  if (!attention_tc_supported(dm)) return cudaErrorInvalidValue;
+  CUtensorMap tm_qk, tm_vt;
+  // Q and K tiles: [slot][Tp][nqkv], box 64 dims x 128 rows
+  cudaError_t e = make_map(&tm_qk, qkv, dm.nqkv, Tp, slots, dm.nqkv, (long long)Tp * dm.nqkv, HD, BQ);
+  if (e != cudaSuccess) return e;
+  // V^T tiles: [slot * KV + g][hd][pitch], box 64 keys x 64 dims
+  const int pitch = attention_tc_vt_pitch(Tp);
+  e = make_map(&tm_vt, vt, Tp, HD, slots * dm.KV, pitch, (long long)HD * pitch, 64, HD);
+  if (e != cudaSuccess) return e;
+  AttnParams p;
+  p.nodes = nodes;
+  p.Tp = Tp;
+  p.H = dm.H;
+  p.KV = dm.KV;
+  p.nqkv = dm.nqkv;
+  p.q_tiles = (Tp + BQ - 1) / BQ;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
+  p.out = (f16*)out;
+  p.err = err;
+  dim3 grid(p.q_tiles, dm.KV, n);
+  attention_tc_kernel<<<grid, NUM_THREADS, SMEM_TOTAL, st>>>(tm_qk, tm_vt, p);
+  return cudaGetLastError();
+}
+
+}  // namespace armt

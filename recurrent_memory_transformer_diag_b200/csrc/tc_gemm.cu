@@ -31,128 +31,18 @@
 
 #include "armt_internal.cuh"
 #include "tc_gemm.cuh"
+#include "tcgen05_ptx.cuh"
 
 namespace armt {
 
 namespace {
 
+using namespace tc;
+
 constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
 constexpr int EPI_WARPS = 8;           // two warps per TMEM lane quarter, each half of the columns
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase of `parity`; false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
-  }
-}
-
-__device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
-                                            int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, K-major operand, 128-byte swizzle:
-// rows of 128 bytes, 8-row groups 1024 bytes apart (SBO), LBO unused (1),
-// descriptor version 1 (sm_100), layout type 2 = SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
-  d |= (uint64_t)1 << 16;                 // LBO (16 B units)
-  d |= (uint64_t)(1024 >> 4) << 32;       // SBO (16 B units)
-  d |= (uint64_t)1 << 46;                 // version
-  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
-  return d;
-}
-
-// Instruction descriptor: D fp32, A/B both fp16 (format 0) or both bf16
-// (format 1), both K-major, shape 128 x N.
-__host__ __device__ constexpr uint32_t idesc_f16(int n, int ab_bf16) {
-  return (1u << 4) | ((uint32_t)ab_bf16 << 7) | ((uint32_t)ab_bf16 << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(BM >> 4) << 24);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 __device__ __forceinline__ void store_f16x32(f16* dst, const float* v) {
   // 32 values = 64 bytes: four 16-byte stores (dst 16-byte aligned)
@@ -339,6 +229,16 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
         store_act32(C + col1, v1, p.N - col1);
         if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+        if (p.vt && !rot) {
+          // value head: dims pc*32.. and hd/2 + pc*32.. of this row, transposed
+          const int vh = head - p.rope_heads;
+          f16* vt = p.vt + (((long long)slot * p.n_vheads + vh) * hd) * p.vt_pitch + row;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            vt[(long long)(pc * 32 + i) * p.vt_pitch] = __float2half_rn(v1[i]);
+            vt[(long long)(hd / 2 + pc * 32 + i) * p.vt_pitch] = __float2half_rn(v2[i]);
+          }
+        }
       }
     }
   } else if constexpr (EPI == TC_EPI_SWIGLU) {
@@ -466,7 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+            mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
                      (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
@@ -524,7 +424,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+}  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* ptr = nullptr;
@@ -535,6 +437,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   }
   return fn;
 }
+
+namespace {
 
 template <int BN, int EPI>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, int sm_count,
@@ -557,7 +461,7 @@ cudaError_t configure() {
 cudaError_t setup_tc_gemm() {
   static bool done = false;
   if (done) return cudaSuccess;
-  if (!get_encode_fn()) return cudaErrorNotSupported;
+  if (!get_tensor_map_encoder()) return cudaErrorNotSupported;
   cudaError_t e = configure<256, TC_EPI_F32>();
   if (e == cudaSuccess) e = configure<128, TC_EPI_F32>();
   if (e == cudaSuccess) e = configure<64, TC_EPI_F32>();
@@ -574,7 +478,7 @@ cudaError_t setup_tc_gemm() {
 // box_rows x 1, 128-byte swizzle, zero fill out of bounds.
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows, int outer, int box_inner,
                          int box_rows, int pitch_rows, bool is_bf16) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode_fn();
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   if (pitch_rows <= 0) pitch_rows = rows;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
@@ -589,7 +493,7 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows
 
 bool tc_gemm_supported(int m, int n, int k) {
   (void)m;
-  return k % 8 == 0 && n % 16 == 0 && get_encode_fn() != nullptr;
+  return k % 8 == 0 && n % 16 == 0 && get_tensor_map_encoder() != nullptr;
 }
 
 int tc_pick_bn(int n) { return n >= 256 ? 256 : (n >= 128 ? 128 : 64); }

@@ -26,6 +26,9 @@ struct TcGemmParams {
   float* h; long long h_slot_stride; int ldh;
   const float* rowscale; long long rs_slot_stride;
   const float2* rope; int rope_half; int rope_heads; int head_dim;
+  // QKV epilogue: also write the value heads (heads >= rope_heads) transposed,
+  // vt[slot][head - rope_heads][dim][row] with rows vt_pitch apart (optional)
+  f16* vt; int vt_pitch; int n_vheads;
   int f_out;                // SWIGLU: number of valid output features
   // RMSNorm folded into the GEMMs.  Residual epilogues write, per row and per
   // half n-tile, the partial sum of squares of the new residual over those
