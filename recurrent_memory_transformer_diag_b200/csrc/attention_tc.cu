@@ -236,13 +236,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool got = mbar_wait(&o_full[st], (t >> 1) & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) return false;
       tc_fence_after();
+      uint32_t orr[HD];
+      tmem_ld64_nowait(tmem_base + lane_off + 2 * BKEY + st * HD, orr);
+      tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < HD / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem_base + lane_off + 2 * BKEY + st * HD + c * 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[c * 32 + i] = fmaf(o[c * 32 + i], corr, v[i]);
-      }
+      for (int i = 0; i < HD; ++i) o[i] = fmaf(o[i], corr, __uint_as_float(orr[i]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_empty[st]);
@@ -282,33 +280,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t sbase = tmem_base + lane_off + st * BKEY;
       const bool diag = j == ntiles - 1;
       const int k0 = j * BKEY;
-      // pass 1: row max of the scaled, masked scores
+      // the whole score row in registers: two x64 loads, one wait
+      uint32_t sr[BKEY];
+      tmem_ld64_nowait(sbase, sr);
+      tmem_ld64_nowait(sbase + 64, sr + 64);
+      tmem_wait_ld();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < BKEY / 32; ++c) {
-        float v[32];
-        tmem_ld32(sbase + c * 32, v);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool masked = diag && (k0 + c * 32 + i > row);
-          mx = fmaxf(mx, masked ? -INFINITY : v[i] * p.scale_log2);
-        }
+      for (int i = 0; i < BKEY; ++i) {
+        float v = __uint_as_float(sr[i]);
+        if (diag && k0 + i > row) v = -INFINITY;
+        sr[i] = __float_as_uint(v);
+        mx = fmaxf(mx, v);
       }
-      const float m_new = fmaxf(m, mx);
+      const float m_new = fmaxf(m, mx * p.scale_log2);   // scale > 0: max commutes with it
       const float corr = exp2f(m - m_new);
       got = mbar_wait(&p_empty[st], ((t >> 1) & 1) ^ 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      // pass 2: probabilities -> P (fp16, swizzled K-major rows of the O = P V operand)
+      // probabilities -> P (fp16, swizzled K-major rows of the O = P V operand)
       uint8_t* pbuf = smem + OFF_P + st * P_BYTES;
       float sum = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < BKEY / 32; ++c) {
         float v[32];
-        tmem_ld32(sbase + c * 32, v);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const bool masked = diag && (k0 + c * 32 + i > row);
-          const float e = masked ? 0.f : exp2f(v[i] * p.scale_log2 - m_new);
+          const float e = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_new));
           v[i] = e;
           sum += e;
         }

@@ -120,8 +120,40 @@ constexpr int MEMW_ROWS_PER_BLOCK = 64;
 // value past the fp16 range sets the error word).
 // grid (ceil(d / MEMW_ROWS_PER_BLOCK), nodes), 8 warps, one A row per warp per
 // iteration; phi, G and coef are staged once per block.
-// M <= 32: lane j carries memory row j through the recurrence.
-template <int MAXC>
+// Transposed warp reduction of MT per-lane partial sums: afterwards lane l
+// holds the warp-wide total of index j = l >> (5 - log2 MT).  Each stage
+// halves the values a lane keeps and exchanges the other half with its
+// partner (MT - 1 shuffles in the halving stages instead of 5 per index).
+template <int K, int O, int MT>
+__device__ __forceinline__ void transpose_stage(float (&v)[MT], int lane) {
+  if constexpr (O >= 1) {
+    if constexpr (K > 1) {
+      const bool upper = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < K / 2; ++i) {
+        const float send = upper ? v[i] : v[i + K / 2];
+        const float keep = upper ? v[i + K / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, O);
+      }
+      transpose_stage<K / 2, O / 2, MT>(v, lane);
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], O);
+      transpose_stage<1, O / 2, MT>(v, lane);
+    }
+  }
+}
+
+template <int MT>
+__device__ __forceinline__ float transpose_reduce(float (&v)[MT], int lane) {
+  transpose_stage<MT, 16, MT>(v, lane);
+  return v[0];
+}
+
+template <int MT>
+constexpr int log2_const() { return MT <= 1 ? 0 : 1 + log2_const<MT / 2>(); }
+
+// M <= MT <= 32: lane j carries memory row j through the recurrence.
+template <int MAXC, int MT>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
                                                           const float* gram, const float* coef, float* A_state,
@@ -130,7 +162,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   float* ph = sh;                    // [M][P]
   float* G = ph + M * P;             // [M][M]
   float* cf = G + M * M;             // [M]
-  float* dots = cf + M;              // [8][M]  a . phi_j, then delta_j
+  float* dots = cf + M;              // [8][M]  delta_j per warp
   const NodeEntry nd = nodes[blockIdx.y];
   const int slot = nd.z, layer = nd.y;
   for (int e = threadIdx.x; e < M * P; e += blockDim.x) ph[e] = phik[(long long)slot * M * P + e];
@@ -140,30 +172,35 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* dl = dots + warp * M;
   bool over = false;
+  constexpr int SHIFT = 5 - log2_const<MT>();
+  const float cj = lane < M ? cf[lane] : 0.f;
   const int i_end = min(d, (blockIdx.x + 1) * MEMW_ROWS_PER_BLOCK);
   for (int i = blockIdx.x * MEMW_ROWS_PER_BLOCK + warp; i < i_end; i += 8) {
     float* Arow = A_state + ((long long)layer * d + i) * P;
+    const float vj = lane < M ? kv[((long long)slot * M + lane) * (dk + d) + dk + i] : 0.f;
     float a[MAXC];
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       a[c] = p < P ? Arow[p] : 0.f;
     }
-    // lane j (< M <= 32) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
-    float s = 0.f;
-    for (int j = 0; j < M; ++j) {
-      const float* pj = ph + j * P;
-      float dot = 0.f;
+    // a . phi_j for all j at once (independent accumulators), then one
+    // transposed reduction
+    float part[MT];
 #pragma unroll
-      for (int c = 0; c < MAXC; ++c) {
-        const int p = lane + 32 * c;
-        if (p < P) dot = fmaf(a[c], pj[p], dot);
+    for (int j = 0; j < MT; ++j) part[j] = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+      const int p = lane + 32 * c;
+      if (p < P) {
+#pragma unroll
+        for (int j = 0; j < MT; ++j)
+          if (j < M) part[j] = fmaf(a[c], ph[j * P + p], part[j]);
       }
-      dot = warp_sum_m(dot);
-      if (lane == j) s = dot;
     }
-    const float vj = lane < M ? kv[((long long)slot * M + lane) * (dk + d) + dk + i] : 0.f;
-    const float cj = lane < M ? cf[lane] : 0.f;
+    const float tot = transpose_reduce<MT>(part, lane);
+    // lane j (< M) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
+    float s = __shfl_sync(0xffffffffu, tot, (lane << SHIFT) & 31);
     for (int j = 0; j < M; ++j) {
       // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
       const float dj = __shfl_sync(0xffffffffu, vj - s * cj, j);
@@ -199,14 +236,22 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
   dim3 grid((dm.d + MEMW_ROWS_PER_BLOCK - 1) / MEMW_ROWS_PER_BLOCK, n);
   const size_t sh = memw_update_smem(dm);
   const int chunks = (dm.P + 31) / 32;
-#define ARMT_MEMW_CASE(C)                                                                              \
-  memw_update_kernel<C><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
-                                               A_state, (f16*)a_act, err);
-  if (chunks <= 4) ARMT_MEMW_CASE(4)
-  else if (chunks <= 12) ARMT_MEMW_CASE(12)
-  else if (chunks <= 24) ARMT_MEMW_CASE(24)
-  else if (chunks <= 32) ARMT_MEMW_CASE(32)
+#define ARMT_MEMW_CASE(C, MT)                                                                             \
+  memw_update_kernel<C, MT><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
+                                                   A_state, (f16*)a_act, err);
+#define ARMT_MEMW_M(C)                  \
+  {                                     \
+    if (dm.M <= 4) ARMT_MEMW_CASE(C, 4) \
+    else if (dm.M <= 16) ARMT_MEMW_CASE(C, 16) \
+    else ARMT_MEMW_CASE(C, 32)          \
+  }
+  if (dm.M > 32) return cudaErrorInvalidValue;
+  if (chunks <= 4) ARMT_MEMW_M(4)
+  else if (chunks <= 12) ARMT_MEMW_M(12)
+  else if (chunks <= 24) ARMT_MEMW_M(24)
+  else if (chunks <= 32) ARMT_MEMW_M(32)
   else return cudaErrorInvalidValue;
+#undef ARMT_MEMW_M
 #undef ARMT_MEMW_CASE
   return cudaGetLastError();
 }
@@ -215,10 +260,13 @@ cudaError_t setup_memory_kernels(const Dims& dm) {
   const int sh = (int)memw_update_smem(dm);
   cudaError_t e = cudaSuccess;
   if (sh > 48 * 1024) {
-    e = cudaFuncSetAttribute(memw_update_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(memw_update_kernel<12>, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(memw_update_kernel<24>, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(memw_update_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
+    auto set = [&](auto fn) {
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
+    };
+    set(memw_update_kernel<4, 4>); set(memw_update_kernel<4, 16>); set(memw_update_kernel<4, 32>);
+    set(memw_update_kernel<12, 4>); set(memw_update_kernel<12, 16>); set(memw_update_kernel<12, 32>);
+    set(memw_update_kernel<24, 4>); set(memw_update_kernel<24, 16>); set(memw_update_kernel<24, 32>);
+    set(memw_update_kernel<32, 4>); set(memw_update_kernel<32, 16>); set(memw_update_kernel<32, 32>);
   }
   return e;
 }
