@@ -36,10 +36,11 @@ constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
 constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
 constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB (two 64-key blocks of 8 KB)
 constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
+constexpr int KV_STAGES = 3;
 constexpr int OFF_Q = 0;                          // 2 buffers
-constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // 2 stages
-constexpr int OFF_VT = OFF_K + 2 * K_BYTES;       // 2 stages
-constexpr int OFF_P = OFF_VT + 2 * VT_BYTES;      // 2 buffers
+constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // KV_STAGES stages
+constexpr int OFF_VT = OFF_K + KV_STAGES * K_BYTES;
+constexpr int OFF_P = OFF_VT + KV_STAGES * VT_BYTES;   // 2 buffers
 constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
 constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
 constexpr int TMEM_COLS = 512;                    // S[2] at 0, 128; O[2] at 256, 320
@@ -80,16 +81,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bar;          // [2]
   uint64_t* q_empty = bar + 2;     // [2]
-  uint64_t* kv_full = bar + 4;     // [2]
-  uint64_t* kv_empty = bar + 6;    // [2]
-  uint64_t* s_full = bar + 8;      // [2]
-  uint64_t* s_empty = bar + 10;    // [2]
-  uint64_t* p_full = bar + 12;     // [2]
-  uint64_t* p_empty = bar + 14;    // [2]
-  uint64_t* o_full = bar + 16;     // [2]
-  uint64_t* o_empty = bar + 18;    // [2]
-  uint64_t* drain = bar + 20;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
+  uint64_t* kv_full = bar + 4;     // [KV_STAGES]
+  uint64_t* kv_empty = bar + 8;    // [KV_STAGES]
+  uint64_t* s_full = bar + 12;     // [2]
+  uint64_t* s_empty = bar + 14;    // [2]
+  uint64_t* p_full = bar + 16;     // [2]
+  uint64_t* p_empty = bar + 18;    // [2]
+  uint64_t* o_full = bar + 20;     // [2]
+  uint64_t* o_empty = bar + 22;    // [2]
+  uint64_t* drain = bar + 24;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 25);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,11 +103,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int nsteps = grp * ntiles;
 
   if (threadIdx.x == 0) {
+    for (int b = 0; b < KV_STAGES; ++b) {
+      mbar_init(&kv_full[b], 1);
+      mbar_init(&kv_empty[b], 1);
+    }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
-      mbar_init(&kv_full[b], 1);
-      mbar_init(&kv_empty[b], 1);
       mbar_init(&s_full[b], 1);
       mbar_init(&s_empty[b], 4);
       mbar_init(&p_full[b], 4);
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       bool ok = true;
-      uint32_t armed = 0;   // bits 0-1: Q buffers, 2-3: KV stages with loads in flight
+      uint32_t armed = 0;   // bits 0-1: Q buffers, 2..: KV stages with loads in flight
       for (int t = 0; t < nsteps && ok; ++t) {
         const int hh = t / ntiles, j = t - hh * ntiles;
         const int h = g * grp + hh;
@@ -144,8 +147,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, h * HD, q0, nd.z);
           armed |= 1u << qb;
         }
-        const int st = t & 1;
-        if (!mbar_wait(&kv_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+        const int st = t % KV_STAGES;
+        if (!mbar_wait(&kv_empty[st], ((t / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
         tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
         uint8_t* vt = smem + OFF_VT + st * VT_BYTES;
@@ -159,13 +162,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *abort_flag = 1;
       }
       if (*abort_flag) {   // let every issued copy land before the CTA exits
-        for (int b = 0; b < 2; ++b) {
-          const unsigned long long t0 = global_ns();
+        const unsigned long long t0 = global_ns();
+        for (int b = 0; b < 2; ++b)
           if (armed & (1u << b))
             while (!mbar_try_wait(&q_full[b], 0) && !mbar_try_wait(&q_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
+        for (int b = 0; b < KV_STAGES; ++b)
           if (armed & (4u << b))
             while (!mbar_try_wait(&kv_full[b], 0) && !mbar_try_wait(&kv_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
-        }
       }
     }
   } else if (warp == 1) {
@@ -176,13 +179,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       auto issue_s = [&](int t) -> bool {
         const int hh = t / ntiles, j = t - hh * ntiles;
-        const int st = t & 1, qb = hh & 1;
+        const int st = t & 1, qb = hh & 1, ks = t % KV_STAGES;
         if (j == 0 && !mbar_wait(&q_full[qb], (hh >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&kv_full[st], (t >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[ks], (t / KV_STAGES) & 1, abort_flag)) return false;
         if (!mbar_wait(&s_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
-        const uint32_t ka = smem_u32(smem + OFF_K + st * K_BYTES);
+        const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
           mma_f16(tmem_base + st * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&o_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + st * P_BYTES);
-        const uint32_t va = smem_u32(smem + OFF_VT + st * VT_BYTES);
+        const uint32_t va = smem_u32(smem + OFF_VT + (t % KV_STAGES) * VT_BYTES);
 #pragma unroll
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
@@ -207,7 +210,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     sw128_desc(va + kb * (HD * 128) + kk * 32), idesc_o, (kb > 0 || kk > 0));
         mma_commit(&o_full[st]);
         mma_commit(&p_empty[st]);
-        mma_commit(&kv_empty[st]);
+        mma_commit(&kv_empty[t % KV_STAGES]);
       }
       if (!ok) {
         atomicOr(p.err, 32u);

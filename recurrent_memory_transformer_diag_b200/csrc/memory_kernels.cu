@@ -152,7 +152,9 @@ __device__ __forceinline__ float transpose_reduce(float (&v)[MT], int lane) {
 template <int MT>
 constexpr int log2_const() { return MT <= 1 ? 0 : 1 + log2_const<MT / 2>(); }
 
-// M <= MT <= 32: lane j carries memory row j through the recurrence.
+// M <= MT <= 32: lane j carries memory row j through the recurrence.  A warp
+// updates two rows of A per pass (rows i and i + 8 of its block's range), so
+// every phi element read from shared memory serves both rows.
 template <int MAXC, int MT>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   float* ph = sh;                    // [M][P]
   float* G = ph + M * P;             // [M][M]
   float* cf = G + M * M;             // [M]
-  float* dots = cf + M;              // [8][M]  delta_j per warp
+  float* dots = cf + M;              // [8][2][M]  delta_j per warp and row
   const NodeEntry nd = nodes[blockIdx.y];
   const int slot = nd.z, layer = nd.y;
   for (int e = threadIdx.x; e < M * P; e += blockDim.x) ph[e] = phik[(long long)slot * M * P + e];
@@ -170,54 +172,84 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   for (int e = threadIdx.x; e < M; e += blockDim.x) cf[e] = coef[(long long)slot * M + e];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* dl = dots + warp * M;
+  float* dl0 = dots + warp * 2 * M;
+  float* dl1 = dl0 + M;
   bool over = false;
   constexpr int SHIFT = 5 - log2_const<MT>();
   const float cj = lane < M ? cf[lane] : 0.f;
-  const int i_end = min(d, (blockIdx.x + 1) * MEMW_ROWS_PER_BLOCK);
-  for (int i = blockIdx.x * MEMW_ROWS_PER_BLOCK + warp; i < i_end; i += 8) {
-    float* Arow = A_state + ((long long)layer * d + i) * P;
-    const float vj = lane < M ? kv[((long long)slot * M + lane) * (dk + d) + dk + i] : 0.f;
-    float a[MAXC];
+  const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
+  const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
+  for (int i0 = i_begin + warp; i0 < i_end; i0 += 16) {
+    const int i1 = i0 + 8;
+    const bool has1 = i1 < i_end;
+    float* Arow0 = A_state + ((long long)layer * d + i0) * P;
+    float* Arow1 = A_state + ((long long)layer * d + (has1 ? i1 : i0)) * P;
+    const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+    const float v0 = lane < M ? kvj[i0] : 0.f;
+    const float v1 = (lane < M && has1) ? kvj[i1] : 0.f;
+    float a0[MAXC], a1[MAXC];
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
-      a[c] = p < P ? Arow[p] : 0.f;
+      a0[c] = p < P ? Arow0[p] : 0.f;
+      a1[c] = (p < P && has1) ? Arow1[p] : 0.f;
     }
-    // a . phi_j for all j at once (independent accumulators), then one
-    // transposed reduction
-    float part[MT];
+    float part0[MT], part1[MT];
 #pragma unroll
-    for (int j = 0; j < MT; ++j) part[j] = 0.f;
+    for (int j = 0; j < MT; ++j) part0[j] = part1[j] = 0.f;
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       if (p < P) {
 #pragma unroll
-        for (int j = 0; j < MT; ++j)
-          if (j < M) part[j] = fmaf(a[c], ph[j * P + p], part[j]);
+        for (int j = 0; j < MT; ++j) {
+          if (j < M) {
+            const float f = ph[j * P + p];
+            part0[j] = fmaf(a0[c], f, part0[j]);
+            part1[j] = fmaf(a1[c], f, part1[j]);
+          }
+        }
       }
     }
-    const float tot = transpose_reduce<MT>(part, lane);
+    const float tot0 = transpose_reduce<MT>(part0, lane);
+    const float tot1 = transpose_reduce<MT>(part1, lane);
     // lane j (< M) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
-    float s = __shfl_sync(0xffffffffu, tot, (lane << SHIFT) & 31);
+    float s0 = __shfl_sync(0xffffffffu, tot0, (lane << SHIFT) & 31);
+    float s1 = __shfl_sync(0xffffffffu, tot1, (lane << SHIFT) & 31);
     for (int j = 0; j < M; ++j) {
       // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
-      const float dj = __shfl_sync(0xffffffffu, vj - s * cj, j);
-      if (lane == j) dl[j] = dj;
-      if (lane > j && lane < M) s = fmaf(dj, G[j * M + lane], s);
+      const float d0 = __shfl_sync(0xffffffffu, v0 - s0 * cj, j);
+      const float d1 = __shfl_sync(0xffffffffu, v1 - s1 * cj, j);
+      if (lane == j) {
+        dl0[j] = d0;
+        dl1[j] = d1;
+      }
+      if (lane > j && lane < M) {
+        const float gj = G[j * M + lane];
+        s0 = fmaf(d0, gj, s0);
+        s1 = fmaf(d1, gj, s1);
+      }
     }
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       if (p < P) {
-        float acc = a[c];
-        for (int j = 0; j < M; ++j) acc = fmaf(dl[j], ph[j * P + p], acc);
-        Arow[p] = acc;
+        float acc0 = a0[c], acc1 = a1[c];
+        for (int j = 0; j < M; ++j) {
+          const float f = ph[j * P + p];
+          acc0 = fmaf(dl0[j], f, acc0);
+          acc1 = fmaf(dl1[j], f, acc1);
+        }
+        Arow0[p] = acc0;
+        if (has1) Arow1[p] = acc1;
         if (a_act) {
-          a_act[((long long)layer * d + i) * P + p] = __float2half_rn(acc);
-          over |= fabsf(acc) > 65504.f;
+          a_act[((long long)layer * d + i0) * P + p] = __float2half_rn(acc0);
+          over |= fabsf(acc0) > 65504.f;
+          if (has1) {
+            a_act[((long long)layer * d + i1) * P + p] = __float2half_rn(acc1);
+            over |= fabsf(acc1) > 65504.f;
+          }
         }
       }
     }
@@ -227,7 +259,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
 }
 
 static size_t memw_update_smem(const Dims& dm) {
-  return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 8 * dm.M) * sizeof(float);
+  return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 16 * dm.M) * sizeof(float);
 }
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
