@@ -8,17 +8,21 @@
 // attention).  Each node attends only over the T' rows of its own segment
 // plus memory tokens, causally.
 //
-// Per step (query head h, key tile j of 128 keys):
-//   MMA  S = Q K_j^T        (M=128 queries, N=128 keys, K=64)  -> TMEM S[j%2]
-//   softmax (warps 2..5, one thread per query row): row max, p = exp2(s - m),
-//        P (fp16) -> shared memory in the K-major swizzled operand layout
-//   MMA  O_j = P V_j        (M=128, N=64 dims, K=128 keys)      -> TMEM O[j%2]
-//   softmax warps: o = o * exp2(m_old - m_new) + O_j in registers
-// S of step t+1 is issued before O of step t, so the tensor core works on the
-// next tile while the softmax warps work on this one.  V is read as V^T
-// (written transposed by the QKV epilogue) so that every operand is K-major.
-// All mbarrier waits are bounded; on timeout the kernel sets the error word,
-// drains its copies and MMAs, frees TMEM and exits.
+// Two softmax warpgroups (A: warps 2..5, B: warps 6..9; one thread per query
+// row) take the even and the odd query heads of the group, so two heads are
+// in flight and share every K/V tile.  Per key tile j and warpgroup w:
+//   MMA  S_w = Q_w K_j^T          (M=128 queries, N=128 keys, K=64) -> TMEM
+//   softmax: row max, p = exp2(s - m) as fp16 P_w in shared memory (K-major,
+//            128-byte swizzle)
+//   MMA  O_w += P_w V_j           (M=128, N=64, K=128 keys), O_w stays in TMEM
+// The running max m is only raised when a row's max grows by more than 8 (in
+// log2 units): then that row of O_w is rescaled in TMEM; otherwise the stale
+// max is kept (p <= 2^8 fits fp16 and the row sum uses the same max, so the
+// result is exact).  The MMA warp interleaves O_A(j), S_A(j+1), O_B(j),
+// S_B(j+1) so one warpgroup's softmax overlaps the other's tensor work.  V is
+// read as V^T (written transposed by the QKV epilogue): every operand is
+// K-major.  All mbarrier waits are bounded; on timeout the kernel sets the
+// error word, drains its copies and MMAs, frees TMEM and exits.
 #include "armt_internal.cuh"
 #include "tcgen05_ptx.cuh"
 
@@ -31,19 +35,20 @@ using namespace tc;
 constexpr int HD = 64;
 constexpr int BQ = 128;                 // query rows per tile
 constexpr int BKEY = 128;               // keys per tile
-constexpr int NUM_THREADS = 192;        // warp 0 TMA, warp 1 MMA, warps 2..5 softmax
+constexpr int NUM_THREADS = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (2 warpgroups)
 constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
 constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
 constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB (two 64-key blocks of 8 KB)
 constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
-constexpr int KV_STAGES = 3;
-constexpr int OFF_Q = 0;                          // 2 buffers
-constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;        // KV_STAGES stages
+constexpr int KV_STAGES = 2;
+constexpr int OFF_Q = 0;                               // [2 warpgroups][2 buffers]
+constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // KV_STAGES stages
 constexpr int OFF_VT = OFF_K + KV_STAGES * K_BYTES;
-constexpr int OFF_P = OFF_VT + KV_STAGES * VT_BYTES;   // 2 buffers
+constexpr int OFF_P = OFF_VT + KV_STAGES * VT_BYTES;   // [2 warpgroups]
 constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
 constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
-constexpr int TMEM_COLS = 512;                    // S[2] at 0, 128; O[2] at 256, 320
+constexpr int TMEM_COLS = 512;          // S_A 0, S_B 128, O_A 256, O_B 320
+constexpr float RESCALE_THRESHOLD = 8.f;
 
 struct AttnParams {
   const NodeEntry* nodes;
@@ -79,18 +84,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bar;          // [2]
-  uint64_t* q_empty = bar + 2;     // [2]
-  uint64_t* kv_full = bar + 4;     // [KV_STAGES]
-  uint64_t* kv_empty = bar + 8;    // [KV_STAGES]
-  uint64_t* s_full = bar + 12;     // [2]
-  uint64_t* s_empty = bar + 14;    // [2]
-  uint64_t* p_full = bar + 16;     // [2]
-  uint64_t* p_empty = bar + 18;    // [2]
-  uint64_t* o_full = bar + 20;     // [2]
-  uint64_t* o_empty = bar + 22;    // [2]
-  uint64_t* drain = bar + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 25);
+  uint64_t* q_full = bar;          // [w][2]
+  uint64_t* q_empty = bar + 4;     // [w][2]
+  uint64_t* kv_full = bar + 8;     // [KV_STAGES]
+  uint64_t* kv_empty = bar + 10;   // [KV_STAGES]
+  uint64_t* s_full = bar + 12;     // [w]
+  uint64_t* s_empty = bar + 14;    // [w]
+  uint64_t* p_full = bar + 16;     // [w]
+  uint64_t* o_full = bar + 18;     // [w]
+  uint64_t* drain = bar + 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -100,22 +103,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int qt = p.q_tiles - 1 - blockIdx.x;        // longest tiles first
   const int q0 = qt * BQ;
   const int ntiles = (min(p.Tp, q0 + BQ) + BKEY - 1) / BKEY;   // key tiles 0..qt
-  const int nsteps = grp * ntiles;
+  const int heads_a = (grp + 1) / 2, heads_b = grp / 2;   // warpgroup A: even heads, B: odd heads
+  const int nA = heads_a * ntiles, nB = heads_b * ntiles;
 
   if (threadIdx.x == 0) {
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(&q_full[b], 1);
+      mbar_init(&q_empty[b], 1);
+    }
     for (int b = 0; b < KV_STAGES; ++b) {
       mbar_init(&kv_full[b], 1);
       mbar_init(&kv_empty[b], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&q_full[b], 1);
-      mbar_init(&q_empty[b], 1);
-      mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 4);
-      mbar_init(&p_full[b], 4);
-      mbar_init(&p_empty[b], 1);
-      mbar_init(&o_full[b], 1);
-      mbar_init(&o_empty[b], 4);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&s_empty[w], 4);
+      mbar_init(&p_full[w], 4);
+      mbar_init(&o_full[w], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -134,18 +138,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer: per step t, the warpgroups' Q when a head starts, then K_j, V_j^T
       bool ok = true;
-      uint32_t armed = 0;   // bits 0-1: Q buffers, 2..: KV stages with loads in flight
-      for (int t = 0; t < nsteps && ok; ++t) {
-        const int hh = t / ntiles, j = t - hh * ntiles;
-        const int h = g * grp + hh;
+      uint32_t armed = 0;   // bits 0-3: Q buffers, 4..: KV stages with loads in flight
+      for (int t = 0; t < nA && ok; ++t) {
+        const int k = t / ntiles, j = t - k * ntiles;
         if (j == 0) {
-          const int qb = hh & 1;
-          if (!mbar_wait(&q_empty[qb], ((hh >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&q_full[qb], Q_BYTES);
-          tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, h * HD, q0, nd.z);
-          armed |= 1u << qb;
+          for (int w = 0; w < 2; ++w) {
+            if (k >= (w == 0 ? heads_a : heads_b)) continue;
+            const int qb = w * 2 + (k & 1);
+            if (!mbar_wait(&q_empty[qb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            mbar_expect_tx(&q_full[qb], Q_BYTES);
+            tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * k) * HD, q0, nd.z);
+            armed |= 1u << qb;
+          }
+          if (!ok) break;
         }
         const int st = t % KV_STAGES;
         if (!mbar_wait(&kv_empty[st], ((t / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int vt_outer = nd.z * p.KV + g;
         tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
         tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BYTES / 2, j * BKEY + 64, 0, vt_outer);
-        armed |= 4u << st;
+        armed |= 16u << st;
       }
       if (!ok) {
         atomicOr(p.err, 16u);
@@ -163,11 +170,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (*abort_flag) {   // let every issued copy land before the CTA exits
         const unsigned long long t0 = global_ns();
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < 4; ++b)
           if (armed & (1u << b))
             while (!mbar_try_wait(&q_full[b], 0) && !mbar_try_wait(&q_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
         for (int b = 0; b < KV_STAGES; ++b)
-          if (armed & (4u << b))
+          if (armed & (16u << b))
             while (!mbar_try_wait(&kv_full[b], 0) && !mbar_try_wait(&kv_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
       }
     }
@@ -176,41 +183,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
       const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x 64 x 16
-      bool ok = true;
-      auto issue_s = [&](int t) -> bool {
-        const int hh = t / ntiles, j = t - hh * ntiles;
-        const int st = t & 1, qb = hh & 1, ks = t % KV_STAGES;
-        if (j == 0 && !mbar_wait(&q_full[qb], (hh >> 1) & 1, abort_flag)) return false;
+      auto issue_s = [&](int w, int t) -> bool {
+        const int k = t / ntiles, j = t - k * ntiles;
+        const int qb = w * 2 + (k & 1), ks = t % KV_STAGES;
+        if (j == 0 && !mbar_wait(&q_full[qb], (k >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(&kv_full[ks], (t / KV_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(&s_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) return false;
+        if (!mbar_wait(&s_empty[w], (t & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
         const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
-          mma_f16(tmem_base + st * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
-        mma_commit(&s_full[st]);
+          mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+        mma_commit(&s_full[w]);
         if (j == ntiles - 1) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
         return true;
       };
-      if (nsteps > 0) ok = issue_s(0);
-      for (int t = 0; t < nsteps && ok; ++t) {
-        if (t + 1 < nsteps && !issue_s(t + 1)) { ok = false; break; }
-        const int st = t & 1;
-        if (!mbar_wait(&p_full[st], (t >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&o_empty[st], ((t >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+      auto issue_o = [&](int w, int t) -> bool {
+        const int j = t % ntiles;
+        if (!mbar_wait(&p_full[w], t & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(smem + OFF_P + st * P_BYTES);
+        const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
         const uint32_t va = smem_u32(smem + OFF_VT + (t % KV_STAGES) * VT_BYTES);
 #pragma unroll
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem_base + 2 * BKEY + st * HD, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
-                    sw128_desc(va + kb * (HD * 128) + kk * 32), idesc_o, (kb > 0 || kk > 0));
-        mma_commit(&o_full[st]);
-        mma_commit(&p_empty[st]);
-        mma_commit(&kv_empty[t % KV_STAGES]);
+            mma_f16(tmem_base + 2 * BKEY + w * HD, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
+                    sw128_desc(va + kb * (HD * 128) + kk * 32), idesc_o, (j > 0 || kb > 0 || kk > 0));
+        mma_commit(&o_full[w]);
+        return true;
+      };
+      bool ok = nA > 0 ? issue_s(0, 0) : true;
+      if (ok && nB > 0) ok = issue_s(1, 0);
+      for (int t = 0; t < nA && ok; ++t) {
+        if (!issue_o(0, t)) { ok = false; break; }
+        if (t + 1 < nA && !issue_s(0, t + 1)) { ok = false; break; }
+        if (t < nB && !issue_o(1, t)) { ok = false; break; }
+        mma_commit(&kv_empty[t % KV_STAGES]);   // K_t, V_t no longer read once these MMAs finish
+        if (t + 1 < nB && !issue_s(1, t + 1)) { ok = false; break; }
       }
       if (!ok) {
         atomicOr(p.err, 32u);
@@ -223,71 +234,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    // ---------------- softmax / accumulation (warps 2..5, thread = query row) ----------------
+    // ---------------- softmax (warpgroup w, one thread per query row) ----------------
+    const int w = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;
     const int row = q0 + rloc;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    float m = -INFINITY, l = 0.f, corr_pend = 0.f, l_prev = 0.f;
-    float o[HD];
-#pragma unroll
-    for (int i = 0; i < HD; ++i) o[i] = 0.f;
+    const uint32_t s_tm = tmem_base + lane_off + w * BKEY;
+    const uint32_t o_tm = tmem_base + lane_off + 2 * BKEY + w * HD;
+    uint8_t* pbuf = smem + OFF_P + w * P_BYTES;
+    const int nw = (w == 0 ? heads_a : heads_b) * ntiles;
+    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    // o <- o * corr + O_t (step t of the head in o), then release the O buffer
-    auto accumulate = [&](int t, float corr) -> bool {
-      const int st = t & 1;
-      const bool got = mbar_wait(&o_full[st], (t >> 1) & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) return false;
-      tc_fence_after();
-      uint32_t orr[HD];
-      tmem_ld64_nowait(tmem_base + lane_off + 2 * BKEY + st * HD, orr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < HD; ++i) o[i] = fmaf(o[i], corr, __uint_as_float(orr[i]));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[st]);
-      return true;
-    };
-    auto finalize = [&](int hh, float lsum) {
-      const int h = g * grp + hh;
-      if (row < p.Tp) {
-        const float inv = 1.f / lsum;
-        f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
-#pragma unroll
-        for (int q = 0; q < HD / 8; ++q) {
-          uint4 pk;
-          uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __half2 h2 = __floats2half2_rn(o[q * 8 + 2 * i] * inv, o[q * 8 + 2 * i + 1] * inv);
-            w[i] = *reinterpret_cast<uint32_t*>(&h2);
-          }
-          reinterpret_cast<uint4*>(dst)[q] = pk;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < HD; ++i) o[i] = 0.f;
-    };
-    for (int t = 0; t < nsteps && ok; ++t) {
-      const int hh = t / ntiles, j = t - hh * ntiles;
-      const int st = t & 1;
-      if (j == 0) {   // new head: its running max and sum start over
-        l_prev = l;
-        m = -INFINITY;
+    for (int t = 0; t < nw && ok; ++t) {
+      const int k = t / ntiles, j = t - k * ntiles;
+      if (j == 0) {
+        m_used = -INFINITY;
         l = 0.f;
       }
-      bool got = mbar_wait(&s_full[st], (t >> 1) & 1, abort_flag);
+      bool got = mbar_wait(&s_full[w], t & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sbase = tmem_base + lane_off + st * BKEY;
+      uint32_t sr[BKEY];
+      tmem_ld64_nowait(s_tm, sr);
+      tmem_ld64_nowait(s_tm + 64, sr + 64);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[w]);   // S is in registers: the next S may be computed
       const bool diag = j == ntiles - 1;
       const int k0 = j * BKEY;
-      // the whole score row in registers: two x64 loads, one wait
-      uint32_t sr[BKEY];
-      tmem_ld64_nowait(sbase, sr);
-      tmem_ld64_nowait(sbase + 64, sr + 64);
-      tmem_wait_ld();
       float mx = -INFINITY;
 #pragma unroll
       for (int i = 0; i < BKEY; ++i) {
@@ -296,43 +272,75 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sr[i] = __float_as_uint(v);
         mx = fmaxf(mx, v);
       }
-      const float m_new = fmaxf(m, mx * p.scale_log2);   // scale > 0: max commutes with it
-      const float corr = exp2f(m - m_new);
-      got = mbar_wait(&p_empty[st], ((t >> 1) & 1) ^ 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      // probabilities -> P (fp16, swizzled K-major rows of the O = P V operand)
-      uint8_t* pbuf = smem + OFF_P + st * P_BYTES;
+      const float m_tile = mx * p.scale_log2;     // scale > 0: max commutes with it
+      float corr = 1.f;
+      bool rescale = false;
+      if (j == 0) {
+        m_used = m_tile;
+      } else if (m_tile > m_used + RESCALE_THRESHOLD) {
+        corr = exp2f(m_used - m_tile);
+        m_used = m_tile;
+        l *= corr;
+        rescale = true;
+      }
+      // O(t-1) must be complete: its MMA read the P buffer, and O may be rescaled below
+      if (t > 0) {
+        got = mbar_wait(&o_full[w], (t - 1) & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+      }
       float sum = 0.f;
 #pragma unroll
       for (int c = 0; c < BKEY / 32; ++c) {
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const float e = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_new));
+          const float e = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
           v[i] = e;
           sum += e;
         }
         store_p_chunk(pbuf, rloc, c, v);
       }
+      l += sum;
+      if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
+        uint32_t orr[HD];
+        tmem_ld64_nowait(o_tm, orr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
+        tmem_st64(o_tm, orr);
+        tmem_wait_st();
+      }
       tc_fence_before();
       fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&s_empty[st]);
-        mbar_arrive(&p_full[st]);
+      if (lane == 0) mbar_arrive(&p_full[w]);
+      if (j == ntiles - 1) {      // head done: wait for its last O, normalise, store
+        got = mbar_wait(&o_full[w], t & 1, abort_flag);
+        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t orr[HD];
+        tmem_ld64_nowait(o_tm, orr);
+        tmem_wait_ld();
+        tc_fence_before();
+        if (row < p.Tp) {
+          const int h = g * grp + w + 2 * k;
+          const float inv = 1.f / l;
+          f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
+#pragma unroll
+          for (int q = 0; q < HD / 8; ++q) {
+            uint4 pk;
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
+                                             __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
+              wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            reinterpret_cast<uint4*>(dst)[q] = pk;
+          }
+        }
       }
-      l = l * corr + sum;
-      m = m_new;
-      // accumulate the previous step's O (computed while this softmax ran)
-      if (t > 0) {
-        if (!accumulate(t - 1, corr_pend)) { ok = false; break; }
-        if (j == 0) finalize(hh - 1, l_prev);
-      }
-      corr_pend = corr;
-    }
-    if (ok && nsteps > 0) {
-      if (accumulate(nsteps - 1, corr_pend)) finalize(grp - 1, l);
-      else ok = false;
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, 64u);
