@@ -153,18 +153,21 @@ template <int MT>
 constexpr int log2_const() { return MT <= 1 ? 0 : 1 + log2_const<MT / 2>(); }
 
 // M <= MT <= 32: lane j carries memory row j through the recurrence.  A warp
-// updates two rows of A per pass (rows i and i + 8 of its block's range), so
-// every phi element read from shared memory serves both rows.
+// updates R rows of A per pass (rows i, i + 8, ..., i + 8 (R-1) of its block's
+// range), so every phi element read from shared memory serves R rows.
+constexpr int MEMW_R = 4;
+
 template <int MAXC, int MT>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                           const float* kv, const float* phik,
                                                           const float* gram, const float* coef, float* A_state,
                                                           f16* a_act, unsigned* err) {
+  constexpr int R = MEMW_R;
   extern __shared__ float sh[];
   float* ph = sh;                    // [M][P]
   float* G = ph + M * P;             // [M][M]
   float* cf = G + M * M;             // [M]
-  float* dots = cf + M;              // [8][2][M]  delta_j per warp and row
+  float* dots = cf + M;              // [8][R][M]  delta_j per warp and row
   const NodeEntry nd = nodes[blockIdx.y];
   const int slot = nd.z, layer = nd.y;
   for (int e = threadIdx.x; e < M * P; e += blockDim.x) ph[e] = phik[(long long)slot * M * P + e];
@@ -172,31 +175,35 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   for (int e = threadIdx.x; e < M; e += blockDim.x) cf[e] = coef[(long long)slot * M + e];
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* dl0 = dots + warp * 2 * M;
-  float* dl1 = dl0 + M;
+  float* dl = dots + warp * R * M;
   bool over = false;
   constexpr int SHIFT = 5 - log2_const<MT>();
   const float cj = lane < M ? cf[lane] : 0.f;
   const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
   const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
-  for (int i0 = i_begin + warp; i0 < i_end; i0 += 16) {
-    const int i1 = i0 + 8;
-    const bool has1 = i1 < i_end;
-    float* Arow0 = A_state + ((long long)layer * d + i0) * P;
-    float* Arow1 = A_state + ((long long)layer * d + (has1 ? i1 : i0)) * P;
-    const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
-    const float v0 = lane < M ? kvj[i0] : 0.f;
-    const float v1 = (lane < M && has1) ? kvj[i1] : 0.f;
-    float a0[MAXC], a1[MAXC];
+  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+  for (int i0 = i_begin + warp; i0 < i_end; i0 += 8 * R) {
+    float a[R][MAXC];
+    float v[R];
+    bool has[R];
 #pragma unroll
-    for (int c = 0; c < MAXC; ++c) {
-      const int p = lane + 32 * c;
-      a0[c] = p < P ? Arow0[p] : 0.f;
-      a1[c] = (p < P && has1) ? Arow1[p] : 0.f;
+    for (int r = 0; r < R; ++r) {
+      const int i = i0 + 8 * r;
+      has[r] = i < i_end;
+      const float* Arow = A_state + ((long long)layer * d + (has[r] ? i : i0)) * P;
+      v[r] = (lane < M && has[r]) ? kvj[i] : 0.f;
+#pragma unroll
+      for (int c = 0; c < MAXC; ++c) {
+        const int p = lane + 32 * c;
+        a[r][c] = (p < P && has[r]) ? Arow[p] : 0.f;
+      }
     }
-    float part0[MT], part1[MT];
+    // a_r . phi_j for all rows and j at once (independent accumulators)
+    float part[R][MT];
 #pragma unroll
-    for (int j = 0; j < MT; ++j) part0[j] = part1[j] = 0.f;
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < MT; ++j) part[r][j] = 0.f;
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
@@ -205,29 +212,27 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
         for (int j = 0; j < MT; ++j) {
           if (j < M) {
             const float f = ph[j * P + p];
-            part0[j] = fmaf(a0[c], f, part0[j]);
-            part1[j] = fmaf(a1[c], f, part1[j]);
+#pragma unroll
+            for (int r = 0; r < R; ++r) part[r][j] = fmaf(a[r][c], f, part[r][j]);
           }
         }
       }
     }
-    const float tot0 = transpose_reduce<MT>(part0, lane);
-    const float tot1 = transpose_reduce<MT>(part1, lane);
     // lane j (< M) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
-    float s0 = __shfl_sync(0xffffffffu, tot0, (lane << SHIFT) & 31);
-    float s1 = __shfl_sync(0xffffffffu, tot1, (lane << SHIFT) & 31);
+    float sv[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float tot = transpose_reduce<MT>(part[r], lane);
+      sv[r] = __shfl_sync(0xffffffffu, tot, (lane << SHIFT) & 31);
+    }
     for (int j = 0; j < M; ++j) {
       // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
-      const float d0 = __shfl_sync(0xffffffffu, v0 - s0 * cj, j);
-      const float d1 = __shfl_sync(0xffffffffu, v1 - s1 * cj, j);
-      if (lane == j) {
-        dl0[j] = d0;
-        dl1[j] = d1;
-      }
-      if (lane > j && lane < M) {
-        const float gj = G[j * M + lane];
-        s0 = fmaf(d0, gj, s0);
-        s1 = fmaf(d1, gj, s1);
+      const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
+        if (lane == j) dl[r * M + j] = dj;
+        sv[r] = fmaf(dj, gj, sv[r]);
       }
     }
     __syncwarp();
@@ -235,20 +240,22 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
     for (int c = 0; c < MAXC; ++c) {
       const int p = lane + 32 * c;
       if (p < P) {
-        float acc0 = a0[c], acc1 = a1[c];
+        float acc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = a[r][c];
         for (int j = 0; j < M; ++j) {
           const float f = ph[j * P + p];
-          acc0 = fmaf(dl0[j], f, acc0);
-          acc1 = fmaf(dl1[j], f, acc1);
+#pragma unroll
+          for (int r = 0; r < R; ++r) acc[r] = fmaf(dl[r * M + j], f, acc[r]);
         }
-        Arow0[p] = acc0;
-        if (has1) Arow1[p] = acc1;
-        if (a_act) {
-          a_act[((long long)layer * d + i0) * P + p] = __float2half_rn(acc0);
-          over |= fabsf(acc0) > 65504.f;
-          if (has1) {
-            a_act[((long long)layer * d + i1) * P + p] = __float2half_rn(acc1);
-            over |= fabsf(acc1) > 65504.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (!has[r]) continue;
+          const long long off = ((long long)layer * d + i0 + 8 * r) * P + p;
+          A_state[off] = acc[r];
+          if (a_act) {
+            a_act[off] = __float2half_rn(acc[r]);
+            over |= fabsf(acc[r]) > 65504.f;
           }
         }
       }
@@ -259,7 +266,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
 }
 
 static size_t memw_update_smem(const Dims& dm) {
-  return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 16 * dm.M) * sizeof(float);
+  return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 8 * MEMW_R * dm.M) * sizeof(float);
 }
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
