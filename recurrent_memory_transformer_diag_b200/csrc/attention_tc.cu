@@ -14,7 +14,10 @@
 //   MMA  S_w = Q_w K_j^T          (M=128 queries, N=128 keys, K=64) -> TMEM
 //   softmax: row max, p = exp2(s - m) as fp16 P_w in shared memory (K-major,
 //            128-byte swizzle)
-//   MMA  O_w += P_w V_j           (M=128, N=64, K=128 keys), O_w stays in TMEM
+//   MMA  O_w += P_w [V_j | 1]     (M=128, N=80, K=128 keys), O_w stays in TMEM;
+//        column 64 of O_w accumulates the row sums of P (a ones row is
+//        appended to V^T in shared memory), so the softmax never sums
+//        probabilities itself and the sum follows every rescaling of O
 // The running max m is only raised when a row's max grows by more than 8 (in
 // log2 units): then that row of O_w is rescaled in TMEM; otherwise the stale
 // max is kept (p <= 2^8 fits fp16 and the row sum uses the same max, so the
@@ -38,16 +41,18 @@ constexpr int BKEY = 128;               // keys per tile
 constexpr int NUM_THREADS = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (2 warpgroups)
 constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
 constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
-constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB (two 64-key blocks of 8 KB)
+constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB loaded per stage (two 64-key blocks of 8 KB)
+constexpr int ON = HD + 16;             // O columns: 64 dims, the row-sum column, 15 zero columns
+constexpr int VT_BLK = ON * 128;        // V^T block in shared memory: 80 rows of 64 keys (10 KB)
 constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
 constexpr int KV_STAGES = 2;
 constexpr int OFF_Q = 0;                               // [2 warpgroups][2 buffers]
 constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // KV_STAGES stages
-constexpr int OFF_VT = OFF_K + KV_STAGES * K_BYTES;
-constexpr int OFF_P = OFF_VT + KV_STAGES * VT_BYTES;   // [2 warpgroups]
+constexpr int OFF_VT = OFF_K + KV_STAGES * K_BYTES;    // [stage][2 blocks of VT_BLK]
+constexpr int OFF_P = OFF_VT + KV_STAGES * 2 * VT_BLK;  // [2 warpgroups]
 constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
 constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
-constexpr int TMEM_COLS = 512;          // S_A 0, S_B 128, O_A 256, O_B 320
+constexpr int TMEM_COLS = 512;          // S_A 0, S_B 128, O_A 256, O_B 256 + ON
 constexpr float RESCALE_THRESHOLD = 8.f;
 
 struct AttnParams {
@@ -131,6 +136,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  if (warp >= 2) {
+    // rows HD .. ON-1 of every V^T block: a row of ones (row sums), then zeros;
+    // TMA only ever writes rows 0 .. HD-1
+    for (int e = threadIdx.x - 64; e < KV_STAGES * 2 * 16 * 8; e += NUM_THREADS - 64) {
+      const int blk = e / (16 * 8), rr = (e / 8) % 16, chunk = e % 8;
+      const uint32_t one2 = 0x3C003C00u;   // two fp16 ones
+      const uint4 val = rr == 0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(smem + OFF_VT + blk * VT_BLK + (HD + rr) * 128 + chunk * 16) = val;
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -158,10 +174,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&kv_empty[st], ((t / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
         tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
-        uint8_t* vt = smem + OFF_VT + st * VT_BYTES;
+        uint8_t* vt = smem + OFF_VT + st * 2 * VT_BLK;
         const int vt_outer = nd.z * p.KV + g;
         tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
-        tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BYTES / 2, j * BKEY + 64, 0, vt_outer);
+        tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
         armed |= 16u << st;
       }
       if (!ok) {
@@ -182,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
-      const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x 64 x 16
+      const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
       auto issue_s = [&](int w, int t) -> bool {
         const int k = t / ntiles, j = t - k * ntiles;
         const int qb = w * 2 + (k & 1), ks = t % KV_STAGES;
@@ -204,13 +220,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!mbar_wait(&p_full[w], t & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
-        const uint32_t va = smem_u32(smem + OFF_VT + (t % KV_STAGES) * VT_BYTES);
+        const uint32_t va = smem_u32(smem + OFF_VT + (t % KV_STAGES) * 2 * VT_BLK);
 #pragma unroll
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem_base + 2 * BKEY + w * HD, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
-                    sw128_desc(va + kb * (HD * 128) + kk * 32), idesc_o, (j > 0 || kb > 0 || kk > 0));
+            mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
+                    sw128_desc(va + kb * VT_BLK + kk * 32), idesc_o, (j > 0 || kb > 0 || kk > 0));
         mma_commit(&o_full[w]);
         return true;
       };
@@ -241,17 +257,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row = q0 + rloc;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tm = tmem_base + lane_off + w * BKEY;
-    const uint32_t o_tm = tmem_base + lane_off + 2 * BKEY + w * HD;
+    const uint32_t o_tm = tmem_base + lane_off + 2 * BKEY + w * ON;
     uint8_t* pbuf = smem + OFF_P + w * P_BYTES;
     const int nw = (w == 0 ? heads_a : heads_b) * ntiles;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY;
     bool ok = true;
     for (int t = 0; t < nw && ok; ++t) {
       const int k = t / ntiles, j = t - k * ntiles;
-      if (j == 0) {
-        m_used = -INFINITY;
-        l = 0.f;
-      }
+      if (j == 0) m_used = -INFINITY;
       bool got = mbar_wait(&s_full[w], t & 1, abort_flag);
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       tc_fence_after();
@@ -265,12 +278,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool diag = j == ntiles - 1;
       const int k0 = j * BKEY;
       float mx = -INFINITY;
+      if (diag) {   // causal mask on the tile that holds the diagonal
 #pragma unroll
-      for (int i = 0; i < BKEY; ++i) {
-        float v = __uint_as_float(sr[i]);
-        if (diag && k0 + i > row) v = -INFINITY;
-        sr[i] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int i = 0; i < BKEY; ++i) {
+          float v = __uint_as_float(sr[i]);
+          if (k0 + i > row) v = -INFINITY;
+          sr[i] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < BKEY; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
       }
       const float m_tile = mx * p.scale_log2;     // scale > 0: max commutes with it
       float corr = 1.f;
@@ -280,7 +298,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if (m_tile > m_used + RESCALE_THRESHOLD) {
         corr = exp2f(m_used - m_tile);
         m_used = m_tile;
-        l *= corr;
         rescale = true;
       }
       // O(t-1) must be complete: its MMA read the P buffer, and O may be rescaled below
@@ -289,26 +306,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
       }
-      float sum = 0.f;
 #pragma unroll
       for (int c = 0; c < BKEY / 32; ++c) {
         float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float e = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
-          v[i] = e;
-          sum += e;
-        }
+        for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
         store_p_chunk(pbuf, rloc, c, v);
       }
-      l += sum;
       if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
-        uint32_t orr[HD];
+        uint32_t orr[HD], osum[16];
         tmem_ld64_nowait(o_tm, orr);
+        tmem_ld16_nowait(o_tm + HD, osum);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) osum[i] = __float_as_uint(__uint_as_float(osum[i]) * corr);
         tmem_st64(o_tm, orr);
+        tmem_st16(o_tm + HD, osum);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -319,13 +334,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         got = mbar_wait(&o_full[w], t & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
-        uint32_t orr[HD];
+        uint32_t orr[HD], osum[16];
         tmem_ld64_nowait(o_tm, orr);
+        tmem_ld16_nowait(o_tm + HD, osum);
         tmem_wait_ld();
         tc_fence_before();
         if (row < p.Tp) {
           const int h = g * grp + w + 2 * k;
-          const float inv = 1.f / l;
+          const float inv = 1.f / __uint_as_float(osum[0]);   // row sum of P (column 64 of O)
           f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
 #pragma unroll
           for (int q = 0; q < HD / 8; ++q) {

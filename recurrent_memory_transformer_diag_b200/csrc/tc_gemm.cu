@@ -147,34 +147,76 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
   return rsqrtf(ss / (float)p.norm_dim + p.norm_eps);
 }
 
+// Residual chunk (32 fp32 columns from col) of this thread's row, for the
+// residual epilogues; zeros when the row or chunk is out of range (the
+// partial-chunk path re-reads the residual itself).
+__device__ __forceinline__ void prefetch_h(const TcGemmParams& p, int slot, int row, bool valid, int col,
+                                           float4 (&hb)[8]) {
+  if (valid && col + 32 <= p.N) {
+    const float4* H = reinterpret_cast<const float4*>(p.h + (long long)slot * p.h_slot_stride +
+                                                      (long long)row * p.ldh + col);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hb[q] = H[q];
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hb[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb, int half) {
+                                             bool valid, int nb, int half, float4 (&hcur)[8]) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
-  if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+  if constexpr (EPI == TC_EPI_F32) {
     float rs = 1.f;
-    if (EPI != TC_EPI_F32 && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
-    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
-    if (EPI == TC_EPI_F32 && p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
-    float ss = 0.f;
+    if (p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
 #pragma unroll 1
     for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
       const int col = nb * BN + c * 32;
       if (!valid || col >= p.N) continue;
-      const int nv = p.N - col;
-      if (EPI == TC_EPI_F32) {
-        float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-        if (p.rsq) {
+      float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+      if (p.rsq) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= rs;
-        }
-        store_f32x32(C, v, nv);
-      } else {
+        for (int i = 0; i < 32; ++i) v[i] *= rs;
+      }
+      store_f32x32(C, v, p.N - col);
+    }
+  } else if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+    // h += acc * rs; the residual chunk of column block c+1 is loaded while
+    // chunk c is processed (hcur holds chunk c, prefetched by the caller for
+    // the first chunk before the accumulator wait)
+    float rs = 1.f;
+    if (p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
+    float ss = 0.f;
+    const int c_begin = half * (BN / 64), c_end = (half + 1) * (BN / 64);
+#pragma unroll 1
+    for (int c = c_begin; c < c_end; ++c) {
+      const int col = nb * BN + c * 32;
+      float4 hnext[8];
+      if (c + 1 < c_end) prefetch_h(p, slot, row, valid, col + 32, hnext);
+      float v[32];
+      tmem_ld32(tbase + c * 32, v);
+      if (valid && col < p.N) {
+        const int nv = p.N - col;
         float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
-        resid_add32(H, v, rs, nv);
+        if (nv >= 32) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 o = hcur[q];
+            o.x = fmaf(v[4 * q], rs, o.x);
+            o.y = fmaf(v[4 * q + 1], rs, o.y);
+            o.z = fmaf(v[4 * q + 2], rs, o.z);
+            o.w = fmaf(v[4 * q + 3], rs, o.w);
+            reinterpret_cast<float4*>(H)[q] = o;
+            v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+          }
+        } else {
+          resid_add32(H, v, rs, nv);
+        }
         if (p.rsq) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
@@ -188,8 +230,12 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
           }
         }
       }
+      if (c + 1 < c_end) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) hcur[q] = hnext[q];
+      }
     }
-    if (EPI != TC_EPI_F32 && p.rsq && valid)
+    if (p.rsq && valid)
       p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + 2 * nb + half] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
@@ -395,6 +441,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int buf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = mb * BM + row_in_tile;
+      const bool valid = row < p.M;
+      // the residual rows do not depend on this tile's MMAs: start loading
+      // them before waiting for the accumulator
+      float4 hcur[8];
+      if (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT)
+        prefetch_h(p, nd.z, row, valid, nb * BN + half * (BN / 2), hcur);
       const bool got = mbar_wait(&tfull[buf], acc_phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -402,13 +458,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
-      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
-      const NodeEntry nd = p.nodes[node];
-      const int row = mb * BM + row_in_tile;
-      const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hcur);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
