@@ -102,6 +102,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // an earlier kernel of this forward already gave up on a wait: do nothing
+  if (*reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK) return;
   const NodeEntry nd = p.nodes[blockIdx.z];
   const int g = blockIdx.y;                         // kv head
   const int grp = p.H / p.KV;                       // query heads per kv head

@@ -153,9 +153,10 @@ template <int MT>
 constexpr int log2_const() { return MT <= 1 ? 0 : 1 + log2_const<MT / 2>(); }
 
 // M <= MT <= 32: lane j carries memory row j through the recurrence.  A warp
-// updates R rows of A per pass (rows i, i + 8, ..., i + 8 (R-1) of its block's
-// range), so every phi element read from shared memory serves R rows.
-constexpr int MEMW_R = 4;
+// updates R = 2 rows of A per pass (rows i and i + 8 of its block's range), so
+// every phi element read from shared memory serves both rows (R = 4 measured
+// slower: 212 registers leave one block per SM).
+constexpr int MEMW_R = 2;
 
 template <int MAXC, int MT>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,

@@ -66,7 +66,9 @@ struct Smem {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
+  static constexpr int STG_OFFSET = BAR_OFFSET + 256;     // epilogue staging: [warp][32][33] fp32
+  static constexpr int STG_BYTES = EPI_WARPS * 32 * 33 * 4;
+  static constexpr int TOTAL = STG_OFFSET + STG_BYTES + 1024;   // + alignment slack
 };
 
 __device__ __forceinline__ void store_f32x32(float* dst, const float* v, int valid_cols) {
@@ -147,25 +149,9 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
   return rsqrtf(ss / (float)p.norm_dim + p.norm_eps);
 }
 
-// Residual chunk (32 fp32 columns from col) of this thread's row, for the
-// residual epilogues; zeros when the row or chunk is out of range (the
-// partial-chunk path re-reads the residual itself).
-__device__ __forceinline__ void prefetch_h(const TcGemmParams& p, int slot, int row, bool valid, int col,
-                                           float4 (&hb)[8]) {
-  if (valid && col + 32 <= p.N) {
-    const float4* H = reinterpret_cast<const float4*>(p.h + (long long)slot * p.h_slot_stride +
-                                                      (long long)row * p.ldh + col);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) hb[q] = H[q];
-  } else {
-#pragma unroll
-    for (int q = 0; q < 8; ++q) hb[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-}
-
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb, int half, float4 (&hcur)[8]) {
+                                             bool valid, int nb, int half, float* stg) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
   if constexpr (EPI == TC_EPI_F32) {
@@ -185,55 +171,57 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       store_f32x32(C, v, p.N - col);
     }
   } else if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
-    // h += acc * rs; the residual chunk of column block c+1 is loaded while
-    // chunk c is processed (hcur holds chunk c, prefetched by the caller for
-    // the first chunk before the accumulator wait)
+    // h += acc * rs, coalesced: each 32 x 32 block (thread = row after the
+    // TMEM load) is transposed through the warp's shared-memory staging tile,
+    // so that every global access of the residual, of its fp16 operand copy
+    // and of the output rows covers 32 consecutive columns of one row.
     float rs = 1.f;
     if (p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
-    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
+    const int row0 = row - (threadIdx.x & 31);          // first row of this warp's 32
+    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer;
     float ss = 0.f;
-    const int c_begin = half * (BN / 64), c_end = (half + 1) * (BN / 64);
 #pragma unroll 1
-    for (int c = c_begin; c < c_end; ++c) {
-      const int col = nb * BN + c * 32;
-      float4 hnext[8];
-      if (c + 1 < c_end) prefetch_h(p, slot, row, valid, col + 32, hnext);
+    for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
-      if (valid && col < p.N) {
-        const int nv = p.N - col;
-        float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
-        if (nv >= 32) {
+      const int lane = threadIdx.x & 31;
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            float4 o = hcur[q];
-            o.x = fmaf(v[4 * q], rs, o.x);
-            o.y = fmaf(v[4 * q + 1], rs, o.y);
-            o.z = fmaf(v[4 * q + 2], rs, o.z);
-            o.w = fmaf(v[4 * q + 3], rs, o.w);
-            reinterpret_cast<float4*>(H)[q] = o;
-            v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
-          }
-        } else {
-          resid_add32(H, v, rs, nv);
-        }
-        if (p.rsq) {
+      for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = v[i] * rs;
+      __syncwarp();
+      const int col = nb * BN + c * 32 + lane;
+      const bool cvalid = col < p.N;
+      float* H = p.h + (long long)slot * p.h_slot_stride + col;
+      float hv[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
-        }
-        if (EPI == TC_EPI_RESID_ACT) {
-          f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-          store_act32(X, v, nv);
-          if (to_out) {
-            bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
-            store_bf16_32(O, v, nv);
+      for (int r = 0; r < 32; ++r) {
+        const int gr = row0 + r;
+        hv[r] = (cvalid && gr < p.M) ? H[(long long)gr * p.ldh] : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const int gr = row0 + r;
+        if (cvalid && gr < p.M) {
+          const float nh = hv[r] + stg[r * 33 + lane];
+          H[(long long)gr * p.ldh] = nh;
+          stg[r * 33 + lane] = nh;
+          if (EPI == TC_EPI_RESID_ACT) {
+            reinterpret_cast<f16*>(p.C)[(long long)slot * p.c_slot_stride + (long long)gr * p.ldc + col] =
+                __float2half_rn(nh);
+            if (to_out && gr < p.seg_len)
+              reinterpret_cast<bf16*>(p.out)[((long long)nd.x * p.seg_len + gr) * p.N + col] = __float2bfloat16_rn(nh);
           }
         }
       }
-      if (c + 1 < c_end) {
+      __syncwarp();
+      if (p.rsq) {   // this thread's row again: sum of squares of the new residual
+        const int nv = p.N - (nb * BN + c * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) hcur[q] = hnext[q];
+        for (int i = 0; i < 32; ++i) {
+          const float x = stg[lane * 33 + i];
+          ss = (i < nv) ? fmaf(x, x, ss) : ss;
+        }
       }
+      __syncwarp();
     }
     if (p.rsq && valid)
       p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + 2 * nb + half] = ss;
@@ -326,6 +314,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // an earlier kernel of this forward already gave up on a wait: do nothing
+  // (the forward's result is reported as failed), so a systematic failure
+  // costs one bounded wait, not one per CTA and launch
+  if (*reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK) return;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SM::STAGES; ++s) {
       mbar_init(&full[s], 1);
@@ -437,6 +429,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- epilogue (warps 2..9) ----------------
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
+    float* stg = reinterpret_cast<float*>(smem + SM::STG_OFFSET) + (warp - 2) * 32 * 33;
     const int row_in_tile = quarter * 32 + lane;
     int buf = 0;
     uint32_t acc_phase = 0;
@@ -446,11 +439,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const NodeEntry nd = p.nodes[node];
       const int row = mb * BM + row_in_tile;
       const bool valid = row < p.M;
-      // the residual rows do not depend on this tile's MMAs: start loading
-      // them before waiting for the accumulator
-      float4 hcur[8];
-      if (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT)
-        prefetch_h(p, nd.z, row, valid, nb * BN + half * (BN / 2), hcur);
       const bool got = mbar_wait(&tfull[buf], acc_phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -459,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hcur);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, stg);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
