@@ -57,6 +57,7 @@ constexpr float RESCALE_THRESHOLD = 8.f;
 
 struct AttnParams {
   const NodeEntry* nodes;
+  int n_nodes;
   int Tp;            // rows per node
   int H, KV, nqkv;
   int q_tiles;
@@ -104,14 +105,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // an earlier kernel of this forward already gave up on a wait: do nothing
   if (*reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK) return;
-  const NodeEntry nd = p.nodes[blockIdx.z];
-  const int g = blockIdx.y;                         // kv head
   const int grp = p.H / p.KV;                       // query heads per kv head
-  const int qt = p.q_tiles - 1 - blockIdx.x;        // longest tiles first
-  const int q0 = qt * BQ;
-  const int ntiles = (min(p.Tp, q0 + BQ) + BKEY - 1) / BKEY;   // key tiles 0..qt
   const int heads_a = (grp + 1) / 2, heads_b = grp / 2;   // warpgroup A: even heads, B: odd heads
-  const int nA = heads_a * ntiles, nB = heads_b * ntiles;
+  const int per_qt = p.n_nodes * p.KV;
+  const int n_items = per_qt * p.q_tiles;
+  // work item u: longest query tiles first, then node, then kv head
+  auto decode = [&](int u, NodeEntry& nd, int& g, int& q0, int& ntiles) {
+    const int qt = p.q_tiles - 1 - u / per_qt;
+    const int rem = u - (u / per_qt) * per_qt;
+    nd = p.nodes[rem / p.KV];
+    g = rem - (rem / p.KV) * p.KV;
+    q0 = qt * BQ;
+    ntiles = (min(p.Tp, q0 + BQ) + BKEY - 1) / BKEY;   // key tiles 0..qt
+  };
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 4; ++b) {
@@ -154,33 +160,44 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Counters run on across work items, so every barrier's phase follows from
+  // them: kv = K/V stages loaded, qh[w] = heads started by warpgroup w,
+  // sw[w] = steps (S and O products) of warpgroup w.
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: per step t, the warpgroups' Q when a head starts, then K_j, V_j^T
+      // ---------------- TMA producer: per step, each warpgroup's Q when a head starts, then K_j, V_j^T
       bool ok = true;
       uint32_t armed = 0;   // bits 0-3: Q buffers, 4..: KV stages with loads in flight
-      for (int t = 0; t < nA && ok; ++t) {
-        const int k = t / ntiles, j = t - k * ntiles;
-        if (j == 0) {
-          for (int w = 0; w < 2; ++w) {
-            if (k >= (w == 0 ? heads_a : heads_b)) continue;
-            const int qb = w * 2 + (k & 1);
-            if (!mbar_wait(&q_empty[qb], ((k >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-            mbar_expect_tx(&q_full[qb], Q_BYTES);
-            tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * k) * HD, q0, nd.z);
-            armed |= 1u << qb;
+      int kv = 0, qh[2] = {0, 0};
+      for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
+        NodeEntry nd; int g, q0, ntiles;
+        decode(u, nd, g, q0, ntiles);
+        const int nA = heads_a * ntiles;
+        for (int t = 0; t < nA && ok; ++t) {
+          const int k = t / ntiles, j = t - k * ntiles;
+          if (j == 0) {
+            for (int w = 0; w < 2; ++w) {
+              if (k >= (w == 0 ? heads_a : heads_b)) continue;
+              const int qb = w * 2 + (qh[w] & 1);
+              if (!mbar_wait(&q_empty[qb], ((qh[w] >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+              mbar_expect_tx(&q_full[qb], Q_BYTES);
+              tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * k) * HD, q0, nd.z);
+              armed |= 1u << qb;
+              ++qh[w];
+            }
+            if (!ok) break;
           }
-          if (!ok) break;
+          const int st = kv % KV_STAGES;
+          if (!mbar_wait(&kv_empty[st], ((kv / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
+          tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
+          uint8_t* vt = smem + OFF_VT + st * 2 * VT_BLK;
+          const int vt_outer = nd.z * p.KV + g;
+          tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
+          tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
+          armed |= 16u << st;
+          ++kv;
         }
-        const int st = t % KV_STAGES;
-        if (!mbar_wait(&kv_empty[st], ((t / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-        mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
-        tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
-        uint8_t* vt = smem + OFF_VT + st * 2 * VT_BLK;
-        const int vt_outer = nd.z * p.KV + g;
-        tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
-        tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
-        armed |= 16u << st;
       }
       if (!ok) {
         atomicOr(p.err, 16u);
@@ -201,12 +218,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
       const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
+      int kv = 0, qh[2] = {0, 0}, sw[2] = {0, 0};
+      int ntiles = 1;
+      // S_w for step t of the current item (kv stage kv + t, step sw[w] + t, head qh[w] + k)
       auto issue_s = [&](int w, int t) -> bool {
         const int k = t / ntiles, j = t - k * ntiles;
-        const int qb = w * 2 + (k & 1), ks = t % KV_STAGES;
-        if (j == 0 && !mbar_wait(&q_full[qb], (k >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&kv_full[ks], (t / KV_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(&s_empty[w], (t & 1) ^ 1, abort_flag)) return false;
+        const int hidx = qh[w] + k, sidx = sw[w] + t, kidx = kv + t;
+        const int qb = w * 2 + (hidx & 1), ks = kidx % KV_STAGES;
+        if (j == 0 && !mbar_wait(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(&kv_full[ks], (kidx / KV_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
         const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
@@ -219,10 +240,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_o = [&](int w, int t) -> bool {
         const int j = t % ntiles;
-        if (!mbar_wait(&p_full[w], t & 1, abort_flag)) return false;
+        const int sidx = sw[w] + t, kidx = kv + t;
+        if (!mbar_wait(&p_full[w], sidx & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
-        const uint32_t va = smem_u32(smem + OFF_VT + (t % KV_STAGES) * 2 * VT_BLK);
+        const uint32_t va = smem_u32(smem + OFF_VT + (kidx % KV_STAGES) * 2 * VT_BLK);
 #pragma unroll
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
@@ -232,14 +254,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&o_full[w]);
         return true;
       };
-      bool ok = nA > 0 ? issue_s(0, 0) : true;
-      if (ok && nB > 0) ok = issue_s(1, 0);
-      for (int t = 0; t < nA && ok; ++t) {
-        if (!issue_o(0, t)) { ok = false; break; }
-        if (t + 1 < nA && !issue_s(0, t + 1)) { ok = false; break; }
-        if (t < nB && !issue_o(1, t)) { ok = false; break; }
-        mma_commit(&kv_empty[t % KV_STAGES]);   // K_t, V_t no longer read once these MMAs finish
-        if (t + 1 < nB && !issue_s(1, t + 1)) { ok = false; break; }
+      bool ok = true;
+      for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
+        NodeEntry nd; int g, q0;
+        decode(u, nd, g, q0, ntiles);
+        const int nA = heads_a * ntiles, nB = heads_b * ntiles;
+        ok = issue_s(0, 0);
+        if (ok && nB > 0) ok = issue_s(1, 0);
+        for (int t = 0; t < nA && ok; ++t) {
+          if (!issue_o(0, t)) { ok = false; break; }
+          if (t + 1 < nA && !issue_s(0, t + 1)) { ok = false; break; }
+          if (t < nB && !issue_o(1, t)) { ok = false; break; }
+          mma_commit(&kv_empty[(kv + t) % KV_STAGES]);   // K_t, V_t no longer read once these MMAs finish
+          if (t + 1 < nB && !issue_s(1, t + 1)) { ok = false; break; }
+        }
+        kv += nA;
+        qh[0] += heads_a;
+        qh[1] += heads_b;
+        sw[0] += nA;
+        sw[1] += nB;
       }
       if (!ok) {
         atomicOr(p.err, 32u);
@@ -256,109 +289,118 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int w = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;
-    const int row = q0 + rloc;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tm = tmem_base + lane_off + w * BKEY;
     const uint32_t o_tm = tmem_base + lane_off + 2 * BKEY + w * ON;
     uint8_t* pbuf = smem + OFF_P + w * P_BYTES;
-    const int nw = (w == 0 ? heads_a : heads_b) * ntiles;
-    float m_used = -INFINITY;
+    const int heads = w == 0 ? heads_a : heads_b;
+    int sbase = 0;
     bool ok = true;
-    for (int t = 0; t < nw && ok; ++t) {
-      const int k = t / ntiles, j = t - k * ntiles;
-      if (j == 0) m_used = -INFINITY;
-      bool got = mbar_wait(&s_full[w], t & 1, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[BKEY];
-      tmem_ld64_nowait(s_tm, sr);
-      tmem_ld64_nowait(s_tm + 64, sr + 64);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_empty[w]);   // S is in registers: the next S may be computed
-      const bool diag = j == ntiles - 1;
-      const int k0 = j * BKEY;
-      float mx = -INFINITY;
-      if (diag) {   // causal mask on the tile that holds the diagonal
-#pragma unroll
-        for (int i = 0; i < BKEY; ++i) {
-          float v = __uint_as_float(sr[i]);
-          if (k0 + i > row) v = -INFINITY;
-          sr[i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < BKEY; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-      }
-      const float m_tile = mx * p.scale_log2;     // scale > 0: max commutes with it
-      float corr = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_used = m_tile;
-      } else if (m_tile > m_used + RESCALE_THRESHOLD) {
-        corr = exp2f(m_used - m_tile);
-        m_used = m_tile;
-        rescale = true;
-      }
-      // O(t-1) must be complete: its MMA read the P buffer, and O may be rescaled below
-      if (t > 0) {
-        got = mbar_wait(&o_full[w], (t - 1) & 1, abort_flag);
+    for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
+      NodeEntry nd; int g, q0, ntiles;
+      decode(u, nd, g, q0, ntiles);
+      const int row = q0 + rloc;
+      const int nw = heads * ntiles;
+      float m_used = -INFINITY;
+      for (int t = 0; t < nw && ok; ++t) {
+        const int sidx = sbase + t;
+        const int k = t / ntiles, j = t - k * ntiles;
+        if (j == 0) m_used = -INFINITY;
+        bool got = mbar_wait(&s_full[w], sidx & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
-      }
-#pragma unroll
-      for (int c = 0; c < BKEY / 32; ++c) {
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
-        store_p_chunk(pbuf, rloc, c, v);
-      }
-      if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
-        uint32_t orr[HD], osum[16];
-        tmem_ld64_nowait(o_tm, orr);
-        tmem_ld16_nowait(o_tm + HD, osum);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) osum[i] = __float_as_uint(__uint_as_float(osum[i]) * corr);
-        tmem_st64(o_tm, orr);
-        tmem_st16(o_tm + HD, osum);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[w]);
-      if (j == ntiles - 1) {      // head done: wait for its last O, normalise, store
-        got = mbar_wait(&o_full[w], t & 1, abort_flag);
-        if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-        tc_fence_after();
-        uint32_t orr[HD], osum[16];
-        tmem_ld64_nowait(o_tm, orr);
-        tmem_ld16_nowait(o_tm + HD, osum);
+        uint32_t sr[BKEY];
+        tmem_ld64_nowait(s_tm, sr);
+        tmem_ld64_nowait(s_tm + 64, sr + 64);
         tmem_wait_ld();
         tc_fence_before();
-        if (row < p.Tp) {
-          const int h = g * grp + w + 2 * k;
-          const float inv = 1.f / __uint_as_float(osum[0]);   // row sum of P (column 64 of O)
-          f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[w]);   // S is in registers: the next S may be computed
+        const bool diag = j == ntiles - 1;
+        const int k0 = j * BKEY;
+        float mx = -INFINITY;
+        if (diag) {   // causal mask on the tile that holds the diagonal
 #pragma unroll
-          for (int q = 0; q < HD / 8; ++q) {
-            uint4 pk;
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&pk);
+          for (int i = 0; i < BKEY; ++i) {
+            float v = __uint_as_float(sr[i]);
+            if (k0 + i > row) v = -INFINITY;
+            sr[i] = __float_as_uint(v);
+            mx = fmaxf(mx, v);
+          }
+        } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
-                                             __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
-              wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+          for (int i = 0; i < BKEY; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+        }
+        const float m_tile = mx * p.scale_log2;     // scale > 0: max commutes with it
+        float corr = 1.f;
+        bool rescale = false;
+        if (j == 0) {
+          m_used = m_tile;
+        } else if (m_tile > m_used + RESCALE_THRESHOLD) {
+          corr = exp2f(m_used - m_tile);
+          m_used = m_tile;
+          rescale = true;
+        }
+        // O(t-1) must be complete: its MMA read the P buffer, and O may be rescaled below
+        // (at t == 0 the previous head's last O was already waited for)
+        if (t > 0) {
+          got = mbar_wait(&o_full[w], (sidx - 1) & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int c = 0; c < BKEY / 32; ++c) {
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
+          store_p_chunk(pbuf, rloc, c, v);
+        }
+        if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
+          uint32_t orr[HD], osum[16];
+          tmem_ld64_nowait(o_tm, orr);
+          tmem_ld16_nowait(o_tm + HD, osum);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) osum[i] = __float_as_uint(__uint_as_float(osum[i]) * corr);
+          tmem_st64(o_tm, orr);
+          tmem_st16(o_tm + HD, osum);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[w]);
+        if (j == ntiles - 1) {      // head done: wait for its last O, normalise, store
+          got = mbar_wait(&o_full[w], sidx & 1, abort_flag);
+          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t orr[HD], osum[16];
+          tmem_ld64_nowait(o_tm, orr);
+          tmem_ld16_nowait(o_tm + HD, osum);
+          tmem_wait_ld();
+          tc_fence_before();
+          if (row < p.Tp) {
+            const int h = g * grp + w + 2 * k;
+            const float inv = 1.f / __uint_as_float(osum[0]);   // row sum of P (column 64 of O)
+            f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
+#pragma unroll
+            for (int q = 0; q < HD / 8; ++q) {
+              uint4 pk;
+              uint32_t* wv = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
+                                               __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
+                wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+              reinterpret_cast<uint4*>(dst)[q] = pk;
             }
-            reinterpret_cast<uint4*>(dst)[q] = pk;
           }
         }
       }
+      sbase += nw;
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, 64u);
@@ -414,6 +456,7 @@ cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, i
   if (e != cudaSuccess) return e;
   AttnParams p;
   p.nodes = nodes;
+  p.n_nodes = n;
   p.Tp = Tp;
   p.H = dm.H;
   p.KV = dm.KV;
@@ -422,8 +465,11 @@ cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, i
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)HD);
   p.out = (f16*)out;
   p.err = err;
-  dim3 grid(p.q_tiles, dm.KV, n);
-  attention_tc_kernel<<<grid, NUM_THREADS, SMEM_TOTAL, st>>>(tm_qk, tm_vt, p);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int items = n * dm.KV * p.q_tiles;
+  attention_tc_kernel<<<items < sms ? items : sms, NUM_THREADS, SMEM_TOTAL, st>>>(tm_qk, tm_vt, p);
   return cudaGetLastError();
 }
 

@@ -66,9 +66,7 @@ struct Smem {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int STG_OFFSET = BAR_OFFSET + 256;     // epilogue staging: [warp][32][33] fp32
-  static constexpr int STG_BYTES = EPI_WARPS * 32 * 33 * 4;
-  static constexpr int TOTAL = STG_OFFSET + STG_BYTES + 1024;   // + alignment slack
+  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
 };
 
 __device__ __forceinline__ void store_f32x32(float* dst, const float* v, int valid_cols) {
@@ -151,79 +149,47 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
 
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb, int half, float* stg) {
+                                             bool valid, int nb, int half) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
-  if constexpr (EPI == TC_EPI_F32) {
+  if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
     float rs = 1.f;
-    if (p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
+    if (EPI != TC_EPI_F32 && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
+    if (EPI == TC_EPI_F32 && p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
+    float ss = 0.f;
 #pragma unroll 1
     for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
       const int col = nb * BN + c * 32;
       if (!valid || col >= p.N) continue;
-      float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-      if (p.rsq) {
+      const int nv = p.N - col;
+      if (EPI == TC_EPI_F32) {
+        float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+        if (p.rsq) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] *= rs;
-      }
-      store_f32x32(C, v, p.N - col);
-    }
-  } else if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
-    // h += acc * rs, coalesced: each 32 x 32 block (thread = row after the
-    // TMEM load) is transposed through the warp's shared-memory staging tile,
-    // so that every global access of the residual, of its fp16 operand copy
-    // and of the output rows covers 32 consecutive columns of one row.
-    float rs = 1.f;
-    if (p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
-    const int row0 = row - (threadIdx.x & 31);          // first row of this warp's 32
-    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer;
-    float ss = 0.f;
-#pragma unroll 1
-    for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
-      float v[32];
-      tmem_ld32(tbase + c * 32, v);
-      const int lane = threadIdx.x & 31;
+          for (int i = 0; i < 32; ++i) v[i] *= rs;
+        }
+        store_f32x32(C, v, nv);
+      } else {
+        float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
+        resid_add32(H, v, rs, nv);
+        if (p.rsq) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) stg[lane * 33 + i] = v[i] * rs;
-      __syncwarp();
-      const int col = nb * BN + c * 32 + lane;
-      const bool cvalid = col < p.N;
-      float* H = p.h + (long long)slot * p.h_slot_stride + col;
-      float hv[32];
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const int gr = row0 + r;
-        hv[r] = (cvalid && gr < p.M) ? H[(long long)gr * p.ldh] : 0.f;
-      }
-#pragma unroll
-      for (int r = 0; r < 32; ++r) {
-        const int gr = row0 + r;
-        if (cvalid && gr < p.M) {
-          const float nh = hv[r] + stg[r * 33 + lane];
-          H[(long long)gr * p.ldh] = nh;
-          stg[r * 33 + lane] = nh;
-          if (EPI == TC_EPI_RESID_ACT) {
-            reinterpret_cast<f16*>(p.C)[(long long)slot * p.c_slot_stride + (long long)gr * p.ldc + col] =
-                __float2half_rn(nh);
-            if (to_out && gr < p.seg_len)
-              reinterpret_cast<bf16*>(p.out)[((long long)nd.x * p.seg_len + gr) * p.N + col] = __float2bfloat16_rn(nh);
+          for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
+        }
+        if (EPI == TC_EPI_RESID_ACT) {
+          f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+          store_act32(X, v, nv);
+          if (to_out) {
+            bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
+            store_bf16_32(O, v, nv);
           }
         }
       }
-      __syncwarp();
-      if (p.rsq) {   // this thread's row again: sum of squares of the new residual
-        const int nv = p.N - (nb * BN + c * 32);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float x = stg[lane * 33 + i];
-          ss = (i < nv) ? fmaf(x, x, ss) : ss;
-        }
-      }
-      __syncwarp();
     }
-    if (p.rsq && valid)
+    if (EPI != TC_EPI_F32 && p.rsq && valid)
       p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + 2 * nb + half] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
@@ -429,16 +395,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ---------------- epilogue (warps 2..9) ----------------
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
-    float* stg = reinterpret_cast<float*>(smem + SM::STG_OFFSET) + (warp - 2) * 32 * 33;
     const int row_in_tile = quarter * 32 + lane;
     int buf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
-      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
-      const NodeEntry nd = p.nodes[node];
-      const int row = mb * BM + row_in_tile;
-      const bool valid = row < p.M;
       const bool got = mbar_wait(&tfull[buf], acc_phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -446,8 +406,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = mb * BM + row_in_tile;
+      const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, stg);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
