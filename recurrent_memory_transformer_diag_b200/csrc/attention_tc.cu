@@ -104,7 +104,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // an earlier kernel of this forward already gave up on a wait: do nothing
-  if (*reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK) return;
+  // (one thread reads the word, so the whole CTA takes the same decision)
+  __shared__ unsigned skip_cta;
+  if (threadIdx.x == 0) skip_cta = *reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK;
+  __syncthreads();
+  if (skip_cta) return;
   const int grp = p.H / p.KV;                       // query heads per kv head
   const int heads_a = (grp + 1) / 2, heads_b = grp / 2;   // warpgroup A: even heads, B: odd heads
   const int per_qt = p.n_nodes * p.KV;

@@ -283,7 +283,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // an earlier kernel of this forward already gave up on a wait: do nothing
   // (the forward's result is reported as failed), so a systematic failure
   // costs one bounded wait, not one per CTA and launch
-  if (*reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK) return;
+  // (one thread reads the word, so the whole CTA takes the same decision)
+  __shared__ unsigned skip_cta;
+  if (threadIdx.x == 0) skip_cta = *reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK;
+  __syncthreads();
+  if (skip_cta) return;
   if (threadIdx.x == 0) {
     for (int s = 0; s < SM::STAGES; ++s) {
       mbar_init(&full[s], 1);
