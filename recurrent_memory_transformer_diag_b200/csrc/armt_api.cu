@@ -243,7 +243,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.epi = EPI_STORE_ACT;
     L("gemm_qkv", [&] { return launch_simt_gemm(g, st); });
   }
-  L("rope", [&] { return launch_rope(dm, nodes, n, Tp, ws.qkv, ws.rope, st); });
+  L("rope", [&] { return launch_rope(dm, nodes, n, Tp, ws.qkv, ws.rope, ws.tp_max, st); });
   L("attention", [&] { return launch_attention_simt(dm, nodes, n, Tp, ws.qkv, ws.attn, st); });
   {
     GemmArgs g{};
@@ -315,6 +315,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   const NodeEntry* nodes = ws.nodes + wv.first;
   const int slots = ws.slots;
   const long long hs = (long long)Tp * dm.d;
+  const long long hs_blk = (long long)rows_blocked(Tp) * dm.d;   // row-blocked residual, per slot
   const int Hh = dm.H * dm.hd;
   const int f_pad = (dm.F + 127) / 128 * 128;
   const int sms = ctx->sm_count;
@@ -325,7 +326,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   };
   const int rsq_parts = 2 * ((dm.d + 255) / 256);   // one partial per half of a 256-column tile
   auto norm_partials = [&](TcGemmParams& p) {
-    p.rsq = ws.rsq; p.rsq_slot_stride = (long long)Tp * rsq_parts; p.rsq_parts = rsq_parts;
+    p.rsq = ws.rsq; p.rsq_slot_stride = (long long)Tp * rsq_parts; p.rsq_parts = rsq_parts; p.rsq_pitch = Tp;
     p.norm_dim = dm.d; p.norm_eps = dm.rms_eps;
   };
 
@@ -344,7 +345,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     // h += phi A^T / (z.phi + eps); new h -> fp16 operand copy + norm partials
     TcGemmOperands op{ws.phi, Tp, slots, ws.a_act, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.P);
-    p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
+    p.h = ws.h; p.h_slot_stride = hs_blk; p.ldh = dm.d;
     p.rowscale = ws.inv_den; p.rs_slot_stride = Tp;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
     norm_partials(p);
@@ -356,7 +357,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     TcGemmOperands op{ws.xb, Tp, slots, w.w_qkv, dm.nqkv, dm.L};
     TcGemmParams p; base(p, Tp, dm.nqkv, dm.d);
     p.C = ws.qkv; p.c_slot_stride = (long long)Tp * dm.nqkv; p.ldc = dm.nqkv;
-    p.rope = ws.rope; p.rope_half = dm.hd / 2; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
+    p.rope = ws.rope; p.rope_pitch = ws.tp_max; p.rope_heads = dm.H + dm.KV; p.head_dim = dm.hd;
     if (ws.vt) {
       p.vt = (f16*)ws.vt; p.vt_pitch = attention_tc_vt_pitch(Tp); p.n_vheads = dm.KV;
     }
@@ -370,7 +371,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   L("tc_o", [&] {
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
-    p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
+    p.h = ws.h; p.h_slot_stride = hs_blk; p.ldh = dm.d;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
     norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
@@ -389,7 +390,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     // this node's memory-write rows); last layer: rows < T -> out_hidden
     TcGemmOperands op{ws.u, Tp, slots, w.w_down, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.F);
-    p.h = ws.h; p.h_slot_stride = hs; p.ldh = dm.d;
+    p.h = ws.h; p.h_slot_stride = hs_blk; p.ldh = dm.d;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
     p.out = out; p.out_layer = dm.L - 1; p.seg_len = T;
     norm_partials(p);   // for the memory-write rows
@@ -553,7 +554,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   const size_t ntab = (size_t)cfg->max_segments * dm.L;
   e = cudaSuccess;
   auto A = [&](auto** p, size_t bytes) { if (e == cudaSuccess) e = dalloc(p, bytes); };
-  A(&ws.h, rows * dm.d * 4);
+  A(&ws.h, (size_t)ws.slots * rows_blocked(ws.tp_max) * dm.d * 4);   // >= rows * d (row-blocked slots)
   A(&ws.xb, rows * dm.d * as);
   A(&ws.qm, rows * dm.dk * 4);
   A(&ws.phi, rows * dm.P * as);
@@ -582,7 +583,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
     for (int p = 0; p < ws.tp_max; ++p)
       for (int j = 0; j < dm.hd / 2; ++j) {
         const double ang = (double)p * pow((double)dm.theta, -2.0 * j / dm.hd);
-        tab[(size_t)p * (dm.hd / 2) + j] = make_float2((float)cos(ang), (float)sin(ang));
+        tab[(size_t)j * ws.tp_max + p] = make_float2((float)cos(ang), (float)sin(ang));
       }
     e = cudaMemcpy(ws.rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
   }

@@ -21,6 +21,17 @@ typedef __half f16;
 constexpr unsigned ERR_WAIT_TIMEOUT_MASK = 0x77u; // bits 0-2 (GEMM), 4-6 (attention): a bounded wait ran out
 constexpr unsigned ERR_FP16_RANGE = 8u;           // an fp16 operand copy exceeded the fp16 range
 
+// Residual stream layout on the tensor-core path ("row-blocked"): rows in
+// blocks of 32, each block stored as [d/4 column groups][32 rows][4 columns].
+// Epilogue threads own one accumulator row each (32 consecutive rows per
+// warp), so a 16-byte access of 4 columns by the 32 threads of a warp covers
+// one contiguous 512-byte span instead of 32 separate rows.  d % 4 == 0;
+// a slot holds rows_blocked(T') rows.
+__host__ __device__ inline long long h_blocked_offset(int row, int col, int d) {
+  return ((long long)(row >> 5) * (d >> 2) + (col >> 2)) * 128 + (row & 31) * 4 + (col & 3);
+}
+__host__ __device__ inline int rows_blocked(int Tp) { return (Tp + 31) & ~31; }
+
 // One node of the (segment, layer) grid as the kernels see it: x = segment s,
 // y = layer l, z = activation slot (s mod number-of-slots), w = flags.
 typedef int4 NodeEntry;
@@ -38,12 +49,13 @@ struct Wave {
 struct Workspace {
   int slots = 0;
   int tp_max = 0;           // max rows per node (max_seg_len + n_mem)
-  float* h = nullptr;       // [slots][T'][d] residual stream, fp32
+  float* h = nullptr;       // residual stream, fp32: [slots][T'][d] (fp32 path), row-blocked
+                            // [slots][rows_blocked(T')][d] (tensor-core path)
   void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (fp32, or fp16 on the tensor-core path)
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
   void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or fp16 on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
-  float* rsq = nullptr;     // [slots][T'][2 ceil(d/256)] RMSNorm partial sums (tensor-core path)
+  float* rsq = nullptr;     // [slots][2 ceil(d/256)][T'] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
   void* attn = nullptr;     // [slots][T'][H*hd]  (fp32 / fp16)
   void* vt = nullptr;       // [slots][KV][hd][pitch] fp16 V^T for the tcgen05 attention
@@ -55,7 +67,7 @@ struct Workspace {
   float* coef = nullptr;    // [slots][M] 1 / (z_j . phi_j + eps)
   float* gamma = nullptr;   // [slots][M]
   void* a_act = nullptr;    // [L][d][P] fp16 copy of A (tensor-core path: the read GEMM operand)
-  float2* rope = nullptr;   // [tp_max][hd/2] (cos, sin)
+  float2* rope = nullptr;   // [hd/2][tp_max] (cos, sin), frequency-major
   NodeEntry* nodes = nullptr;
   int nodes_cap = 0;
   unsigned* err = nullptr;  // device error word (bounded waits)
@@ -127,6 +139,8 @@ struct GemmArgs {
 // SIMT grouped GEMM, fp32 operands (fp32 path, unit entry points).
 cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st);
 
+// fp32 path: h row-major.  Tensor-core path (xb != nullptr): h row-blocked,
+// xb the fp16 copy, row-major.
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                                     const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st);
 // RMSNorm (no gain) of rows row0 .. row0+nrows-1 of every node's slot.
@@ -134,8 +148,9 @@ cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp
                            const float* h, void* xb, float eps, cudaStream_t st);
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
                              const float* z_state, void* phi, float* inv_den, unsigned* err, cudaStream_t st);
+// rope: [hd/2][rope_pitch] (cos, sin) of angle p * theta^(-2j/hd) at [j][p]
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
-                        const float2* rope, cudaStream_t st);
+                        const float2* rope, int rope_pitch, cudaStream_t st);
 cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
                                   const void* qkv, void* out, cudaStream_t st);
 cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* gu,

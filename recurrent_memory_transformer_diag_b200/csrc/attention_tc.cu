@@ -66,6 +66,14 @@ struct AttnParams {
   unsigned* err;
 };
 
+// 2^x by the hardware approximation (PTX ex2.approx.ftz.f32; 2^-inf = +0).
+// Its relative error is far below the fp16 rounding that P goes through next.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // P rows: K-major operand, 128 keys = two 64-key blocks, 128-byte swizzle.
 __device__ __forceinline__ void store_p_chunk(uint8_t* pbuf, int row, int c, const float* p) {
   // chunk c = keys c*32 .. c*32+31 -> block c/2, 16-byte chunks (c%2)*4 .. +3
@@ -180,6 +188,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < nA && ok; ++t) {
           const int k = t / ntiles, j = t - k * ntiles;
           if (j == 0) {
+#pragma unroll
             for (int w = 0; w < 2; ++w) {
               if (k >= (w == 0 ? heads_a : heads_b)) continue;
               const int qb = w * 2 + (qh[w] & 1);
@@ -222,12 +231,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
       const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
-      int kv = 0, qh[2] = {0, 0}, sw[2] = {0, 0};
-      int ntiles = 1;
-      // S_w for step t of the current item (kv stage kv + t, step sw[w] + t, head qh[w] + k)
-      auto issue_s = [&](int w, int t) -> bool {
-        const int k = t / ntiles, j = t - k * ntiles;
-        const int hidx = qh[w] + k, sidx = sw[w] + t, kidx = kv + t;
+      // A step: key tile j of head k of a work item (t = k * ntiles + j);
+      // kv0 / qh0[w] / sw0[w] = K/V stages, heads and steps of warpgroup w
+      // consumed by the CTA's earlier items.
+      struct Cursor {   // fields per warpgroup spelled out: no dynamically indexed (local-memory) arrays
+        int u, t, ntiles, nA, nB, kv0, qh0_a, qh0_b, sw0_a, sw0_b;
+      };
+      auto load_item = [&](Cursor& c) {
+        NodeEntry nd; int g, q0;
+        decode(c.u, nd, g, q0, c.ntiles);
+        c.nA = heads_a * c.ntiles;
+        c.nB = heads_b * c.ntiles;
+      };
+      auto advance = [&](Cursor& c) -> bool {
+        if (c.t + 1 < c.nA) { ++c.t; return true; }
+        const int u = c.u + gridDim.x;
+        if (u >= n_items) return false;
+        c.kv0 += c.nA;
+        c.qh0_a += heads_a;
+        c.qh0_b += heads_b;
+        c.sw0_a += c.nA;
+        c.sw0_b += c.nB;
+        c.u = u;
+        c.t = 0;
+        load_item(c);
+        return true;
+      };
+      auto issue_s = [&](int w, const Cursor& c) -> bool {
+        const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
+        const int hidx = (w ? c.qh0_b : c.qh0_a) + k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
         const int qb = w * 2 + (hidx & 1), ks = kidx % KV_STAGES;
         if (j == 0 && !mbar_wait(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
         if (!mbar_wait(&kv_full[ks], (kidx / KV_STAGES) & 1, abort_flag)) return false;
@@ -239,12 +271,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kk = 0; kk < HD / 16; ++kk)
           mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
         mma_commit(&s_full[w]);
-        if (j == ntiles - 1) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
+        if (j == c.ntiles - 1) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
         return true;
       };
-      auto issue_o = [&](int w, int t) -> bool {
-        const int j = t % ntiles;
-        const int sidx = sw[w] + t, kidx = kv + t;
+      auto issue_o = [&](int w, const Cursor& c) -> bool {
+        const int j = c.t % c.ntiles;
+        const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
         if (!mbar_wait(&p_full[w], sidx & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
@@ -258,25 +290,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&o_full[w]);
         return true;
       };
+      // Steps run as one sequence across the CTA's work items: S of the next
+      // step (next key tile, next head or next item) is issued before O of
+      // the current one (the S buffer is free once the softmax has the scores
+      // in registers), so a warpgroup finds its next scores computed when it
+      // finishes a tile.
       bool ok = true;
-      for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        NodeEntry nd; int g, q0;
-        decode(u, nd, g, q0, ntiles);
-        const int nA = heads_a * ntiles, nB = heads_b * ntiles;
-        ok = issue_s(0, 0);
-        if (ok && nB > 0) ok = issue_s(1, 0);
-        for (int t = 0; t < nA && ok; ++t) {
-          if (!issue_o(0, t)) { ok = false; break; }
-          if (t + 1 < nA && !issue_s(0, t + 1)) { ok = false; break; }
-          if (t < nB && !issue_o(1, t)) { ok = false; break; }
-          mma_commit(&kv_empty[(kv + t) % KV_STAGES]);   // K_t, V_t no longer read once these MMAs finish
-          if (t + 1 < nB && !issue_s(1, t + 1)) { ok = false; break; }
+      Cursor cur;
+      if (blockIdx.x < n_items) {
+        cur.u = blockIdx.x; cur.t = 0; cur.kv0 = 0; cur.qh0_a = cur.qh0_b = 0; cur.sw0_a = cur.sw0_b = 0;
+        load_item(cur);
+        ok = issue_s(0, cur);
+        if (ok && cur.nB > 0) ok = issue_s(1, cur);
+        while (ok) {
+          Cursor nxt = cur;
+          const bool more = advance(nxt);
+          // order S_A(next), O_A(cur), S_B(next), O_B(cur): each warpgroup's
+          // O is issued as soon as its P is ready
+          if (more && !issue_s(0, nxt)) { ok = false; break; }
+          if (!issue_o(0, cur)) { ok = false; break; }
+          if (more && nxt.t < nxt.nB && !issue_s(1, nxt)) { ok = false; break; }
+          if (cur.t < cur.nB && !issue_o(1, cur)) { ok = false; break; }
+          mma_commit(&kv_empty[(cur.kv0 + cur.t) % KV_STAGES]);   // K_t, V_t no longer read once these finish
+          if (!more) break;
+          cur = nxt;
         }
-        kv += nA;
-        qh[0] += heads_a;
-        qh[1] += heads_b;
-        sw[0] += nA;
-        sw[1] += nB;
       }
       if (!ok) {
         atomicOr(p.err, 32u);
@@ -322,19 +360,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) mbar_arrive(&s_empty[w]);   // S is in registers: the next S may be computed
         const bool diag = j == ntiles - 1;
         const int k0 = j * BKEY;
-        float mx = -INFINITY;
+        // row max as 8 independent partial maxima (a short dependency chain)
+        float m8[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
         if (diag) {   // causal mask on the tile that holds the diagonal
 #pragma unroll
           for (int i = 0; i < BKEY; ++i) {
             float v = __uint_as_float(sr[i]);
             if (k0 + i > row) v = -INFINITY;
             sr[i] = __float_as_uint(v);
-            mx = fmaxf(mx, v);
+            m8[i & 7] = fmaxf(m8[i & 7], v);
           }
         } else {
 #pragma unroll
-          for (int i = 0; i < BKEY; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+          for (int i = 0; i < BKEY; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
         }
+        const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         const float m_tile = mx * p.scale_log2;     // scale > 0: max commutes with it
         float corr = 1.f;
         bool rescale = false;
@@ -356,7 +399,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int c = 0; c < BKEY / 32; ++c) {
           float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = exp2f(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
+          for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
           store_p_chunk(pbuf, rloc, c, v);
         }
         if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1

@@ -266,6 +266,139 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
+// Same computation with 16-byte accesses (P % 4 == 0): lane l owns the
+// column groups 4 (l + 32 c) .. +3, c < C4, so A rows are read and written as
+// float4 and every phi read from shared memory is one 16-byte load serving
+// 4 columns of both rows.  At most 128 registers: two blocks per SM.
+template <int C4, int MT>
+__global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
+                                                                 const float* kv, const float* phik,
+                                                                 const float* gram, const float* coef,
+                                                                 float* A_state, f16* a_act, unsigned* err) {
+  constexpr int R = MEMW_R;
+  extern __shared__ float sh[];
+  float* ph = sh;                    // [M][P]
+  float* G = ph + M * P;             // [M][M]
+  float* cf = G + M * M;             // [M]
+  float* dots = cf + M;              // [8][R][M]  delta_j per warp and row
+  const NodeEntry nd = nodes[blockIdx.y];
+  const int slot = nd.z, layer = nd.y;
+  const int P4 = P >> 2;
+  {
+    const float4* src = reinterpret_cast<const float4*>(phik + (long long)slot * M * P);
+    float4* dst = reinterpret_cast<float4*>(ph);
+    for (int e = threadIdx.x; e < M * P4; e += blockDim.x) dst[e] = src[e];
+  }
+  for (int e = threadIdx.x; e < M * M; e += blockDim.x) G[e] = gram[(long long)slot * M * M + e];
+  for (int e = threadIdx.x; e < M; e += blockDim.x) cf[e] = coef[(long long)slot * M + e];
+  __syncthreads();
+  const float4* ph4 = reinterpret_cast<const float4*>(ph);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* dl = dots + warp * R * M;
+  bool over = false;
+  constexpr int SHIFT = 5 - log2_const<MT>();
+  const float cj = lane < M ? cf[lane] : 0.f;
+  const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
+  const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
+  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+  for (int i0 = i_begin + warp; i0 < i_end; i0 += 8 * R) {
+    float4 a[R][C4];
+    float v[R];
+    bool has[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = i0 + 8 * r;
+      has[r] = i < i_end;
+      const float4* Arow = reinterpret_cast<const float4*>(A_state + ((long long)layer * d + (has[r] ? i : i0)) * P);
+      v[r] = (lane < M && has[r]) ? kvj[i] : 0.f;
+#pragma unroll
+      for (int c = 0; c < C4; ++c) {
+        const int q = lane + 32 * c;
+        a[r][c] = (q < P4 && has[r]) ? Arow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    // a_r . phi_j for all rows and j at once (independent accumulators)
+    float part[R][MT];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int j = 0; j < MT; ++j) part[r][j] = 0.f;
+#pragma unroll
+    for (int c = 0; c < C4; ++c) {
+      const int q = lane + 32 * c;
+      if (q < P4) {
+#pragma unroll
+        for (int j = 0; j < MT; ++j) {
+          if (j < M) {
+            const float4 f = ph4[j * P4 + q];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              float t = fmaf(a[r][c].x, f.x, part[r][j]);
+              t = fmaf(a[r][c].y, f.y, t);
+              t = fmaf(a[r][c].z, f.z, t);
+              part[r][j] = fmaf(a[r][c].w, f.w, t);
+            }
+          }
+        }
+      }
+    }
+    // lane j (< M) keeps s_j = a . phi_j + sum_{j'<j} delta_j' G[j'][j]
+    float sv[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float tot = transpose_reduce<MT>(part[r], lane);
+      sv[r] = __shfl_sync(0xffffffffu, tot, (lane << SHIFT) & 31);
+    }
+    for (int j = 0; j < M; ++j) {
+      // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
+      const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
+        if (lane == j) dl[r * M + j] = dj;
+        sv[r] = fmaf(dj, gj, sv[r]);
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < C4; ++c) {
+      const int q = lane + 32 * c;
+      if (q < P4) {
+        float4 acc[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) acc[r] = a[r][c];
+        for (int j = 0; j < M; ++j) {
+          const float4 f = ph4[j * P4 + q];
+#pragma unroll
+          for (int r = 0; r < R; ++r) {
+            const float dj = dl[r * M + j];
+            acc[r].x = fmaf(dj, f.x, acc[r].x);
+            acc[r].y = fmaf(dj, f.y, acc[r].y);
+            acc[r].z = fmaf(dj, f.z, acc[r].z);
+            acc[r].w = fmaf(dj, f.w, acc[r].w);
+          }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          if (!has[r]) continue;
+          const long long off = ((long long)layer * d + i0 + 8 * r) * P + 4 * q;
+          *reinterpret_cast<float4*>(A_state + off) = acc[r];
+          if (a_act) {
+            const __half2 lo = __floats2half2_rn(acc[r].x, acc[r].y), hi = __floats2half2_rn(acc[r].z, acc[r].w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(a_act + off) = pk;
+            over |= fmaxf(fmaxf(fabsf(acc[r].x), fabsf(acc[r].y)), fmaxf(fabsf(acc[r].z), fabsf(acc[r].w))) > 65504.f;
+          }
+        }
+      }
+    }
+    __syncwarp();
+  }
+  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
+}
+
 static size_t memw_update_smem(const Dims& dm) {
   return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 8 * MEMW_R * dm.M) * sizeof(float);
 }
@@ -286,6 +419,26 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     else ARMT_MEMW_CASE(C, 32)          \
   }
   if (dm.M > 32) return cudaErrorInvalidValue;
+  if (dm.P % 4 == 0 && dm.P <= 1024) {   // 16-byte path
+    const int c4 = (dm.P / 4 + 31) / 32;
+#define ARMT_MEMWV_CASE(C, MT)                                                                                \
+  memw_update_vec_kernel<C, MT><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
+                                                       A_state, (f16*)a_act, err);
+#define ARMT_MEMWV_M(C)                  \
+  {                                      \
+    if (dm.M <= 4) ARMT_MEMWV_CASE(C, 4) \
+    else if (dm.M <= 16) ARMT_MEMWV_CASE(C, 16) \
+    else ARMT_MEMWV_CASE(C, 32)          \
+  }
+    if (c4 <= 2) ARMT_MEMWV_M(2)
+    else if (c4 <= 3) ARMT_MEMWV_M(3)
+    else if (c4 <= 4) ARMT_MEMWV_M(4)
+    else if (c4 <= 6) ARMT_MEMWV_M(6)
+    else ARMT_MEMWV_M(8)
+#undef ARMT_MEMWV_M
+#undef ARMT_MEMWV_CASE
+    return cudaGetLastError();
+  }
   if (chunks <= 4) ARMT_MEMW_M(4)
   else if (chunks <= 12) ARMT_MEMW_M(12)
   else if (chunks <= 24) ARMT_MEMW_M(24)
@@ -307,6 +460,11 @@ cudaError_t setup_memory_kernels(const Dims& dm) {
     set(memw_update_kernel<12, 4>); set(memw_update_kernel<12, 16>); set(memw_update_kernel<12, 32>);
     set(memw_update_kernel<24, 4>); set(memw_update_kernel<24, 16>); set(memw_update_kernel<24, 32>);
     set(memw_update_kernel<32, 4>); set(memw_update_kernel<32, 16>); set(memw_update_kernel<32, 32>);
+    set(memw_update_vec_kernel<2, 4>); set(memw_update_vec_kernel<2, 16>); set(memw_update_vec_kernel<2, 32>);
+    set(memw_update_vec_kernel<3, 4>); set(memw_update_vec_kernel<3, 16>); set(memw_update_vec_kernel<3, 32>);
+    set(memw_update_vec_kernel<4, 4>); set(memw_update_vec_kernel<4, 16>); set(memw_update_vec_kernel<4, 32>);
+    set(memw_update_vec_kernel<6, 4>); set(memw_update_vec_kernel<6, 16>); set(memw_update_vec_kernel<6, 32>);
+    set(memw_update_vec_kernel<8, 4>); set(memw_update_vec_kernel<8, 16>); set(memw_update_vec_kernel<8, 32>);
   }
   return e;
 }

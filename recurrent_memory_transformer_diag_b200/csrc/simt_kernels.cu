@@ -101,27 +101,54 @@ cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 template <typename TE>
 __global__ void init_first_layer_kernel(const NodeEntry* nodes, int T, int Tp, int d,
-                                        const TE* emb, const float* mem_emb, float* h, f16* xb) {
+                                        const TE* emb, const float* mem_emb, float* h) {
   const NodeEntry nd = nodes[blockIdx.y];
   if (nd.y != 0) return;
   const int t = blockIdx.x;
-  const long long o = ((long long)nd.z * Tp + t) * d;
-  float* dst = h + o;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) {
-    const float v = t < T ? ld(emb, ((long long)nd.x * T + t) * d + c) : mem_emb[(long long)(t - T) * d + c];
-    dst[c] = v;
-    if (xb) xb[o + c] = __float2half_rn(v);
+  float* dst = h + ((long long)nd.z * Tp + t) * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x)
+    dst[c] = t < T ? ld(emb, ((long long)nd.x * T + t) * d + c) : mem_emb[(long long)(t - T) * d + c];
+}
+
+// Tensor-core path: one block per 32 rows x 64 columns of a layer-0 node.
+// Rows are read (and the fp16 copy written) row-major through a shared tile,
+// then the fp32 residual is written in the row-blocked layout, where the
+// tile's 32 x 64 values form one contiguous run of 2048 floats.
+__global__ void init_first_layer_blocked_kernel(const NodeEntry* nodes, int T, int Tp, int d, const bf16* emb,
+                                                const float* mem_emb, float* h, f16* xb) {
+  __shared__ float tile[32][65];
+  const NodeEntry nd = nodes[blockIdx.z];
+  if (nd.y != 0) return;
+  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 64;
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int r = e >> 6, c = e & 63;
+    const int t = r0 + r, col = c0 + c;
+    float v = 0.f;
+    if (col < d && t < Tp) {
+      v = t < T ? __bfloat162float(emb[((long long)nd.x * T + t) * d + col]) : mem_emb[(long long)(t - T) * d + col];
+      xb[((long long)nd.z * Tp + t) * d + col] = __float2half_rn(v);
+    }
+    tile[r][c] = v;
+  }
+  __syncthreads();
+  float* hs = h + (long long)nd.z * rows_blocked(Tp) * d;
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int g = e >> 7, r = (e >> 2) & 31, cc = e & 3;   // column group, row, column in group
+    const int col = c0 + g * 4 + cc;
+    if (col < d) hs[h_blocked_offset(r0 + r, col, d)] = tile[r][g * 4 + cc];
   }
 }
 
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                                     const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st) {
-  dim3 grid(Tp, n);
-  if (dm.bf16)
-    init_first_layer_kernel<bf16><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const bf16*)emb, mem_emb, h, xb);
-  else
-    init_first_layer_kernel<float><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const float*)emb, mem_emb, h,
-                                                         nullptr);
+  if (dm.bf16) {
+    if (!xb || dm.d % 4) return cudaErrorInvalidValue;
+    dim3 grid(rows_blocked(Tp) / 32, (dm.d + 63) / 64, n);
+    init_first_layer_blocked_kernel<<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const bf16*)emb, mem_emb, h, xb);
+  } else {
+    dim3 grid(Tp, n);
+    init_first_layer_kernel<float><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const float*)emb, mem_emb, h);
+  }
   return cudaGetLastError();
 }
 
@@ -218,27 +245,27 @@ cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int 
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void rope_kernel(const NodeEntry* nodes, int Tp, int nheads_qk, int hd, int nqkv,
-                            T* qkv, const float2* rope) {
+                            T* qkv, const float2* rope, int rope_pitch) {
   const NodeEntry nd = nodes[blockIdx.y];
   const int t = blockIdx.x;
   const int half = hd / 2;
   T* row = qkv + ((long long)nd.z * Tp + t) * nqkv;
-  const float2* cs = rope + (long long)t * half;
   for (int idx = threadIdx.x; idx < nheads_qk * half; idx += blockDim.x) {
     const int hh = idx / half, j = idx - hh * half;
     const int c1 = hh * hd + j, c2 = c1 + half;
     const float x1 = ld(row, c1), x2 = ld(row, c2);
-    const float2 a = cs[j];
+    const float2 a = rope[(long long)j * rope_pitch + t];
     st(row, c1, x1 * a.x - x2 * a.y);
     st(row, c2, x2 * a.x + x1 * a.y);
   }
 }
 
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
-                        const float2* rope, cudaStream_t st) {
+                        const float2* rope, int rope_pitch, cudaStream_t st) {
   dim3 grid(Tp, n);
   if (dm.bf16) return cudaErrorInvalidValue;   // the tensor-core path fuses RoPE into the QKV GEMM
-  rope_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.H + dm.KV, dm.hd, dm.nqkv, (float*)qkv, rope);
+  rope_kernel<float><<<grid, 256, 0, st>>>(nodes, Tp, dm.H + dm.KV, dm.hd, dm.nqkv, (float*)qkv, rope,
+                                           rope_pitch);
   return cudaGetLastError();
 }
 

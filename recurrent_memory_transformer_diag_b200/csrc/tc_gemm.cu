@@ -111,25 +111,32 @@ __device__ __forceinline__ void store_bf16_32(bf16* dst, const float* v, int val
   }
 }
 
-// h += v * rs on 32 columns; v receives the new residual values.
-__device__ __forceinline__ void resid_add32(float* H, float* v, float rs, int valid_cols) {
-  if (valid_cols >= 32 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) {
+// h += v * rs on 32 columns (col % 4 == 0) of this thread's row of the
+// row-blocked residual Hs (one slot); v receives the new residual values.
+// Consecutive 4-column groups of a row are 128 floats apart.
+__device__ __forceinline__ void resid_add32(float* Hs, int row, int col, int d, float* v, float rs, int valid_cols) {
+  if (valid_cols >= 32) {
+    float4* H4 = reinterpret_cast<float4*>(Hs + h_blocked_offset(row, col, d));
+    float4 o[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) o[q] = H4[q * 32];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      float4 o = reinterpret_cast<float4*>(H)[q];
-      o.x = fmaf(v[4 * q], rs, o.x);
-      o.y = fmaf(v[4 * q + 1], rs, o.y);
-      o.z = fmaf(v[4 * q + 2], rs, o.z);
-      o.w = fmaf(v[4 * q + 3], rs, o.w);
-      reinterpret_cast<float4*>(H)[q] = o;
-      v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+      o[q].x = fmaf(v[4 * q], rs, o[q].x);
+      o[q].y = fmaf(v[4 * q + 1], rs, o[q].y);
+      o[q].z = fmaf(v[4 * q + 2], rs, o[q].z);
+      o[q].w = fmaf(v[4 * q + 3], rs, o[q].w);
+      v[4 * q] = o[q].x; v[4 * q + 1] = o[q].y; v[4 * q + 2] = o[q].z; v[4 * q + 3] = o[q].w;
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) H4[q * 32] = o[q];
   } else {
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       if (i < valid_cols) {
-        const float o = fmaf(v[i], rs, H[i]);
-        H[i] = o;
+        float* hp = Hs + h_blocked_offset(row, col + i, d);
+        const float o = fmaf(v[i], rs, *hp);
+        *hp = o;
         v[i] = o;
       }
     }
@@ -141,9 +148,9 @@ __device__ __forceinline__ void resid_add32(float* H, float* v, float rs, int va
 // guarded by the row/column bounds.
 // RMSNorm row scale from the per-tile partial sums of squares.
 __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot, int row) {
-  const float* part = p.rsq + (long long)slot * p.rsq_slot_stride + (long long)row * p.rsq_parts;
+  const float* part = p.rsq + (long long)slot * p.rsq_slot_stride + row;
   float ss = 0.f;
-  for (int i = 0; i < p.rsq_parts; ++i) ss += part[i];
+  for (int i = 0; i < p.rsq_parts; ++i) ss += part[(long long)i * p.rsq_pitch];
   return rsqrtf(ss / (float)p.norm_dim + p.norm_eps);
 }
 
@@ -173,8 +180,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         }
         store_f32x32(C, v, nv);
       } else {
-        float* H = p.h + (long long)slot * p.h_slot_stride + rofs * p.ldh + col;
-        resid_add32(H, v, rs, nv);
+        resid_add32(p.h + (long long)slot * p.h_slot_stride, row, col, p.ldh, v, rs, nv);
         if (p.rsq) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
@@ -190,7 +196,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       }
     }
     if (EPI != TC_EPI_F32 && p.rsq && valid)
-      p.rsq[(long long)slot * p.rsq_slot_stride + rofs * p.rsq_parts + 2 * nb + half] = ss;
+      p.rsq[(long long)slot * p.rsq_slot_stride + (long long)(2 * nb + half) * p.rsq_pitch + row] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
     const int hd = p.head_dim;
@@ -211,10 +217,11 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         const int col1 = nb * BN + c1 * 32, col2 = nb * BN + c2 * 32;
         if (!valid || col1 >= p.N) continue;
         if (rot) {
-          const float2* cs = p.rope + rofs * p.rope_half + pc * 32;
+          // frequency-major table: the warp's 32 rows read 32 consecutive entries
+          const float2* cs = p.rope + (long long)(pc * 32) * p.rope_pitch + row;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            const float2 a = cs[i];
+            const float2 a = cs[(long long)i * p.rope_pitch];
             const float x1 = v1[i] * rs, x2 = v2[i] * rs;
             v1[i] = x1 * a.x - x2 * a.y;
             v2[i] = x2 * a.x + x1 * a.y;

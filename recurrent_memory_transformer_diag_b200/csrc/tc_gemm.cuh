@@ -23,19 +23,20 @@ struct TcGemmParams {
   int a_by_layer;           // A's outer TMA coordinate: 0 = node slot, 1 = node layer
   int ab_bf16;              // operand type: 0 = fp16, 1 = bf16 (both operands alike)
   void* C; long long c_slot_stride; int ldc;
-  float* h; long long h_slot_stride; int ldh;
+  float* h; long long h_slot_stride; int ldh;   // residual, row-blocked (h_blocked_offset), ldh = row length
   const float* rowscale; long long rs_slot_stride;
-  const float2* rope; int rope_half; int rope_heads; int head_dim;
+  const float2* rope; int rope_pitch; int rope_heads; int head_dim;   // rope [hd/2][rope_pitch]
   // QKV epilogue: also write the value heads (heads >= rope_heads) transposed,
   // vt[slot][head - rope_heads][dim][row] with rows vt_pitch apart (optional)
   f16* vt; int vt_pitch; int n_vheads;
   int f_out;                // SWIGLU: number of valid output features
   // RMSNorm folded into the GEMMs.  Residual epilogues write, per row and per
   // half n-tile, the partial sum of squares of the new residual over those
-  // columns (rsq[slot][row][2 * tile + half], rsq_parts entries per row); QKV,
+  // columns (rsq[slot][2 * tile + half][row], parts rsq_pitch rows apart, so a
+  // warp's 32 rows touch 32 consecutive floats); QKV,
   // gate/up and kv-mem epilogues scale their rows by
   // rsqrt(sum of the partials / norm_dim + eps).
-  float* rsq; long long rsq_slot_stride; int rsq_parts; int norm_dim; float norm_eps;
+  float* rsq; long long rsq_slot_stride; int rsq_parts; int rsq_pitch; int norm_dim; float norm_eps;
   int rsq_row0;             // F32 epilogue: output row r is normalised with the partials of row rsq_row0 + r
   // final hidden states (down-projection epilogue of last-layer nodes)
   void* out; int out_layer; int seg_len;
