@@ -45,13 +45,15 @@ constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB loaded per stage (two 64-key bl
 constexpr int ON = HD + 16;             // O columns: 64 dims, the row-sum column, 15 zero columns
 constexpr int VT_BLK = ON * 128;        // V^T block in shared memory: 80 rows of 64 keys (10 KB)
 constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
-constexpr int KV_STAGES = 2;
+constexpr int K_STAGES = 3;             // K is needed first (S of the next step): deeper ring
+constexpr int V_STAGES = 2;             // V^T only at O, a softmax later
 constexpr int OFF_Q = 0;                               // [2 warpgroups][2 buffers]
-constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // KV_STAGES stages
-constexpr int OFF_VT = OFF_K + KV_STAGES * K_BYTES;    // [stage][2 blocks of VT_BLK]
-constexpr int OFF_P = OFF_VT + KV_STAGES * 2 * VT_BLK;  // [2 warpgroups]
+constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // [K_STAGES]
+constexpr int OFF_VT = OFF_K + K_STAGES * K_BYTES;     // [V_STAGES][2 blocks of VT_BLK]
+constexpr int OFF_P = OFF_VT + V_STAGES * 2 * VT_BLK;  // [2 warpgroups]
 constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
 constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
+static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
 constexpr int TMEM_COLS = 512;          // S_A 0, S_B 128, O_A 256, O_B 256 + ON
 constexpr float RESCALE_THRESHOLD = 8.f;
 
@@ -100,14 +102,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
   uint64_t* q_full = bar;          // [w][2]
   uint64_t* q_empty = bar + 4;     // [w][2]
-  uint64_t* kv_full = bar + 8;     // [KV_STAGES]
-  uint64_t* kv_empty = bar + 10;   // [KV_STAGES]
-  uint64_t* s_full = bar + 12;     // [w]
-  uint64_t* s_empty = bar + 14;    // [w]
-  uint64_t* p_full = bar + 16;     // [w]
-  uint64_t* o_full = bar + 18;     // [w]
-  uint64_t* drain = bar + 20;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
+  uint64_t* k_full = bar + 8;      // [K_STAGES]
+  uint64_t* k_empty = bar + 11;    // [K_STAGES]
+  uint64_t* v_full = bar + 14;     // [V_STAGES]
+  uint64_t* v_empty = bar + 16;    // [V_STAGES]
+  uint64_t* s_full = bar + 18;     // [w]
+  uint64_t* s_empty = bar + 20;    // [w]
+  uint64_t* p_full = bar + 22;     // [w]
+  uint64_t* o_full = bar + 24;     // [w]
+  uint64_t* drain = bar + 26;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 27);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,9 +140,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
     }
-    for (int b = 0; b < KV_STAGES; ++b) {
-      mbar_init(&kv_full[b], 1);
-      mbar_init(&kv_empty[b], 1);
+    for (int b = 0; b < K_STAGES; ++b) {
+      mbar_init(&k_full[b], 1);
+      mbar_init(&k_empty[b], 1);
+    }
+    for (int b = 0; b < V_STAGES; ++b) {
+      mbar_init(&v_full[b], 1);
+      mbar_init(&v_empty[b], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
@@ -159,7 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp >= 2) {
     // rows HD .. ON-1 of every V^T block: a row of ones (row sums), then zeros;
     // TMA only ever writes rows 0 .. HD-1
-    for (int e = threadIdx.x - 64; e < KV_STAGES * 2 * 16 * 8; e += NUM_THREADS - 64) {
+    for (int e = threadIdx.x - 64; e < V_STAGES * 2 * 16 * 8; e += NUM_THREADS - 64) {
       const int blk = e / (16 * 8), rr = (e / 8) % 16, chunk = e % 8;
       const uint32_t one2 = 0x3C003C00u;   // two fp16 ones
       const uint4 val = rr == 0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0u, 0u, 0u, 0u);
@@ -172,45 +180,119 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  // Counters run on across work items, so every barrier's phase follows from
-  // them: kv = K/V stages loaded, qh[w] = heads started by warpgroup w,
-  // sw[w] = steps (S and O products) of warpgroup w.
+  // The CTA's work is one sequence of steps: work items u = blockIdx.x,
+  // blockIdx.x + gridDim.x, ...; within an item, head k (of each warpgroup)
+  // and key tile j, step t = k * ntiles + j.  Warpgroup B has no step t when
+  // k >= heads_b (odd group size).  kv0 / qh0_* / sw0_* count the K/V tiles,
+  // heads and steps of each warpgroup consumed by the earlier items, so every
+  // barrier phase follows from them.
+  struct Cursor {   // fields per warpgroup spelled out: no dynamically indexed (local-memory) arrays
+    int u, t, ntiles, nA, nB, kv0, qh0_a, qh0_b, sw0_a, sw0_b;
+  };
+  auto load_item = [&](Cursor& c) {
+    NodeEntry nd; int g, q0;
+    decode(c.u, nd, g, q0, c.ntiles);
+    c.nA = heads_a * c.ntiles;
+    c.nB = heads_b * c.ntiles;
+  };
+  auto first_step = [&](Cursor& c) {
+    c.u = blockIdx.x; c.t = 0; c.kv0 = 0; c.qh0_a = c.qh0_b = 0; c.sw0_a = c.sw0_b = 0;
+    load_item(c);
+  };
+  auto advance = [&](Cursor& c) -> bool {
+    if (c.t + 1 < c.nA) { ++c.t; return true; }
+    const int u = c.u + gridDim.x;
+    if (u >= n_items) return false;
+    c.kv0 += c.nA;
+    c.qh0_a += heads_a;
+    c.qh0_b += heads_b;
+    c.sw0_a += c.nA;
+    c.sw0_b += c.nB;
+    c.u = u;
+    c.t = 0;
+    load_item(c);
+    return true;
+  };
+
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer: per step, each warpgroup's Q when a head starts, then K_j, V_j^T
+      // ---------------- TMA producer ----------------
+      // Per step: K_t (3-stage ring), then V^T of the previous step (2-stage
+      // ring), so K runs about two steps ahead of the tensor core and V one.
+      // Q tiles (two buffers per warpgroup) are loaded when a head is about to
+      // start at the latest, and one head ahead whenever the buffer is free.
       bool ok = true;
-      uint32_t armed = 0;   // bits 0-3: Q buffers, 4..: KV stages with loads in flight
-      int kv = 0, qh[2] = {0, 0};
-      for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
-        NodeEntry nd; int g, q0, ntiles;
-        decode(u, nd, g, q0, ntiles);
-        const int nA = heads_a * ntiles;
-        for (int t = 0; t < nA && ok; ++t) {
-          const int k = t / ntiles, j = t - k * ntiles;
-          if (j == 0) {
-#pragma unroll
-            for (int w = 0; w < 2; ++w) {
-              if (k >= (w == 0 ? heads_a : heads_b)) continue;
-              const int qb = w * 2 + (qh[w] & 1);
-              if (!mbar_wait(&q_empty[qb], ((qh[w] >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
-              mbar_expect_tx(&q_full[qb], Q_BYTES);
-              tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * k) * HD, q0, nd.z);
-              armed |= 1u << qb;
-              ++qh[w];
-            }
-            if (!ok) break;
-          }
-          const int st = kv % KV_STAGES;
-          if (!mbar_wait(&kv_empty[st], ((kv / KV_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&kv_full[st], K_BYTES + VT_BYTES);
-          tma_load_3d(&tm_qk, &kv_full[st], smem + OFF_K + st * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
-          uint8_t* vt = smem + OFF_VT + st * 2 * VT_BLK;
-          const int vt_outer = nd.z * p.KV + g;
-          tma_load_3d(&tm_vt, &kv_full[st], vt, j * BKEY, 0, vt_outer);
-          tma_load_3d(&tm_vt, &kv_full[st], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
-          armed |= 16u << st;
-          ++kv;
+      uint32_t armed = 0;   // bits 0-3: Q buffers, 4-6: K stages, 8-9: V stages with loads in flight
+      int qi_a = 0, qi_b = 0;            // Q loads issued per warpgroup
+      int qu_a = blockIdx.x, qk_a = 0;   // item and head of warpgroup A's next Q load
+      int qu_b = blockIdx.x, qk_b = 0;
+      // Q load for warpgroup w's next head; block: wait for the buffer, else only if it is free now.
+      // Returns 1 issued, 0 buffer busy, -1 wait failed.
+      auto q_issue = [&](int w, bool block) -> int {
+        int& qi = w ? qi_b : qi_a;
+        int& qu = w ? qu_b : qu_a;
+        int& qk = w ? qk_b : qk_a;
+        const int qb = w * 2 + (qi & 1);
+        const uint32_t par = ((qi >> 1) & 1) ^ 1;
+        if (block) {
+          if (!mbar_wait(&q_empty[qb], par, abort_flag)) return -1;
+        } else if (!mbar_try_wait(&q_empty[qb], par)) {
+          return 0;
         }
+        NodeEntry nd; int g, q0, nt;
+        decode(qu, nd, g, q0, nt);
+        mbar_expect_tx(&q_full[qb], Q_BYTES);
+        tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * qk) * HD, q0, nd.z);
+        armed |= 1u << qb;
+        ++qi;
+        if (++qk >= (w ? heads_b : heads_a)) { qk = 0; qu += gridDim.x; }
+        return 1;
+      };
+      auto load_v = [&](const Cursor& c) -> bool {
+        const int kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
+        const int j = c.t % c.ntiles;
+        if (!mbar_wait(&v_empty[vs], ((kidx / V_STAGES) & 1) ^ 1, abort_flag)) return false;
+        NodeEntry nd; int g, q0, nt;
+        decode(c.u, nd, g, q0, nt);
+        mbar_expect_tx(&v_full[vs], VT_BYTES);
+        uint8_t* vt = smem + OFF_VT + vs * 2 * VT_BLK;
+        const int vt_outer = nd.z * p.KV + g;
+        tma_load_3d(&tm_vt, &v_full[vs], vt, j * BKEY, 0, vt_outer);
+        tma_load_3d(&tm_vt, &v_full[vs], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
+        armed |= 256u << vs;
+        return true;
+      };
+      if (blockIdx.x < n_items) {
+        Cursor c, prev;
+        first_step(c);
+        bool has_prev = false;
+        while (ok) {
+          const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
+          // this step's Q tiles must be on their way (normally issued a head earlier)
+          const int ha = c.qh0_a + k, hb = c.qh0_b + k;
+          while (ok && qi_a <= ha) ok = q_issue(0, true) > 0;
+          if (k < heads_b)
+            while (ok && qi_b <= hb) ok = q_issue(1, true) > 0;
+          if (!ok) break;
+          {   // K_t
+            const int kidx = c.kv0 + c.t, ks = kidx % K_STAGES;
+            if (!mbar_wait(&k_empty[ks], ((kidx / K_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            NodeEntry nd; int g, q0, nt;
+            decode(c.u, nd, g, q0, nt);
+            mbar_expect_tx(&k_full[ks], K_BYTES);
+            tma_load_3d(&tm_qk, &k_full[ks], smem + OFF_K + ks * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
+            armed |= 16u << ks;
+          }
+          if (has_prev && !load_v(prev)) { ok = false; break; }
+          // one head ahead, if that buffer is already free
+          // (B's latest head in this item is min(k, heads_b - 1))
+          if (qi_a == ha + 1 && qu_a < n_items) q_issue(0, false);
+          if (heads_b > 0 && qi_b == c.qh0_b + min(k, heads_b - 1) + 1 && qu_b < n_items) q_issue(1, false);
+          prev = c;
+          has_prev = true;
+          if (!advance(c)) break;
+        }
+        if (ok && has_prev && !load_v(prev)) ok = false;
       }
       if (!ok) {
         atomicOr(p.err, 16u);
@@ -221,9 +303,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int b = 0; b < 4; ++b)
           if (armed & (1u << b))
             while (!mbar_try_wait(&q_full[b], 0) && !mbar_try_wait(&q_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
-        for (int b = 0; b < KV_STAGES; ++b)
+        for (int b = 0; b < K_STAGES; ++b)
           if (armed & (16u << b))
-            while (!mbar_try_wait(&kv_full[b], 0) && !mbar_try_wait(&kv_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
+            while (!mbar_try_wait(&k_full[b], 0) && !mbar_try_wait(&k_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
+        for (int b = 0; b < V_STAGES; ++b)
+          if (armed & (256u << b))
+            while (!mbar_try_wait(&v_full[b], 0) && !mbar_try_wait(&v_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
       }
     }
   } else if (warp == 1) {
@@ -231,38 +316,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer ----------------
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
       const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
-      // A step: key tile j of head k of a work item (t = k * ntiles + j);
-      // kv0 / qh0[w] / sw0[w] = K/V stages, heads and steps of warpgroup w
-      // consumed by the CTA's earlier items.
-      struct Cursor {   // fields per warpgroup spelled out: no dynamically indexed (local-memory) arrays
-        int u, t, ntiles, nA, nB, kv0, qh0_a, qh0_b, sw0_a, sw0_b;
-      };
-      auto load_item = [&](Cursor& c) {
-        NodeEntry nd; int g, q0;
-        decode(c.u, nd, g, q0, c.ntiles);
-        c.nA = heads_a * c.ntiles;
-        c.nB = heads_b * c.ntiles;
-      };
-      auto advance = [&](Cursor& c) -> bool {
-        if (c.t + 1 < c.nA) { ++c.t; return true; }
-        const int u = c.u + gridDim.x;
-        if (u >= n_items) return false;
-        c.kv0 += c.nA;
-        c.qh0_a += heads_a;
-        c.qh0_b += heads_b;
-        c.sw0_a += c.nA;
-        c.sw0_b += c.nB;
-        c.u = u;
-        c.t = 0;
-        load_item(c);
-        return true;
-      };
       auto issue_s = [&](int w, const Cursor& c) -> bool {
         const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
         const int hidx = (w ? c.qh0_b : c.qh0_a) + k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
-        const int qb = w * 2 + (hidx & 1), ks = kidx % KV_STAGES;
+        const int qb = w * 2 + (hidx & 1), ks = kidx % K_STAGES;
         if (j == 0 && !mbar_wait(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&kv_full[ks], (kidx / KV_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
         if (!mbar_wait(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
@@ -276,11 +335,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto issue_o = [&](int w, const Cursor& c) -> bool {
         const int j = c.t % c.ntiles;
-        const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
+        const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
         if (!mbar_wait(&p_full[w], sidx & 1, abort_flag)) return false;
+        if (!mbar_wait(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
-        const uint32_t va = smem_u32(smem + OFF_VT + (kidx % KV_STAGES) * 2 * VT_BLK);
+        const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
 #pragma unroll
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
@@ -290,28 +350,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         mma_commit(&o_full[w]);
         return true;
       };
-      // Steps run as one sequence across the CTA's work items: S of the next
-      // step (next key tile, next head or next item) is issued before O of
-      // the current one (the S buffer is free once the softmax has the scores
-      // in registers), so a warpgroup finds its next scores computed when it
-      // finishes a tile.
+      // S of the next step (next key tile, next head or next item) is issued
+      // before O of the current one (the S buffer is free once the softmax
+      // has the scores in registers), so a warpgroup finds its next scores
+      // computed when it finishes a tile.  Order per step: S_A(next), O_A,
+      // S_B(next), O_B: each warpgroup's O is issued as soon as its P is ready.
       bool ok = true;
-      Cursor cur;
       if (blockIdx.x < n_items) {
-        cur.u = blockIdx.x; cur.t = 0; cur.kv0 = 0; cur.qh0_a = cur.qh0_b = 0; cur.sw0_a = cur.sw0_b = 0;
-        load_item(cur);
+        Cursor cur;
+        first_step(cur);
         ok = issue_s(0, cur);
         if (ok && cur.nB > 0) ok = issue_s(1, cur);
+        if (ok) mma_commit(&k_empty[cur.kv0 % K_STAGES]);   // K_0 read by both S products
         while (ok) {
           Cursor nxt = cur;
           const bool more = advance(nxt);
-          // order S_A(next), O_A(cur), S_B(next), O_B(cur): each warpgroup's
-          // O is issued as soon as its P is ready
           if (more && !issue_s(0, nxt)) { ok = false; break; }
           if (!issue_o(0, cur)) { ok = false; break; }
           if (more && nxt.t < nxt.nB && !issue_s(1, nxt)) { ok = false; break; }
+          if (more) mma_commit(&k_empty[(nxt.kv0 + nxt.t) % K_STAGES]);
           if (cur.t < cur.nB && !issue_o(1, cur)) { ok = false; break; }
-          mma_commit(&kv_empty[(cur.kv0 + cur.t) % KV_STAGES]);   // K_t, V_t no longer read once these finish
+          mma_commit(&v_empty[(cur.kv0 + cur.t) % V_STAGES]);   // V_t no longer read once these finish
           if (!more) break;
           cur = nxt;
         }
