@@ -76,21 +76,15 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// P rows: K-major operand, 128 keys = two 64-key blocks, 128-byte swizzle.
-__device__ __forceinline__ void store_p_chunk(uint8_t* pbuf, int row, int c, const float* p) {
-  // chunk c = keys c*32 .. c*32+31 -> block c/2, 16-byte chunks (c%2)*4 .. +3
-  uint8_t* blk = pbuf + (c >> 1) * (BQ * 128) + row * 128;
+// P row of 128 keys from 64 packed fp16 pairs (pk[i] = keys 2i, 2i+1): K-major
+// operand, two 64-key blocks, 128-byte swizzle (16-byte chunk c of row r at
+// chunk position c ^ (r & 7)).
+__device__ __forceinline__ void store_p(uint8_t* pbuf, int row, const uint32_t* pk) {
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int chunk = ((c & 1) << 2) + q;
-    uint4 pk;
-    uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __half2 h2 = __floats2half2_rn(p[q * 8 + 2 * i], p[q * 8 + 2 * i + 1]);
-      w[i] = *reinterpret_cast<uint32_t*>(&h2);
-    }
-    *reinterpret_cast<uint4*>(blk + ((chunk ^ (row & 7)) << 4)) = pk;
+  for (int c = 0; c < 16; ++c) {   // 16-byte chunk c = keys 8c .. 8c+7
+    uint8_t* blk = pbuf + (c >> 3) * (BQ * 128) + row * 128;
+    *reinterpret_cast<uint4*>(blk + (((c & 7) ^ (row & 7)) << 4)) =
+        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
   }
 }
 
@@ -215,8 +209,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer ----------------
+    {
+      // ---------------- TMA producer (the whole warp runs the loop; one elected lane issues) ----------------
+      const bool issuer = elect_one();
       // Per step: K_t (3-stage ring), then V^T of the previous step (2-stage
       // ring), so K runs about two steps ahead of the tensor core and V one.
       // Q tiles (two buffers per warpgroup) are loaded when a head is about to
@@ -235,14 +230,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int qb = w * 2 + (qi & 1);
         const uint32_t par = ((qi >> 1) & 1) ^ 1;
         if (block) {
-          if (!mbar_wait(&q_empty[qb], par, abort_flag)) return -1;
-        } else if (!mbar_try_wait(&q_empty[qb], par)) {
+          if (!mbar_wait_warp(&q_empty[qb], par, abort_flag)) return -1;
+        } else if (!__any_sync(0xffffffffu, mbar_try_wait(&q_empty[qb], par))) {
           return 0;
         }
         NodeEntry nd; int g, q0, nt;
         decode(qu, nd, g, q0, nt);
-        mbar_expect_tx(&q_full[qb], Q_BYTES);
-        tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * qk) * HD, q0, nd.z);
+        if (issuer) mbar_expect_tx(&q_full[qb], Q_BYTES);
+        if (issuer) tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * qk) * HD, q0, nd.z);
         armed |= 1u << qb;
         ++qi;
         if (++qk >= (w ? heads_b : heads_a)) { qk = 0; qu += gridDim.x; }
@@ -251,14 +246,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       auto load_v = [&](const Cursor& c) -> bool {
         const int kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
         const int j = c.t % c.ntiles;
-        if (!mbar_wait(&v_empty[vs], ((kidx / V_STAGES) & 1) ^ 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&v_empty[vs], ((kidx / V_STAGES) & 1) ^ 1, abort_flag)) return false;
         NodeEntry nd; int g, q0, nt;
         decode(c.u, nd, g, q0, nt);
-        mbar_expect_tx(&v_full[vs], VT_BYTES);
+        if (issuer) mbar_expect_tx(&v_full[vs], VT_BYTES);
         uint8_t* vt = smem + OFF_VT + vs * 2 * VT_BLK;
         const int vt_outer = nd.z * p.KV + g;
-        tma_load_3d(&tm_vt, &v_full[vs], vt, j * BKEY, 0, vt_outer);
-        tma_load_3d(&tm_vt, &v_full[vs], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
+        if (issuer) tma_load_3d(&tm_vt, &v_full[vs], vt, j * BKEY, 0, vt_outer);
+        if (issuer) tma_load_3d(&tm_vt, &v_full[vs], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
         armed |= 256u << vs;
         return true;
       };
@@ -276,11 +271,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           {   // K_t
             const int kidx = c.kv0 + c.t, ks = kidx % K_STAGES;
-            if (!mbar_wait(&k_empty[ks], ((kidx / K_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(&k_empty[ks], ((kidx / K_STAGES) & 1) ^ 1, abort_flag)) { ok = false; break; }
             NodeEntry nd; int g, q0, nt;
             decode(c.u, nd, g, q0, nt);
-            mbar_expect_tx(&k_full[ks], K_BYTES);
-            tma_load_3d(&tm_qk, &k_full[ks], smem + OFF_K + ks * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
+            if (issuer) mbar_expect_tx(&k_full[ks], K_BYTES);
+            if (issuer) tma_load_3d(&tm_qk, &k_full[ks], smem + OFF_K + ks * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
             armed |= 16u << ks;
           }
           if (has_prev && !load_v(prev)) { ok = false; break; }
@@ -295,7 +290,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (ok && has_prev && !load_v(prev)) ok = false;
       }
       if (!ok) {
-        atomicOr(p.err, 16u);
+        if (issuer) atomicOr(p.err, 16u);
         *abort_flag = 1;
       }
       if (*abort_flag) {   // let every issued copy land before the CTA exits
@@ -312,32 +307,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    {
+      // ---------------- MMA issuer (the whole warp runs the loop; one elected lane issues) ----------------
+      const bool issuer = elect_one();
       const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
       const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
       auto issue_s = [&](int w, const Cursor& c) -> bool {
         const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
         const int hidx = (w ? c.qh0_b : c.qh0_a) + k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
         const int qb = w * 2 + (hidx & 1), ks = kidx % K_STAGES;
-        if (j == 0 && !mbar_wait(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
+        if (j == 0 && !mbar_wait_warp(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
         const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk)
-          mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
-        mma_commit(&s_full[w]);
-        if (j == c.ntiles - 1) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
+          if (issuer) mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+        if (issuer) mma_commit(&s_full[w]);
+        if (j == c.ntiles - 1 && issuer) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
         return true;
       };
       auto issue_o = [&](int w, const Cursor& c) -> bool {
         const int j = c.t % c.ntiles;
         const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
-        if (!mbar_wait(&p_full[w], sidx & 1, abort_flag)) return false;
-        if (!mbar_wait(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&p_full[w], sidx & 1, abort_flag)) return false;
+        if (!mbar_wait_warp(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
         tc_fence_after();
         const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
         const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
@@ -345,9 +341,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
+            if (issuer) mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
                     sw128_desc(va + kb * VT_BLK + kk * 32), idesc_o, (j > 0 || kb > 0 || kk > 0));
-        mma_commit(&o_full[w]);
+        if (issuer) mma_commit(&o_full[w]);
         return true;
       };
       // S of the next step (next key tile, next head or next item) is issued
@@ -361,25 +357,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         first_step(cur);
         ok = issue_s(0, cur);
         if (ok && cur.nB > 0) ok = issue_s(1, cur);
-        if (ok) mma_commit(&k_empty[cur.kv0 % K_STAGES]);   // K_0 read by both S products
+        if (ok && issuer) mma_commit(&k_empty[cur.kv0 % K_STAGES]);   // K_0 read by both S products
         while (ok) {
           Cursor nxt = cur;
           const bool more = advance(nxt);
           if (more && !issue_s(0, nxt)) { ok = false; break; }
           if (!issue_o(0, cur)) { ok = false; break; }
           if (more && nxt.t < nxt.nB && !issue_s(1, nxt)) { ok = false; break; }
-          if (more) mma_commit(&k_empty[(nxt.kv0 + nxt.t) % K_STAGES]);
+          if (more && issuer) mma_commit(&k_empty[(nxt.kv0 + nxt.t) % K_STAGES]);
           if (cur.t < cur.nB && !issue_o(1, cur)) { ok = false; break; }
-          mma_commit(&v_empty[(cur.kv0 + cur.t) % V_STAGES]);   // V_t no longer read once these finish
+          if (issuer) mma_commit(&v_empty[(cur.kv0 + cur.t) % V_STAGES]);   // V_t no longer read once these finish
           if (!more) break;
           cur = nxt;
         }
       }
       if (!ok) {
-        atomicOr(p.err, 32u);
+        if (issuer) atomicOr(p.err, 32u);
         *abort_flag = 1;
       }
-      mma_commit(drain);
+      if (issuer) mma_commit(drain);
       const unsigned long long t0 = global_ns();
       while (!mbar_try_wait(drain, 0)) {
         if (global_ns() - t0 > WAIT_LIMIT_NS) break;
@@ -397,6 +393,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int heads = w == 0 ? heads_a : heads_b;
     int sbase = 0;
     bool ok = true;
+    bool first = true;          // no O issued for this warpgroup yet
+    bool pend = false;          // a finished head whose O has not been read
+    f16* pend_dst = nullptr;    // its output row (nullptr: a padding row)
+    int last_sidx = 0;
+    // O of a finished head (complete, waited for): row sum in column 64,
+    // normalise, fp16 row of the head's 64 outputs
+    auto finalize = [&](f16* dst) {
+      uint32_t orr[HD], osum[16];
+      tmem_ld64_nowait(o_tm, orr);
+      tmem_ld16_nowait(o_tm + HD, osum);
+      tmem_wait_ld();
+      if (dst) {
+        const float inv = 1.f / __uint_as_float(osum[0]);
+#pragma unroll
+        for (int q = 0; q < HD / 8; ++q) {
+          uint4 v;
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
+                                           __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
+            wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+          reinterpret_cast<uint4*>(dst)[q] = v;
+        }
+      }
+    };
     for (int u = blockIdx.x; u < n_items && ok; u += gridDim.x) {
       NodeEntry nd; int g, q0, ntiles;
       decode(u, nd, g, q0, ntiles);
@@ -447,19 +470,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           m_used = m_tile;
           rescale = true;
         }
-        // O(t-1) must be complete: its MMA read the P buffer, and O may be rescaled below
-        // (at t == 0 the previous head's last O was already waited for)
-        if (t > 0) {
+        // P = 2^(s - m) as packed fp16 pairs, computed before waiting for the
+        // previous O (the exponentials overlap that product)
+        uint32_t pk[BKEY / 2];
+#pragma unroll
+        for (int i = 0; i < BKEY / 2; ++i) {
+          const __half2 h2 = __floats2half2_rn(ex2_approx(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, -m_used)),
+                                               ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, -m_used)));
+          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        // the previous step's O must be complete: its MMA read the P buffer,
+        // and O is read (head done) or rescaled below
+        if (!first) {
           got = mbar_wait(&o_full[w], (sidx - 1) & 1, abort_flag);
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
           tc_fence_after();
         }
-#pragma unroll
-        for (int c = 0; c < BKEY / 32; ++c) {
-          float v[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + i]), p.scale_log2, -m_used));
-          store_p_chunk(pbuf, rloc, c, v);
+        store_p(pbuf, rloc, pk);
+        if (pend) {   // the previous step ended a head: normalise its O and store it
+          finalize(pend_dst);
+          pend = false;
         }
         if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
           uint32_t orr[HD], osum[16];
@@ -478,35 +508,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[w]);
-        if (j == ntiles - 1) {      // head done: wait for its last O, normalise, store
-          got = mbar_wait(&o_full[w], sidx & 1, abort_flag);
-          if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
-          tc_fence_after();
-          uint32_t orr[HD], osum[16];
-          tmem_ld64_nowait(o_tm, orr);
-          tmem_ld16_nowait(o_tm + HD, osum);
-          tmem_wait_ld();
-          tc_fence_before();
-          if (row < p.Tp) {
-            const int h = g * grp + w + 2 * k;
-            const float inv = 1.f / __uint_as_float(osum[0]);   // row sum of P (column 64 of O)
-            f16* dst = p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + h * HD;
-#pragma unroll
-            for (int q = 0; q < HD / 8; ++q) {
-              uint4 pk;
-              uint32_t* wv = reinterpret_cast<uint32_t*>(&pk);
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
-                                               __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
-                wv[i] = *reinterpret_cast<uint32_t*>(&h2);
-              }
-              reinterpret_cast<uint4*>(dst)[q] = pk;
-            }
-          }
+        first = false;
+        if (j == ntiles - 1) {      // head done: its O is read at the next step (or after the last)
+          pend = true;
+          pend_dst = row < p.Tp ? p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + (g * grp + w + 2 * k) * HD
+                                : nullptr;
+          last_sidx = sidx;
         }
       }
       sbase += nw;
+    }
+    if (ok && pend) {   // the CTA's last head
+      const bool got = mbar_wait(&o_full[w], last_sidx & 1, abort_flag);
+      if (__all_sync(0xffffffffu, got)) {
+        tc_fence_after();
+        finalize(pend_dst);
+      } else {
+        ok = false;
+      }
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, 64u);

@@ -26,6 +26,8 @@
 // Every mbarrier wait is bounded (about one second); on timeout the kernel
 // sets the device error word, drains its own outstanding copies and MMAs,
 // frees TMEM and returns.
+#include <cstdlib>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -323,8 +325,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int total = p.n_nodes * tiles_per_node;
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ---------------- TMA producer ----------------
+    {
+      // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+      const bool issuer = elect_one();
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0;   // bit s: stage s has an issued load not yet seen complete by the consumer
@@ -335,18 +338,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const NodeEntry nd = p.nodes[node];
         const int a_outer = p.a_by_layer ? nd.y : nd.z;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           armed &= ~(1u << stage);
           uint8_t* sa = smem + stage * SM::STAGE_BYTES;
-          mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
-          tma_load_3d(&tmA, &full[stage], sa, kb * BK, mb * BM, a_outer);
-          tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BK, nb * BN, nd.y);
+          if (issuer) mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
+          if (issuer) tma_load_3d(&tmA, &full[stage], sa, kb * BK, p.row0 + mb * BM, a_outer);
+          if (issuer) tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BK, nb * BN, nd.y);
           armed |= 1u << stage;
           if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {
-        atomicOr(p.err, 1u);
+        if (issuer) atomicOr(p.err, 1u);
         *abort_flag = 1;
       }
       // drain: wait (bounded) until every issued copy has landed
@@ -362,8 +365,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    {
+      // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+      const bool issuer = elect_one();
       const uint32_t IDESC = idesc_f16(BN, p.ab_bf16);
       int stage = 0;
       uint32_t phase = 0;
@@ -371,32 +375,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        if (!mbar_wait(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * SM::STAGE_BYTES);
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+            if (issuer) mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
                      (kb > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&empty[stage]);
+          if (issuer) mma_commit(&empty[stage]);
           if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        mma_commit(&tfull[buf]);
+        if (issuer) mma_commit(&tfull[buf]);
         if (++buf == 2) { buf = 0; acc_phase ^= 1; }
       }
       if (!ok) {
-        atomicOr(p.err, 2u);
+        if (issuer) atomicOr(p.err, 2u);
         *abort_flag = 1;
       }
       // make sure no MMA is still writing TMEM before it is freed
-      mma_commit(drain);
+      if (issuer) mma_commit(drain);
       const unsigned long long t0 = global_ns();
       while (!mbar_try_wait(drain, 0)) {
         if (global_ns() - t0 > WAIT_LIMIT_NS) break;
@@ -420,7 +424,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int node = t / tiles_per_node, r = t - node * tiles_per_node;
       const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
       const NodeEntry nd = p.nodes[node];
-      const int row = mb * BM + row_in_tile;
+      const int row = p.row0 + mb * BM + row_in_tile;
       const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
       run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half);
@@ -436,6 +440,210 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(2 * BN) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (cluster of 2, tcgen05 cta_group::2) for 256-column tiles:
+// a pair computes 256 rows x 256 columns.  Each CTA loads its own 128 rows of
+// A and its half (128 rows) of the B tile, so per CTA a pipeline stage is
+// 32 KB instead of 48 KB and every B byte is fetched once per 256 output
+// rows: less shared-memory and L2 traffic per multiply-add than one CTA per
+// 128 x 256 tile.  The even CTA's single MMA thread issues
+// tcgen05.mma.cta_group::2 (M = 256); each CTA's accumulator rows land in its
+// own TMEM, so the epilogue is the one-CTA epilogue unchanged.
+//   full[s]   (even CTA) both CTAs' copies of stage s, counted in bytes
+//   empty[s]  (each CTA) stage s consumed (multicast commit)
+//   tfull[b]  (each CTA) accumulator b complete (multicast commit)
+//   tempty[b] (even CTA) accumulator b drained by both CTAs' epilogues
+// Rows [row0, row0 + 256 m_tiles) of every node; the caller covers a ragged
+// rest with the one-CTA kernel.  Every wait is bounded; the only unbounded
+// waits are the two cluster barriers that every thread reaches.
+struct SmemPair {
+  static constexpr int A_BYTES = BM * BK * 2;        // this CTA's 128 rows
+  static constexpr int B_BYTES = 128 * BK * 2;       // this CTA's 128 of the tile's 256 B rows
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = 6;
+  static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
+  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;
+};
+
+__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const TcGemmParams p) {
+  using SM = SmemPair;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SM::BAR_OFFSET);
+  uint64_t* empty = full + SM::STAGES;
+  uint64_t* tfull = empty + SM::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint32_t* skip_word = tmem_slot + 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SM::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], 2 * EPI_WARPS);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    // an earlier kernel of this forward already gave up on a wait: the pair
+    // skips its work (the even CTA decides for both)
+    *skip_word = *reinterpret_cast<volatile unsigned*>(p.err) & ERR_WAIT_TIMEOUT_MASK;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();   // both CTAs' barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool skip = ld_shared_cluster_u32(mapa_shared(smem_u32(skip_word), 0)) != 0;
+
+  const int tiles_per_node = p.m_tiles * p.n_tiles;
+  const int total = p.n_nodes * tiles_per_node;
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (skip) {
+    // nothing to do
+  } else if (warp == 0) {
+    {
+      // ---------------- TMA producer (both CTAs; whole warp, one elected lane issues) ----------------
+      const bool issuer = elect_one();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;
+      bool ok = true;
+      const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);   // the even CTA's full[0]
+      for (int t = cid; t < total && ok; t += ncl) {
+        const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+        const int nb = r / p.m_tiles, mp = r - nb * p.m_tiles;
+        const NodeEntry nd = p.nodes[node];
+        const int a_outer = p.a_by_layer ? nd.y : nd.z;
+        const int arow = p.row0 + mp * 256 + (int)rank * BM;
+        const int brow = nb * 256 + (int)rank * 128;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait_cluster_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+          armed &= ~(1u << stage);
+          uint8_t* sa = smem + stage * SM::STAGE_BYTES;
+          if (leader && issuer) mbar_expect_tx(&full[stage], 2 * SM::STAGE_BYTES);   // both CTAs' copies
+          const uint32_t fb = full0 + (uint32_t)(stage * sizeof(uint64_t));
+          if (issuer) tma_load_3d_pair(&tmA, fb, sa, kb * BK, arow, a_outer);
+          if (issuer) tma_load_3d_pair(&tmB, fb, sa + SM::A_BYTES, kb * BK, brow, nd.y);
+          armed |= 1u << stage;
+          if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+      if (!ok) {
+        if (issuer) atomicOr(p.err, 1u);
+        *abort_flag = 1;
+      }
+      if (*abort_flag && leader) {   // copies of both CTAs are counted on the even CTA's barriers
+        for (int s = 0; s < SM::STAGES; ++s) {
+          if (!(armed & (1u << s))) continue;
+          const unsigned long long t0 = global_ns();
+          while (!mbar_try_wait_cluster(&full[s], 0) && !mbar_try_wait_cluster(&full[s], 1)) {
+            if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (leader) {
+      // ---------------- MMA issuer (even CTA; whole warp, one elected lane issues) ----------------
+      const bool issuer = elect_one();
+      const uint32_t IDESC = idesc_f16(256, p.ab_bf16, 256);
+      int stage = 0;
+      uint32_t phase = 0;
+      int buf = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = cid; t < total && ok; t += ncl) {
+        if (!mbar_wait_cluster_warp(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait_cluster_warp(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * SM::STAGE_BYTES);
+          const uint32_t sb = sa + SM::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            if (issuer) mma_f16_pair(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+                         (kb > 0 || kk > 0) ? 1u : 0u);
+          if (issuer) mma_commit_pair(&empty[stage], 0x3);
+          if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        if (issuer) mma_commit_pair(&tfull[buf], 0x3);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      }
+      if (!ok) {
+        if (issuer) atomicOr(p.err, 2u);
+        *abort_flag = 1;
+      }
+      if (issuer) mma_commit_pair(drain, 0x1);   // no MMA writes either CTA's TMEM after this arrives
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(drain, 0)) {
+        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..9, both CTAs) ----------------
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int row_in_tile = quarter * 32 + lane;
+    const uint32_t tempty0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    int buf = 0;
+    uint32_t acc_phase = 0;
+    for (int t = cid; t < total; t += ncl) {
+      const bool got = mbar_wait_cluster(&tfull[buf], acc_phase, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) {
+        if (lane == 0) atomicOr(p.err, 4u);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mp = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = p.row0 + mp * 256 + (int)rank * BM + row_in_tile;
+      const bool valid = row < p.M;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
+      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0 + (uint32_t)(buf * sizeof(uint64_t)));
+      if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();   // no MMA, copy or epilogue of either CTA still uses TMEM or shared memory
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512) : "memory");
   }
 }
 
@@ -471,6 +679,59 @@ cudaError_t configure() {
                               Smem<BN>::TOTAL);
 }
 
+// Clusters of the pair kernel that fit on the device at once (persistent grid).
+template <int EPI>
+int& pair_clusters() {
+  static int n = 0;
+  return n;
+}
+
+template <int EPI>
+cudaError_t configure_pair() {
+  cudaError_t e = cudaFuncSetAttribute(tc_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SmemPair::TOTAL);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SmemPair::TOTAL;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 2; attr.val.clusterDim.y = 1; attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  // a device or driver that cannot place the pairs leaves them unused (the
+  // one-CTA kernel covers every row then)
+  if (cudaOccupancyMaxActiveClusters(&n, tc_gemm_pair_kernel<EPI>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  pair_clusters<EPI>() = n;
+  return cudaSuccess;
+}
+
+bool pair_available(int epi) {
+  switch (epi) {
+    case TC_EPI_F32: return pair_clusters<TC_EPI_F32>() > 0;
+    case TC_EPI_RESID: return pair_clusters<TC_EPI_RESID>() > 0;
+    case TC_EPI_RESID_ACT: return pair_clusters<TC_EPI_RESID_ACT>() > 0;
+    case TC_EPI_QKV_ROPE: return pair_clusters<TC_EPI_QKV_ROPE>() > 0;
+    case TC_EPI_SWIGLU: return pair_clusters<TC_EPI_SWIGLU>() > 0;
+    default: return false;
+  }
+}
+
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, cudaStream_t st) {
+  const int total = p.n_nodes * p.m_tiles * p.n_tiles;
+  const int cl = pair_clusters<EPI>();
+  if (cl <= 0) return cudaErrorInvalidConfiguration;
+  const int clusters = total < cl ? total : cl;
+  tc_gemm_pair_kernel<EPI><<<2 * clusters, NUM_THREADS, SmemPair::TOTAL, st>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t setup_tc_gemm() {
@@ -484,6 +745,11 @@ cudaError_t setup_tc_gemm() {
   if (e == cudaSuccess) e = configure<256, TC_EPI_RESID_ACT>();
   if (e == cudaSuccess) e = configure<256, TC_EPI_QKV_ROPE>();
   if (e == cudaSuccess) e = configure<256, TC_EPI_SWIGLU>();
+  if (e == cudaSuccess) e = configure_pair<TC_EPI_F32>();
+  if (e == cudaSuccess) e = configure_pair<TC_EPI_RESID>();
+  if (e == cudaSuccess) e = configure_pair<TC_EPI_RESID_ACT>();
+  if (e == cudaSuccess) e = configure_pair<TC_EPI_QKV_ROPE>();
+  if (e == cudaSuccess) e = configure_pair<TC_EPI_SWIGLU>();
   if (e == cudaSuccess) done = true;
   return e;
 }
@@ -506,6 +772,16 @@ cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 256-column tiles of 256 or more rows run on CTA pairs unless the
+// environment sets ARMT_GEMM_CTA_PAIRS=0 (then every tile runs on one CTA).
+bool tc_gemm_pairs_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("ARMT_GEMM_CTA_PAIRS");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 bool tc_gemm_supported(int m, int n, int k) {
   (void)m;
   return k % 8 == 0 && n % 16 == 0 && get_tensor_map_encoder() != nullptr;
@@ -518,11 +794,33 @@ cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, in
   CUtensorMap ta, tb;
   cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM, op.a_pitch, p.ab_bf16 != 0);
   if (e != cudaSuccess) return e;
+  p.k_blocks = (p.K + BK - 1) / BK;
+  p.row0 = 0;
+  if (bn == 256 && p.M >= 256 && tc_gemm_pairs_enabled() && pair_available(epi)) {
+    // rows [0, 256 floor(M / 256)) on CTA pairs, the rest on the one-CTA kernel
+    CUtensorMap tbp;
+    e = make_tmap_3d(&tbp, op.B, p.K, op.b_rows, op.b_outer, BK, 128, 0, p.ab_bf16 != 0);
+    if (e != cudaSuccess) return e;
+    TcGemmParams pp = p;
+    pp.m_tiles = p.M / 256;
+    pp.n_tiles = (p.N + 255) / 256;
+#define ARMT_TC_PAIR(E) \
+    if (epi == E) e = launch_pair<E>(ta, tbp, pp, st);
+    e = cudaErrorInvalidValue;
+    ARMT_TC_PAIR(TC_EPI_F32)
+    ARMT_TC_PAIR(TC_EPI_RESID)
+    ARMT_TC_PAIR(TC_EPI_RESID_ACT)
+    ARMT_TC_PAIR(TC_EPI_QKV_ROPE)
+    ARMT_TC_PAIR(TC_EPI_SWIGLU)
+#undef ARMT_TC_PAIR
+    if (e != cudaSuccess) return e;
+    p.row0 = pp.m_tiles * 256;
+    if (p.row0 >= p.M) return cudaSuccess;
+  }
   e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BK, bn, 0, p.ab_bf16 != 0);
   if (e != cudaSuccess) return e;
-  p.m_tiles = (p.M + BM - 1) / BM;
+  p.m_tiles = (p.M - p.row0 + BM - 1) / BM;
   p.n_tiles = (p.N + bn - 1) / bn;
-  p.k_blocks = (p.K + BK - 1) / BK;
 #define ARMT_TC_CASE(BNV, E) \
   if (bn == BNV && epi == E) return launch_kernel<BNV, E>(ta, tb, p, sm_count, st);
   ARMT_TC_CASE(256, TC_EPI_F32)

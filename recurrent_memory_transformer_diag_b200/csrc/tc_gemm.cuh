@@ -20,6 +20,7 @@ struct TcGemmParams {
   int n_nodes;
   int M, N, K;              // per node: rows, B rows (output columns), reduction
   int m_tiles, n_tiles, k_blocks;
+  int row0;                 // first row of the range this launch covers (rows row0 .. M-1)
   int a_by_layer;           // A's outer TMA coordinate: 0 = node slot, 1 = node layer
   int ab_bf16;              // operand type: 0 = fp16, 1 = bf16 (both operands alike)
   void* C; long long c_slot_stride; int ldc;
@@ -51,6 +52,7 @@ struct TcGemmOperands {
 
 cudaError_t setup_tc_gemm();
 int tc_pick_bn(int n);
+bool tc_gemm_pairs_enabled();
 bool tc_gemm_supported(int m, int n, int k);
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st);

@@ -17,6 +17,8 @@ pytestmark = pytest.mark.gpu
     (4, 200, 64, 384, 2),       # N = 64 tile width
     (2, 77, 128, 136, 3),       # N = 128, tiny ragged M and K
     (16, 1040, 3072, 2048, 16), # a full 1B wave of QKV shapes
+    (2, 512, 256, 128, 2),      # rows in whole 256-row CTA-pair tiles only
+    (1, 300, 304, 200, 1),      # one pair tile + a 44-row one-CTA rest, ragged N and K
 ])
 def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b, dtype):
     import torch
