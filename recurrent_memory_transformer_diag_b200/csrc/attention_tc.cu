@@ -38,7 +38,7 @@ using namespace tc;
 constexpr int HD = 64;
 constexpr int BQ = 128;                 // query rows per tile
 constexpr int BKEY = 128;               // keys per tile
-constexpr int NUM_THREADS = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (2 warpgroups)
+constexpr int NUM_THREADS = 352;        // warp 0 TMA, warps 1 / 10 MMA for warpgroup A / B, warps 2..9 softmax
 constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
 constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
 constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB loaded per stage (two 64-key blocks of 8 KB)
@@ -104,8 +104,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* s_empty = bar + 20;    // [w]
   uint64_t* p_full = bar + 22;     // [w]
   uint64_t* o_full = bar + 24;     // [w]
-  uint64_t* drain = bar + 26;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 27);
+  uint64_t* drain = bar + 26;      // [w]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 28);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -136,11 +136,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int b = 0; b < K_STAGES; ++b) {
       mbar_init(&k_full[b], 1);
-      mbar_init(&k_empty[b], 1);
+      mbar_init(&k_empty[b], 2);   // one release per MMA warp
     }
     for (int b = 0; b < V_STAGES; ++b) {
       mbar_init(&v_full[b], 1);
-      mbar_init(&v_empty[b], 1);
+      mbar_init(&v_empty[b], 2);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
@@ -148,7 +148,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&p_full[w], 4);
       mbar_init(&o_full[w], 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -181,7 +182,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // heads and steps of each warpgroup consumed by the earlier items, so every
   // barrier phase follows from them.
   struct Cursor {   // fields per warpgroup spelled out: no dynamically indexed (local-memory) arrays
-    int u, t, ntiles, nA, nB, kv0, qh0_a, qh0_b, sw0_a, sw0_b;
+    int u, t, j, k, ntiles, nA, nB, kv0, qh0_a, qh0_b, sw0_a, sw0_b;   // t = k * ntiles + j
   };
   auto load_item = [&](Cursor& c) {
     NodeEntry nd; int g, q0;
@@ -190,11 +191,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     c.nB = heads_b * c.ntiles;
   };
   auto first_step = [&](Cursor& c) {
-    c.u = blockIdx.x; c.t = 0; c.kv0 = 0; c.qh0_a = c.qh0_b = 0; c.sw0_a = c.sw0_b = 0;
+    c.u = blockIdx.x; c.t = 0; c.j = 0; c.k = 0; c.kv0 = 0; c.qh0_a = c.qh0_b = 0; c.sw0_a = c.sw0_b = 0;
     load_item(c);
   };
   auto advance = [&](Cursor& c) -> bool {
-    if (c.t + 1 < c.nA) { ++c.t; return true; }
+    if (c.t + 1 < c.nA) {
+      ++c.t;
+      if (++c.j == c.ntiles) { c.j = 0; ++c.k; }
+      return true;
+    }
     const int u = c.u + gridDim.x;
     if (u >= n_items) return false;
     c.kv0 += c.nA;
@@ -203,7 +208,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     c.sw0_a += c.nA;
     c.sw0_b += c.nB;
     c.u = u;
-    c.t = 0;
+    c.t = 0; c.j = 0; c.k = 0;
     load_item(c);
     return true;
   };
@@ -245,7 +250,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       };
       auto load_v = [&](const Cursor& c) -> bool {
         const int kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
-        const int j = c.t % c.ntiles;
+        const int j = c.j;
         if (!mbar_wait_warp(&v_empty[vs], ((kidx / V_STAGES) & 1) ^ 1, abort_flag)) return false;
         NodeEntry nd; int g, q0, nt;
         decode(c.u, nd, g, q0, nt);
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         first_step(c);
         bool has_prev = false;
         while (ok) {
-          const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
+          const int k = c.k, j = c.j;
           // this step's Q tiles must be on their way (normally issued a head earlier)
           const int ha = c.qh0_a + k, hb = c.qh0_b + k;
           while (ok && qi_a <= ha) ok = q_issue(0, true) > 0;
@@ -306,80 +311,104 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (!mbar_try_wait(&v_full[b], 0) && !mbar_try_wait(&v_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
       }
     }
-  } else if (warp == 1) {
-    {
-      // ---------------- MMA issuer (the whole warp runs the loop; one elected lane issues) ----------------
-      const bool issuer = elect_one();
-      const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
-      const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
-      auto issue_s = [&](int w, const Cursor& c) -> bool {
-        const int k = c.t / c.ntiles, j = c.t - k * c.ntiles;
-        const int hidx = (w ? c.qh0_b : c.qh0_a) + k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
-        const int qb = w * 2 + (hidx & 1), ks = kidx % K_STAGES;
-        if (j == 0 && !mbar_wait_warp(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
+  } else if (warp == 1 || warp == 10) {
+    // ---------------- MMA issuers: warp 1 for warpgroup A, warp 10 for B ----------------
+    // Each runs the step sequence on the whole warp; one elected lane issues.
+    // Two issuers halve the per-step issue chain (waits, descriptors, MMAs);
+    // the K/V stages are released by both (count 2).
+    const int w = warp == 1 ? 0 : 1;
+    const bool issuer = elect_one();
+    const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
+    const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
+    auto active = [&](const Cursor& c) { return w == 0 || c.t < c.nB; };
+    // S_w = Q_w K_j^T for step c
+    auto issue_s = [&](const Cursor& c) -> bool {
+      const int hidx = (w ? c.qh0_b : c.qh0_a) + c.k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
+      const int qb = w * 2 + (hidx & 1), ks = kidx % K_STAGES;
+      if (c.j == 0 && !mbar_wait_warp(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
+      if (!mbar_wait_warp(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
+      if (!mbar_wait_warp(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
+      const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
+#pragma unroll
+      for (int kk = 0; kk < HD / 16; ++kk)
+        if (issuer) mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+      if (issuer) mma_commit(&s_full[w]);
+      if (c.j == c.ntiles - 1 && issuer) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
+      return true;
+    };
+    // O_w (+)= P_w [V_j | 1] for step c
+    auto issue_o = [&](const Cursor& c) -> bool {
+      const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
+      if (!mbar_wait_warp(&p_full[w], sidx & 1, abort_flag)) return false;
+      if (!mbar_wait_warp(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
+      const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
+#pragma unroll
+      for (int kb = 0; kb < BKEY / 64; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          if (issuer)
+            mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
+                    sw128_desc(va + kb * VT_BLK + kk * 32), idesc_o, (c.j > 0 || kb > 0 || kk > 0));
+      if (issuer) mma_commit(&o_full[w]);
+      return true;
+    };
+    // release of step c's K (V) stage: after this warp's product that reads
+    // it, or, for a step warpgroup B does not take, once the stage is loaded
+    // (so that the arrival counts toward this use of the stage, not an earlier one)
+    auto release_k = [&](const Cursor& c) -> bool {
+      const int kidx = c.kv0 + c.t, ks = kidx % K_STAGES;
+      if (active(c)) {
+        if (issuer) mma_commit(&k_empty[ks]);
+      } else {
         if (!mbar_wait_warp(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
-        if (!mbar_wait_warp(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
-        const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          if (issuer) mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
-        if (issuer) mma_commit(&s_full[w]);
-        if (j == c.ntiles - 1 && issuer) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
-        return true;
-      };
-      auto issue_o = [&](int w, const Cursor& c) -> bool {
-        const int j = c.t % c.ntiles;
-        const int sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
-        if (!mbar_wait_warp(&p_full[w], sidx & 1, abort_flag)) return false;
+        if (issuer) mbar_arrive(&k_empty[ks]);
+      }
+      return true;
+    };
+    auto release_v = [&](const Cursor& c) -> bool {
+      const int kidx = c.kv0 + c.t, vs = kidx % V_STAGES;
+      if (active(c)) {
+        if (issuer) mma_commit(&v_empty[vs]);
+      } else {
         if (!mbar_wait_warp(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
-        const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
-#pragma unroll
-        for (int kb = 0; kb < BKEY / 64; ++kb)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            if (issuer) mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
-                    sw128_desc(va + kb * VT_BLK + kk * 32), idesc_o, (j > 0 || kb > 0 || kk > 0));
-        if (issuer) mma_commit(&o_full[w]);
-        return true;
-      };
-      // S of the next step (next key tile, next head or next item) is issued
-      // before O of the current one (the S buffer is free once the softmax
-      // has the scores in registers), so a warpgroup finds its next scores
-      // computed when it finishes a tile.  Order per step: S_A(next), O_A,
-      // S_B(next), O_B: each warpgroup's O is issued as soon as its P is ready.
-      bool ok = true;
-      if (blockIdx.x < n_items) {
-        Cursor cur;
-        first_step(cur);
-        ok = issue_s(0, cur);
-        if (ok && cur.nB > 0) ok = issue_s(1, cur);
-        if (ok && issuer) mma_commit(&k_empty[cur.kv0 % K_STAGES]);   // K_0 read by both S products
-        while (ok) {
-          Cursor nxt = cur;
-          const bool more = advance(nxt);
-          if (more && !issue_s(0, nxt)) { ok = false; break; }
-          if (!issue_o(0, cur)) { ok = false; break; }
-          if (more && nxt.t < nxt.nB && !issue_s(1, nxt)) { ok = false; break; }
-          if (more && issuer) mma_commit(&k_empty[(nxt.kv0 + nxt.t) % K_STAGES]);
-          if (cur.t < cur.nB && !issue_o(1, cur)) { ok = false; break; }
-          if (issuer) mma_commit(&v_empty[(cur.kv0 + cur.t) % V_STAGES]);   // V_t no longer read once these finish
-          if (!more) break;
-          cur = nxt;
+        if (issuer) mbar_arrive(&v_empty[vs]);
+      }
+      return true;
+    };
+    // S of the next step is issued before O of the current one (the S buffer
+    // is free once the softmax has the scores in registers), so the softmax
+    // finds its next scores computed when it finishes a tile.
+    bool ok = true;
+    if (blockIdx.x < n_items) {
+      Cursor cur;
+      first_step(cur);
+      if (active(cur)) ok = issue_s(cur);
+      if (ok) ok = release_k(cur);
+      while (ok) {
+        Cursor nxt = cur;
+        const bool more = advance(nxt);
+        if (more) {
+          if (active(nxt) && !issue_s(nxt)) { ok = false; break; }
+          if (!release_k(nxt)) { ok = false; break; }
         }
+        if (active(cur) && !issue_o(cur)) { ok = false; break; }
+        if (!release_v(cur)) { ok = false; break; }
+        if (!more) break;
+        cur = nxt;
       }
-      if (!ok) {
-        if (issuer) atomicOr(p.err, 32u);
-        *abort_flag = 1;
-      }
-      if (issuer) mma_commit(drain);
-      const unsigned long long t0 = global_ns();
-      while (!mbar_try_wait(drain, 0)) {
-        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
-      }
+    }
+    if (!ok) {
+      if (issuer) atomicOr(p.err, 32u);
+      *abort_flag = 1;
+    }
+    if (issuer) mma_commit(&drain[w]);   // no MMA of this warp still writes TMEM after this arrives
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(&drain[w], 0)) {
+      if (global_ns() - t0 > WAIT_LIMIT_NS) break;
     }
   } else {
     // ---------------- softmax (warpgroup w, one thread per query row) ----------------
@@ -426,9 +455,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = q0 + rloc;
       const int nw = heads * ntiles;
       float m_used = -INFINITY;
-      for (int t = 0; t < nw && ok; ++t) {
+      for (int t = 0, j = 0, k = 0; t < nw && ok; ++t, j = (j + 1 == ntiles) ? 0 : j + 1, k += (j == 0)) {
         const int sidx = sbase + t;
-        const int k = t / ntiles, j = t - k * ntiles;
         if (j == 0) m_used = -INFINITY;
         bool got = mbar_wait(&s_full[w], sidx & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
