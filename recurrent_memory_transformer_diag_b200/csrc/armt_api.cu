@@ -97,7 +97,9 @@ armt_status validate_config(const armt_config* c, const char** why) {
   const long long P = 2LL * c->d_key * c->dpfp_nu;
   if (P > 1024) { *why = "phi dimension 2*d_key*nu must be <= 1024"; return ARMT_ERR_UNSUPPORTED; }
   if (c->n_mem > 32) { *why = "n_mem must be <= 32"; return ARMT_ERR_UNSUPPORTED; }
-  if (((long long)c->n_mem * P + (long long)c->n_mem * c->n_mem + 17LL * c->n_mem) * 4 > 200 * 1024) {
+  if (((long long)c->n_mem * P + (long long)c->n_mem * c->n_mem + 17LL * c->n_mem) * 4 > 200 * 1024 ||
+      ((long long)P + (long long)c->n_mem * P + (long long)(c->n_mem < 32 ? c->n_mem : 32) * 2 * c->d_key +
+       2LL * c->n_mem + (long long)c->n_mem * c->n_mem) * 4 > 200 * 1024) {
     *why = "n_mem * phi dimension too large for the write kernel"; return ARMT_ERR_UNSUPPORTED;
   }
   if (c->dtype == ARMT_BF16 && (c->d_model % 8 || c->d_ffn % 8 || (c->n_heads * c->head_dim) % 8 || P % 8)) {

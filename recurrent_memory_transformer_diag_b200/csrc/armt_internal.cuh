@@ -155,6 +155,8 @@ cudaError_t launch_attention_simt(const Dims& dm, const NodeEntry* nodes, int n,
                                   const void* qkv, void* out, cudaStream_t st);
 cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* gu,
                           void* u, cudaStream_t st);
+// shared memory of memw_phi (bytes)
+size_t memw_phi_smem(const Dims& dm);
 cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                             float* z_state, float* phik, float* gram, float* coef, float* gamma,
                             cudaStream_t st);

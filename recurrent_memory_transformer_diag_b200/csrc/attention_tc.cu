@@ -42,20 +42,25 @@ constexpr int NUM_THREADS = 352;        // warp 0 TMA, warps 1 / 10 MMA for warp
 constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
 constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
 constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB loaded per stage (two 64-key blocks of 8 KB)
-constexpr int ON = HD + 16;             // O columns: 64 dims, the row-sum column, 15 zero columns
-constexpr int VT_BLK = ON * 128;        // V^T block in shared memory: 80 rows of 64 keys (10 KB)
-constexpr int P_BYTES = BQ * BKEY * 2;  // 32 KB (two 64-key blocks of 16 KB)
-constexpr int K_STAGES = 3;             // K is needed first (S of the next step): deeper ring
-constexpr int V_STAGES = 2;             // V^T only at O, a softmax later
+constexpr int VT_BLK = HD * 128;        // V^T block in shared memory: 64 rows (dims) of 64 keys (8 KB)
+constexpr int K_STAGES = 4;             // K is needed first (S of the next step): deeper ring
+constexpr int V_STAGES = 3;             // V^T only at O, a softmax later
 constexpr int OFF_Q = 0;                               // [2 warpgroups][2 buffers]
 constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // [K_STAGES]
 constexpr int OFF_VT = OFF_K + K_STAGES * K_BYTES;     // [V_STAGES][2 blocks of VT_BLK]
-constexpr int OFF_P = OFF_VT + V_STAGES * 2 * VT_BLK;  // [2 warpgroups]
-constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-constexpr int SMEM_TOTAL = OFF_BAR + 256 + 1024;
+constexpr int OFF_BAR = OFF_VT + V_STAGES * 2 * VT_BLK;
+constexpr int SMEM_TOTAL = OFF_BAR + 512 + 1024;
 static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
-constexpr int TMEM_COLS = 512;          // S_A 0, S_B 128, O_A 256, O_B 256 + ON
+// TMEM columns: S_A, S_B (fp32 scores, 128 each), O_A, O_B (fp32, 64 each),
+// P_A, P_B (fp16 probabilities packed in pairs, 64 each)
+constexpr int TM_S = 0, TM_O = 2 * BKEY, TM_P = TM_O + 2 * HD;
+constexpr int TMEM_COLS = 512;
+static_assert(TM_P + 2 * (BKEY / 2) <= TMEM_COLS, "tensor memory");
 constexpr float RESCALE_THRESHOLD = 8.f;
+// Share of the exponentials taken off the MUFU unit (every POLY_EVERY-th
+// pair by polynomial; 0 = none).  A quarter measured 3 % faster than none on
+// the 1B wave (the softmax is mostly issue-bound, so more would cost).
+constexpr int POLY_EVERY = 4;
 
 struct AttnParams {
   const NodeEntry* nodes;
@@ -76,16 +81,22 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// P row of 128 keys from 64 packed fp16 pairs (pk[i] = keys 2i, 2i+1): K-major
-// operand, two 64-key blocks, 128-byte swizzle (16-byte chunk c of row r at
-// chunk position c ^ (r & 7)).
-__device__ __forceinline__ void store_p(uint8_t* pbuf, int row, const uint32_t* pk) {
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {   // 16-byte chunk c = keys 8c .. 8c+7
-    uint8_t* blk = pbuf + (c >> 3) * (BQ * 128) + row * 128;
-    *reinterpret_cast<uint4*>(blk + (((c & 7) ^ (row & 7)) << 4)) =
-        make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-  }
+// 2^x on the FMA pipe, for the share of the probabilities that bypasses the
+// MUFU unit: x = j + f with j = round(x) (the 1.5 * 2^23 shift puts j in the
+// low mantissa bits of t) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
+// fitted here by the Remez exchange for minimal relative error (7.5e-5, well
+// under the fp16 rounding P goes through next); 2^j is added to the exponent
+// field.  x is clamped to -125 so the exponent field stays normal (-inf ->
+// 2^-125, zero in fp16).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const float f = x - (t - 12582912.f);
+  float q = fmaf(0.0551716685f, f, 0.2426111251f);
+  q = fmaf(q, f, 0.6932609677f);
+  q = fmaf(q, f, 0.9999280572f);
+  // bits(t) = bits(1.5 * 2^23) + j and bits(1.5 * 2^23) << 23 == 0 (mod 2^32)
+  return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -94,18 +105,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* q_full = bar;          // [w][2]
-  uint64_t* q_empty = bar + 4;     // [w][2]
-  uint64_t* k_full = bar + 8;      // [K_STAGES]
-  uint64_t* k_empty = bar + 11;    // [K_STAGES]
-  uint64_t* v_full = bar + 14;     // [V_STAGES]
-  uint64_t* v_empty = bar + 16;    // [V_STAGES]
-  uint64_t* s_full = bar + 18;     // [w]
-  uint64_t* s_empty = bar + 20;    // [w]
-  uint64_t* p_full = bar + 22;     // [w]
-  uint64_t* o_full = bar + 24;     // [w]
-  uint64_t* drain = bar + 26;      // [w]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 28);
+  uint64_t* q_full = bar;                        // [w][2]
+  uint64_t* q_empty = q_full + 4;                // [w][2]
+  uint64_t* k_full = q_empty + 4;                // [K_STAGES]
+  uint64_t* k_empty = k_full + K_STAGES;         // [K_STAGES]
+  uint64_t* v_full = k_empty + K_STAGES;         // [V_STAGES]
+  uint64_t* v_empty = v_full + V_STAGES;         // [V_STAGES]
+  uint64_t* s_full = v_empty + V_STAGES;         // [w]
+  uint64_t* s_empty = s_full + 2;                // [w]
+  uint64_t* p_full = s_empty + 2;                // [w]
+  uint64_t* o_full = p_full + 2;                 // [w]
+  uint64_t* drain = o_full + 2;                  // [w]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -158,17 +169,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                  "r"(TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  if (warp >= 2) {
-    // rows HD .. ON-1 of every V^T block: a row of ones (row sums), then zeros;
-    // TMA only ever writes rows 0 .. HD-1
-    for (int e = threadIdx.x - 64; e < V_STAGES * 2 * 16 * 8; e += NUM_THREADS - 64) {
-      const int blk = e / (16 * 8), rr = (e / 8) % 16, chunk = e % 8;
-      const uint32_t one2 = 0x3C003C00u;   // two fp16 ones
-      const uint4 val = rr == 0 ? make_uint4(one2, one2, one2, one2) : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(smem + OFF_VT + blk * VT_BLK + (HD + rr) * 128 + chunk * 16) = val;
-    }
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int w = warp == 1 ? 0 : 1;
     const bool issuer = elect_one();
     const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
-    const uint32_t idesc_o = idesc_f16(ON, 0);     // 128 x 80 x 16
+    const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x 64 x 16
     auto active = [&](const Cursor& c) { return w == 0 || c.t < c.nB; };
     // S_w = Q_w K_j^T for step c
     auto issue_s = [&](const Cursor& c) -> bool {
@@ -333,7 +333,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk)
-        if (issuer) mma_f16(tmem_base + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+        if (issuer) mma_f16(tmem_base + TM_S + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
       if (issuer) mma_commit(&s_full[w]);
       if (c.j == c.ntiles - 1 && issuer) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
       return true;
@@ -344,15 +344,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait_warp(&p_full[w], sidx & 1, abort_flag)) return false;
       if (!mbar_wait_warp(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t pa = smem_u32(smem + OFF_P + w * P_BYTES);
+      const uint32_t pa = tmem_base + TM_P + w * (BKEY / 2);   // P_w in TMEM: 8 columns per 16 keys
       const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
 #pragma unroll
       for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           if (issuer)
-            mma_f16(tmem_base + 2 * BKEY + w * ON, sw128_desc(pa + kb * (BQ * 128) + kk * 32),
-                    sw128_desc(va + kb * VT_BLK + kk * 32), idesc_o, (c.j > 0 || kb > 0 || kk > 0));
+            mma_f16_ts(tmem_base + TM_O + w * HD, pa + (kb * 4 + kk) * 8, sw128_desc(va + kb * VT_BLK + kk * 32),
+                       idesc_o, (c.j > 0 || kb > 0 || kk > 0));
       if (issuer) mma_commit(&o_full[w]);
       return true;
     };
@@ -416,25 +416,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t s_tm = tmem_base + lane_off + w * BKEY;
-    const uint32_t o_tm = tmem_base + lane_off + 2 * BKEY + w * ON;
-    uint8_t* pbuf = smem + OFF_P + w * P_BYTES;
+    const uint32_t s_tm = tmem_base + lane_off + TM_S + w * BKEY;
+    const uint32_t o_tm = tmem_base + lane_off + TM_O + w * HD;
+    const uint32_t p_tm = tmem_base + lane_off + TM_P + w * (BKEY / 2);
     const int heads = w == 0 ? heads_a : heads_b;
     int sbase = 0;
     bool ok = true;
     bool first = true;          // no O issued for this warpgroup yet
     bool pend = false;          // a finished head whose O has not been read
     f16* pend_dst = nullptr;    // its output row (nullptr: a padding row)
+    float pend_l = 1.f;         // its row sum of P
     int last_sidx = 0;
-    // O of a finished head (complete, waited for): row sum in column 64,
-    // normalise, fp16 row of the head's 64 outputs
-    auto finalize = [&](f16* dst) {
-      uint32_t orr[HD], osum[16];
+    // O of a finished head (complete, waited for): normalise by the row sum,
+    // fp16 row of the head's 64 outputs
+    auto finalize = [&](f16* dst, float l) {
+      uint32_t orr[HD];
       tmem_ld64_nowait(o_tm, orr);
-      tmem_ld16_nowait(o_tm + HD, osum);
       tmem_wait_ld();
       if (dst) {
-        const float inv = 1.f / __uint_as_float(osum[0]);
+        const float inv = 1.f / l;
 #pragma unroll
         for (int q = 0; q < HD / 8; ++q) {
           uint4 v;
@@ -455,9 +455,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row = q0 + rloc;
       const int nw = heads * ntiles;
       float m_used = -INFINITY;
+      float l = 0.f;             // row sum of P at the running max m_used
       for (int t = 0, j = 0, k = 0; t < nw && ok; ++t, j = (j + 1 == ntiles) ? 0 : j + 1, k += (j == 0)) {
         const int sidx = sbase + t;
-        if (j == 0) m_used = -INFINITY;
+        if (j == 0) { m_used = -INFINITY; l = 0.f; }
         bool got = mbar_wait(&s_full[w], sidx & 1, abort_flag);
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
         tc_fence_after();
@@ -497,16 +498,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           corr = exp2f(m_used - m_tile);
           m_used = m_tile;
           rescale = true;
+          l *= corr;
         }
         // P = 2^(s - m) as packed fp16 pairs, computed before waiting for the
         // previous O (the exponentials overlap that product)
+        // (pairs i with i % POLY_EVERY == POLY_EVERY - 1 on the FMA pipe, the
+        // rest on MUFU); row sum in fp32
         uint32_t pk[BKEY / 2];
+        float l2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < BKEY / 2; ++i) {
-          const __half2 h2 = __floats2half2_rn(ex2_approx(fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, -m_used)),
-                                               ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, -m_used)));
+          const float x0 = fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, -m_used);
+          const float x1 = fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, -m_used);
+          const bool poly = POLY_EVERY > 0 && i % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1;
+          const float e0 = poly ? ex2_poly(x0) : ex2_approx(x0);
+          const float e1 = poly ? ex2_poly(x1) : ex2_approx(x1);
+          l2[i & 3] += e0 + e1;
+          const __half2 h2 = __floats2half2_rn(e0, e1);
           pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
         }
+        l += (l2[0] + l2[1]) + (l2[2] + l2[3]);
         // the previous step's O must be complete: its MMA read the P buffer,
         // and O is read (head done) or rescaled below
         if (!first) {
@@ -514,26 +525,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
           tc_fence_after();
         }
-        store_p(pbuf, rloc, pk);
+        tmem_st64(p_tm, pk);        // P_w: this thread's row, keys 2c, 2c+1 in column c
         if (pend) {   // the previous step ended a head: normalise its O and store it
-          finalize(pend_dst);
+          finalize(pend_dst, pend_l);
           pend = false;
         }
         if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
-          uint32_t orr[HD], osum[16];
+          uint32_t orr[HD];
           tmem_ld64_nowait(o_tm, orr);
-          tmem_ld16_nowait(o_tm + HD, osum);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) osum[i] = __float_as_uint(__uint_as_float(osum[i]) * corr);
           tmem_st64(o_tm, orr);
-          tmem_st16(o_tm + HD, osum);
-          tmem_wait_st();
         }
+        tmem_wait_st();
         tc_fence_before();
-        fence_proxy_async_smem();   // P written by this thread -> visible to the tensor core
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[w]);
         first = false;
@@ -541,6 +547,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pend = true;
           pend_dst = row < p.Tp ? p.out + ((long long)nd.z * p.Tp + row) * (p.H * HD) + (g * grp + w + 2 * k) * HD
                                 : nullptr;
+          pend_l = l;
           last_sidx = sidx;
         }
       }
@@ -550,7 +557,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool got = mbar_wait(&o_full[w], last_sidx & 1, abort_flag);
       if (__all_sync(0xffffffffu, got)) {
         tc_fence_after();
-        finalize(pend_dst);
+        finalize(pend_dst, pend_l);
       } else {
         ok = false;
       }

@@ -32,39 +32,48 @@ __device__ __forceinline__ float warp_sum_m(float v) {
 }
 
 // kv: [slot][M][dk + d] (k first), phik: [slot][M][P], gram: [slot][M][M],
-// coef/gamma: [slot][M].  One block per node (one warp per memory row for the
-// features, warps over row pairs for the Gram matrix, one thread for the
-// M-step recurrence, all threads for the z update).
-__global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
+// coef/gamma: [slot][M].  One block per node: one warp per memory row for the
+// features (phi kept in shared memory for the Gram matrix), warps over row
+// pairs for the Gram matrix, one thread for the M-step recurrence, all
+// threads for the z update.
+__global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, int P, int nu,
                                 const float* kv, float* z_state, float* phik, float* gram, float* coef,
                                 float* gamma, float eps) {
   extern __shared__ float sh[];
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* r = sh + warp * 2 * dk;   // [nw][2 dk]
-  float* gam = sh + nw * 2 * dk;   // [M]
-  float* zp0 = gam + M;            // [M]   z_0 . phi_j
+  const int n2 = 2 * dk;
+  float* zs = sh;                  // [P]     z before the write
+  float* phs = zs + P;             // [M][P]  phi_j
+  float* r = phs + M * P;          // [nw][2 dk]
+  float* gam = r + nw * n2;        // [M]
+  float* zp0 = gam + M;            // [M]     z_0 . phi_j
   float* G = zp0 + M;              // [M][M]
   const NodeEntry nd = nodes[blockIdx.x];
   const int slot = nd.z, layer = nd.y;
   float* z = z_state + (long long)layer * P;
-  const float* ph_all = phik + (long long)slot * M * P;
-  const int n2 = 2 * dk;
+  for (int p = threadIdx.x; p < P; p += blockDim.x) zs[p] = z[p];
+  __syncthreads();
   for (int j = warp; j < M; j += nw) {
     const float* k = kv + ((long long)slot * M + j) * (dk + d);
+    float* rw = r + warp * n2;
     for (int c = lane; c < dk; c += 32) {
-      r[c] = fmaxf(k[c], 0.f);
-      r[c + dk] = fmaxf(-k[c], 0.f);
+      const float kc = k[c];
+      rw[c] = fmaxf(kc, 0.f);
+      rw[c + dk] = fmaxf(-kc, 0.f);
     }
     __syncwarp();
-    float* ph = phik + ((long long)slot * M + j) * P;
+    float* phj = phs + j * P;
+    float* phg = phik + ((long long)slot * M + j) * P;
     float zp = 0.f;
-    for (int p = lane; p < P; p += 32) {
-      const int n = p / n2 + 1, jj0 = p - (n - 1) * n2;
-      int jj = (jj0 - n) % n2;
-      if (jj < 0) jj += n2;
-      const float f = r[jj0] * r[jj];
-      ph[p] = f;
-      zp = fmaf(z[p], f, zp);
+    for (int n = 1; n <= nu; ++n) {      // block n: r_i * r_{(i - n) mod 2dk} (nu <= 2 dk)
+      for (int i = lane; i < n2; i += 32) {
+        const int i2 = i - n < 0 ? i - n + n2 : i - n;
+        const float f = rw[i] * rw[i2];
+        const int p = (n - 1) * n2 + i;
+        phj[p] = f;
+        phg[p] = f;
+        zp = fmaf(zs[p], f, zp);
+      }
     }
     zp = warp_sum_m(zp);
     if (lane == 0) zp0[j] = zp;
@@ -74,8 +83,8 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
   for (int pair = warp; pair < M * M; pair += nw) {
     const int a = pair / M, b = pair - a * M;
     if (b < a) continue;
-    const float* pa = ph_all + (long long)a * P;
-    const float* pb = ph_all + (long long)b * P;
+    const float* pa = phs + a * P;
+    const float* pb = phs + b * P;
     float g = 0.f;
     for (int p = lane; p < P; p += 32) g = fmaf(pa[p], pb[p], g);
     g = warp_sum_m(g);
@@ -98,19 +107,24 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
   __syncthreads();
   for (int e = threadIdx.x; e < M * M; e += blockDim.x) gram[(long long)slot * M * M + e] = G[e];
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    float acc = z[p];
-    for (int j = 0; j < M; ++j) acc = fmaf(gam[j], ph_all[(long long)j * P + p], acc);
+    float acc = zs[p];
+    for (int j = 0; j < M; ++j) acc = fmaf(gam[j], phs[j * P + p], acc);
     z[p] = acc;
   }
+}
+
+size_t memw_phi_smem(const Dims& dm) {
+  const int nw = dm.M < 32 ? dm.M : 32;
+  return ((size_t)dm.P + (size_t)dm.M * dm.P + (size_t)nw * 2 * dm.dk + 2 * dm.M + (size_t)dm.M * dm.M) *
+         sizeof(float);
 }
 
 cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                             float* z_state, float* phik, float* gram, float* coef, float* gamma,
                             cudaStream_t st) {
   const int nw = dm.M < 32 ? dm.M : 32;
-  const size_t sh = ((size_t)nw * 2 * dm.dk + 2 * dm.M + (size_t)dm.M * dm.M) * sizeof(float);
-  memw_phi_kernel<<<n, nw * 32, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, z_state, phik, gram, coef,
-                                          gamma, dm.mem_eps);
+  memw_phi_kernel<<<n, nw * 32, memw_phi_smem(dm), st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, dm.nu, kv, z_state, phik,
+                                                         gram, coef, gamma, dm.mem_eps);
   return cudaGetLastError();
 }
 
@@ -269,8 +283,20 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
 // Same computation with 16-byte accesses (P % 4 == 0): lane l owns the
 // column groups 4 (l + 32 c) .. +3, c < C4, so A rows are read and written as
 // float4 and every phi read from shared memory is one 16-byte load serving
-// 4 columns of both rows.  At most 128 registers: two blocks per SM.
-template <int C4, int MT>
+// 4 columns of both rows.  At most 128 registers: two blocks per SM.  With
+// PF, each warp's next two rows are copied into shared memory (cp.async, a
+// two-buffer ring per warp) while it works on the current two, so the A
+// stream's latency overlaps the arithmetic.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int C4, int MT, bool PF>
 __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
                                                                  const float* kv, const float* phik,
                                                                  const float* gram, const float* coef,
@@ -281,6 +307,7 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
   float* G = ph + M * P;             // [M][M]
   float* cf = G + M * M;             // [M]
   float* dots = cf + M;              // [8][R][M]  delta_j per warp and row
+  float* pf = sh + ((M * P + M * M + M + 8 * R * M + 3) & ~3);   // PF: [8 warps][2][R][P] rows of A in flight (16-byte aligned)
   const NodeEntry nd = nodes[blockIdx.y];
   const int slot = nd.z, layer = nd.y;
   const int P4 = P >> 2;
@@ -301,15 +328,40 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
   const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
   const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
   const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+  // rows i0n + 8 r of this warp -> buffer b (each lane copies the 16-byte
+  // groups it later reads itself)
+  auto issue_rows = [&](int i0n, int b) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = i0n + 8 * r;
+      if (i < i_end) {
+        const float* src = A_state + ((long long)layer * d + i) * P;
+        float* dst = pf + ((warp * 2 + b) * R + r) * P;
+#pragma unroll
+        for (int c = 0; c < C4; ++c) {
+          const int q = lane + 32 * c;
+          if (q < P4) cp_async16(dst + 4 * q, src + 4 * q);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  int buf = 0;
+  if (PF) issue_rows(i_begin + warp, 0);
   for (int i0 = i_begin + warp; i0 < i_end; i0 += 8 * R) {
     float4 a[R][C4];
     float v[R];
     bool has[R];
+    if (PF) {
+      issue_rows(i0 + 8 * R, buf ^ 1);   // the next pass (an empty group past the end)
+      cp_async_wait<1>();                // this pass's rows have landed
+    }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int i = i0 + 8 * r;
       has[r] = i < i_end;
-      const float4* Arow = reinterpret_cast<const float4*>(A_state + ((long long)layer * d + (has[r] ? i : i0)) * P);
+      const float4* Arow = PF ? reinterpret_cast<const float4*>(pf + ((warp * 2 + buf) * R + r) * P)
+                              : reinterpret_cast<const float4*>(A_state + ((long long)layer * d + (has[r] ? i : i0)) * P);
       v[r] = (lane < M && has[r]) ? kvj[i] : 0.f;
 #pragma unroll
       for (int c = 0; c < C4; ++c) {
@@ -317,6 +369,7 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
         a[r][c] = (q < P4 && has[r]) ? Arow[q] : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
+    buf ^= 1;
     // a_r . phi_j for all rows and j at once (independent accumulators)
     float part[R][MT];
 #pragma unroll
@@ -396,12 +449,20 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
     }
     __syncwarp();
   }
+  if (PF) cp_async_wait<0>();
   if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
 static size_t memw_update_smem(const Dims& dm) {
   return ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 8 * MEMW_R * dm.M) * sizeof(float);
 }
+
+// with the per-warp two-buffer ring of A rows; used when two blocks still fit on an SM
+static size_t memw_update_pf_smem(const Dims& dm) {
+  const size_t base = ((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + dm.M + 8 * MEMW_R * dm.M + 3) & ~(size_t)3;
+  return (base + (size_t)8 * 2 * MEMW_R * dm.P) * sizeof(float);
+}
+constexpr size_t MEMW_PF_SMEM_MAX = 110 * 1024;
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                                const float* phik, const float* gram, const float* coef, float* A_state,
@@ -419,11 +480,20 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     else ARMT_MEMW_CASE(C, 32)          \
   }
   if (dm.M > 32) return cudaErrorInvalidValue;
-  if (dm.P % 4 == 0 && dm.P <= 1024) {   // 16-byte path
+  const bool aligned = (reinterpret_cast<uintptr_t>(A_state) & 15) == 0 && (reinterpret_cast<uintptr_t>(a_act) & 7) == 0;
+  if (dm.P % 4 == 0 && dm.P <= 1024 && aligned) {   // 16-byte path
     const int c4 = (dm.P / 4 + 31) / 32;
-#define ARMT_MEMWV_CASE(C, MT)                                                                                \
-  memw_update_vec_kernel<C, MT><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
-                                                       A_state, (f16*)a_act, err);
+    const size_t sh_pf = memw_update_pf_smem(dm);
+    const bool pf = sh_pf <= MEMW_PF_SMEM_MAX;
+#define ARMT_MEMWV_CASE(C, MT)                                                                                      \
+  {                                                                                                                 \
+    if (pf)                                                                                                         \
+      memw_update_vec_kernel<C, MT, true><<<grid, 256, sh_pf, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, \
+                                                                    coef, A_state, (f16*)a_act, err);               \
+    else                                                                                                            \
+      memw_update_vec_kernel<C, MT, false><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram,   \
+                                                                  coef, A_state, (f16*)a_act, err);                 \
+  }
 #define ARMT_MEMWV_M(C)                  \
   {                                      \
     if (dm.M <= 4) ARMT_MEMWV_CASE(C, 4) \
@@ -452,6 +522,8 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
 cudaError_t setup_memory_kernels(const Dims& dm) {
   const int sh = (int)memw_update_smem(dm);
   cudaError_t e = cudaSuccess;
+  if (memw_phi_smem(dm) > 48 * 1024)
+    e = cudaFuncSetAttribute(memw_phi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)memw_phi_smem(dm));
   if (sh > 48 * 1024) {
     auto set = [&](auto fn) {
       if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, sh);
@@ -460,11 +532,22 @@ cudaError_t setup_memory_kernels(const Dims& dm) {
     set(memw_update_kernel<12, 4>); set(memw_update_kernel<12, 16>); set(memw_update_kernel<12, 32>);
     set(memw_update_kernel<24, 4>); set(memw_update_kernel<24, 16>); set(memw_update_kernel<24, 32>);
     set(memw_update_kernel<32, 4>); set(memw_update_kernel<32, 16>); set(memw_update_kernel<32, 32>);
-    set(memw_update_vec_kernel<2, 4>); set(memw_update_vec_kernel<2, 16>); set(memw_update_vec_kernel<2, 32>);
-    set(memw_update_vec_kernel<3, 4>); set(memw_update_vec_kernel<3, 16>); set(memw_update_vec_kernel<3, 32>);
-    set(memw_update_vec_kernel<4, 4>); set(memw_update_vec_kernel<4, 16>); set(memw_update_vec_kernel<4, 32>);
-    set(memw_update_vec_kernel<6, 4>); set(memw_update_vec_kernel<6, 16>); set(memw_update_vec_kernel<6, 32>);
-    set(memw_update_vec_kernel<8, 4>); set(memw_update_vec_kernel<8, 16>); set(memw_update_vec_kernel<8, 32>);
+    set(memw_update_vec_kernel<2, 4, false>); set(memw_update_vec_kernel<2, 16, false>); set(memw_update_vec_kernel<2, 32, false>);
+    set(memw_update_vec_kernel<3, 4, false>); set(memw_update_vec_kernel<3, 16, false>); set(memw_update_vec_kernel<3, 32, false>);
+    set(memw_update_vec_kernel<4, 4, false>); set(memw_update_vec_kernel<4, 16, false>); set(memw_update_vec_kernel<4, 32, false>);
+    set(memw_update_vec_kernel<6, 4, false>); set(memw_update_vec_kernel<6, 16, false>); set(memw_update_vec_kernel<6, 32, false>);
+    set(memw_update_vec_kernel<8, 4, false>); set(memw_update_vec_kernel<8, 16, false>); set(memw_update_vec_kernel<8, 32, false>);
+  }
+  const size_t sh_pf = memw_update_pf_smem(dm);
+  if (sh_pf <= MEMW_PF_SMEM_MAX && sh_pf > 48 * 1024) {
+    auto set = [&](auto fn) {
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sh_pf);
+    };
+    set(memw_update_vec_kernel<2, 4, true>); set(memw_update_vec_kernel<2, 16, true>); set(memw_update_vec_kernel<2, 32, true>);
+    set(memw_update_vec_kernel<3, 4, true>); set(memw_update_vec_kernel<3, 16, true>); set(memw_update_vec_kernel<3, 32, true>);
+    set(memw_update_vec_kernel<4, 4, true>); set(memw_update_vec_kernel<4, 16, true>); set(memw_update_vec_kernel<4, 32, true>);
+    set(memw_update_vec_kernel<6, 4, true>); set(memw_update_vec_kernel<6, 16, true>); set(memw_update_vec_kernel<6, 32, true>);
+    set(memw_update_vec_kernel<8, 4, true>); set(memw_update_vec_kernel<8, 16, true>); set(memw_update_vec_kernel<8, 32, true>);
   }
   return e;
 }

@@ -70,7 +70,8 @@ extern "C" armt_status armt_memory_write_static(int M, int d, int d_key, int nu,
   Dims dm{};
   dm.L = 1; dm.d = d; dm.M = M; dm.dk = d_key; dm.nu = nu; dm.P = 2 * d_key * nu; dm.mem_eps = eps;
   dm.bf16 = false;
-  if (((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + 17 * dm.M) * 4 > 200 * 1024) return ARMT_ERR_UNSUPPORTED;
+  if (((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + 17 * dm.M) * 4 > 200 * 1024 || memw_phi_smem(dm) > 200 * 1024)
+    return ARMT_ERR_UNSUPPORTED;
   if (scratch_floats(M, d, d_key, dm.P) > STATIC_SCRATCH_FLOATS) return ARMT_ERR_SHAPE;
   float* scratch = nullptr;
   cudaError_t e = scratch_on_current_device(&scratch);

@@ -16,6 +16,11 @@ __device__ __forceinline__ void st(float* p, size_t i, float v) { p[i] = v; }
 __device__ __forceinline__ void st(bf16* p, size_t i, float v) { p[i] = __float2bfloat16_rn(v); }
 __device__ __forceinline__ float ld(const f16* p, size_t i) { return __half2float(p[i]); }
 __device__ __forceinline__ void st(f16* p, size_t i, float v) { p[i] = __float2half_rn(v); }
+// v as stored in an array of T (rounded to T's precision)
+template <typename T> __device__ __forceinline__ float rounded(float v);
+template <> __device__ __forceinline__ float rounded<float>(float v) { return v; }
+template <> __device__ __forceinline__ float rounded<f16>(float v) { return __half2float(__float2half_rn(v)); }
+template <> __device__ __forceinline__ float rounded<bf16>(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
@@ -212,14 +217,15 @@ __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu,
   TP* out = phi + roff * P;
   float dot = 0.f;
   bool over = false;
-  for (int p = lane; p < P; p += 32) {
-    const int n = p / n2 + 1, j = p - (n - 1) * n2;
-    int jj = (j - n) % n2;
-    if (jj < 0) jj += n2;
-    const float f = r[j] * r[jj];
-    over |= f > 65504.f;
-    st(out, p, f);
-    dot = fmaf(ld(out, p), z[p], dot);
+  for (int n = 1; n <= nu; ++n) {      // block n: r_j * r_{(j - n) mod 2dk} (nu <= 2 dk)
+    for (int j = lane; j < n2; j += 32) {
+      const int jj = j - n < 0 ? j - n + n2 : j - n;
+      const int p = (n - 1) * n2 + j;
+      const float f = r[j] * r[jj];
+      over |= f > 65504.f;
+      st(out, p, f);
+      dot = fmaf(rounded<TP>(f), z[p], dot);   // the stored (operand-precision) value
+    }
   }
   dot = warp_sum(dot);
   if (lane == 0) inv_den[roff] = 1.f / (dot + eps);

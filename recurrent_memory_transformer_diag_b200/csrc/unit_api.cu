@@ -65,7 +65,8 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
   Dims dm{};
   dm.L = 1; dm.d = d; dm.M = M; dm.dk = d_key; dm.nu = nu; dm.P = 2 * d_key * nu; dm.mem_eps = eps;
   dm.bf16 = false;
-  if (((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + 17 * dm.M) * 4 > 200 * 1024) return ARMT_ERR_UNSUPPORTED;
+  if (((size_t)dm.M * dm.P + (size_t)dm.M * dm.M + 17 * dm.M) * 4 > 200 * 1024 || memw_phi_smem(dm) > 200 * 1024)
+    return ARMT_ERR_UNSUPPORTED;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = setup_memory_kernels(dm);
   if (e != cudaSuccess) return to_status(e);

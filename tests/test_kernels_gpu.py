@@ -54,9 +54,10 @@ def test_simt_grouped_gemm_fp32_matches_fp64():
 
 
 # P = 2 dk nu: multiples of 4 take the 16-byte update kernel (P = 64, 384, 768;
-# M = 32 the widest lane map), P = 10 and 42 the scalar one
+# M = 32 the widest lane map; M = 5 an odd count before the prefetch ring),
+# P = 10 and 42 the scalar one
 @pytest.mark.parametrize("M,d,dk,nu", [(4, 64, 16, 2), (16, 256, 64, 3), (16, 2048, 64, 3), (16, 3072, 128, 3),
-                                       (32, 128, 16, 2), (3, 64, 5, 1), (16, 96, 7, 3)])
+                                       (32, 128, 16, 2), (3, 64, 5, 1), (16, 96, 7, 3), (5, 64, 8, 2)])
 def test_memory_write_matches_oracle(M, d, dk, nu):
     import torch
     from recurrent_memory_transformer_diag_b200 import memory_write
