@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "../../include/armt.h"
@@ -31,6 +32,38 @@ __host__ __device__ inline long long h_blocked_offset(int row, int col, int d) {
   return ((long long)(row >> 5) * (d >> 2) + (col >> 2)) * 128 + (row & 31) * 4 + (col & 3);
 }
 __host__ __device__ inline int rows_blocked(int Tp) { return (Tp + 31) & ~31; }
+
+// Programmatic dependent launch.  The forward's kernels are launched with
+// programmatic stream serialisation, so a kernel's blocks may be scheduled
+// while its predecessor drains (hiding the launch gap); each such kernel
+// starts with grid_dependency_sync(): it lets its own dependant be scheduled
+// early, then waits until the predecessor grid has completed and its memory
+// is visible, before touching any data.  Launched without the attribute, the
+// wait returns at once.
+__device__ __forceinline__ void grid_dependency_sync() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Whether the forward's kernels use programmatic dependent launch (only when
+// the environment sets ARMT_PDL=1).
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // One node of the (segment, layer) grid as the kernels see it: x = segment s,
 // y = layer l, z = activation slot (s mod number-of-slots), w = flags.

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  grid_dependency_sync();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // an earlier kernel of this forward already gave up on a wait: do nothing
   // (one thread reads the word, so the whole CTA takes the same decision)
@@ -629,8 +630,8 @@ cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, i
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int items = n * dm.KV * p.q_tiles;
-  attention_tc_kernel<<<items < sms ? items : sms, NUM_THREADS, SMEM_TOTAL, st>>>(tm_qk, tm_vt, p);
-  return cudaGetLastError();
+  return launch_pdl(attention_tc_kernel, dim3(items < sms ? items : sms), dim3(NUM_THREADS), SMEM_TOTAL, st, tm_qk,
+                    tm_vt, p);
 }
 
 }  // namespace armt

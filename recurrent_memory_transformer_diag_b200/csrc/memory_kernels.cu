@@ -39,6 +39,7 @@ __device__ __forceinline__ float warp_sum_m(float v) {
 __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, int P, int nu,
                                 const float* kv, float* z_state, float* phik, float* gram, float* coef,
                                 float* gamma, float eps) {
+  grid_dependency_sync();
   extern __shared__ float sh[];
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n2 = 2 * dk;
@@ -123,9 +124,8 @@ cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const
                             float* z_state, float* phik, float* gram, float* coef, float* gamma,
                             cudaStream_t st) {
   const int nw = dm.M < 32 ? dm.M : 32;
-  memw_phi_kernel<<<n, nw * 32, memw_phi_smem(dm), st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, dm.nu, kv, z_state, phik,
-                                                         gram, coef, gamma, dm.mem_eps);
-  return cudaGetLastError();
+  return launch_pdl(memw_phi_kernel, dim3(n), dim3(nw * 32), memw_phi_smem(dm), st, nodes, dm.M, dm.dk, dm.d, dm.P,
+                    dm.nu, kv, z_state, phik, gram, coef, gamma, dm.mem_eps);
 }
 
 constexpr int MEMW_ROWS_PER_BLOCK = 64;
@@ -177,6 +177,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
                                                           const float* kv, const float* phik,
                                                           const float* gram, const float* coef, float* A_state,
                                                           f16* a_act, unsigned* err) {
+  grid_dependency_sync();
   constexpr int R = MEMW_R;
   extern __shared__ float sh[];
   float* ph = sh;                    // [M][P]
@@ -301,12 +302,13 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
                                                                  const float* kv, const float* phik,
                                                                  const float* gram, const float* coef,
                                                                  float* A_state, f16* a_act, unsigned* err) {
+  grid_dependency_sync();
   constexpr int R = MEMW_R;
   extern __shared__ float sh[];
   float* ph = sh;                    // [M][P]
   float* G = ph + M * P;             // [M][M]
   float* cf = G + M * M;             // [M]
-  float* dots = cf + M;              // [8][R][M]  delta_j per warp and row
+  // (the next 8 R M floats are unused here: the layout matches the scalar kernel's)
   float* pf = sh + ((M * P + M * M + M + 8 * R * M + 3) & ~3);   // PF: [8 warps][2][R][P] rows of A in flight (16-byte aligned)
   const NodeEntry nd = nodes[blockIdx.y];
   const int slot = nd.z, layer = nd.y;
@@ -321,7 +323,6 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
   __syncthreads();
   const float4* ph4 = reinterpret_cast<const float4*>(ph);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* dl = dots + warp * R * M;
   bool over = false;
   constexpr int SHIFT = 5 - log2_const<MT>();
   const float cj = lane < M ? cf[lane] : 0.f;
@@ -402,17 +403,25 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
       const float tot = transpose_reduce<MT>(part[r], lane);
       sv[r] = __shfl_sync(0xffffffffu, tot, (lane << SHIFT) & 31);
     }
-    for (int j = 0; j < M; ++j) {
-      // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
-      const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
+    // every lane receives each delta_j as it is broadcast, so the deltas stay
+    // in registers for the update (no shared-memory round trip)
+    float dreg[R][MT];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
-        if (lane == j) dl[r * M + j] = dj;
-        sv[r] = fmaf(dj, gj, sv[r]);
+    for (int j = 0; j < MT; ++j) {
+      if (j < M) {
+        // delta_j = v_j[i] - s_j coef_j; s_j is final once rows 0..j-1 are applied
+        const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
+          dreg[r][j] = dj;
+          sv[r] = fmaf(dj, gj, sv[r]);
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < R; ++r) dreg[r][j] = 0.f;
       }
     }
-    __syncwarp();
 #pragma unroll
     for (int c = 0; c < C4; ++c) {
       const int q = lane + 32 * c;
@@ -420,15 +429,18 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
         float4 acc[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) acc[r] = a[r][c];
-        for (int j = 0; j < M; ++j) {
-          const float4 f = ph4[j * P4 + q];
 #pragma unroll
-          for (int r = 0; r < R; ++r) {
-            const float dj = dl[r * M + j];
-            acc[r].x = fmaf(dj, f.x, acc[r].x);
-            acc[r].y = fmaf(dj, f.y, acc[r].y);
-            acc[r].z = fmaf(dj, f.z, acc[r].z);
-            acc[r].w = fmaf(dj, f.w, acc[r].w);
+        for (int j = 0; j < MT; ++j) {
+          if (j < M) {
+            const float4 f = ph4[j * P4 + q];
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              const float dj = dreg[r][j];
+              acc[r].x = fmaf(dj, f.x, acc[r].x);
+              acc[r].y = fmaf(dj, f.y, acc[r].y);
+              acc[r].z = fmaf(dj, f.z, acc[r].z);
+              acc[r].w = fmaf(dj, f.w, acc[r].w);
+            }
           }
         }
 #pragma unroll
@@ -485,14 +497,15 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     const int c4 = (dm.P / 4 + 31) / 32;
     const size_t sh_pf = memw_update_pf_smem(dm);
     const bool pf = sh_pf <= MEMW_PF_SMEM_MAX;
+    cudaError_t e = cudaSuccess;
 #define ARMT_MEMWV_CASE(C, MT)                                                                                      \
   {                                                                                                                 \
     if (pf)                                                                                                         \
-      memw_update_vec_kernel<C, MT, true><<<grid, 256, sh_pf, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, \
-                                                                    coef, A_state, (f16*)a_act, err);               \
+      e = launch_pdl(memw_update_vec_kernel<C, MT, true>, grid, dim3(256), sh_pf, st, nodes, dm.M, dm.dk, dm.d,   \
+                     dm.P, kv, phik, gram, coef, A_state, (f16*)a_act, err);                                        \
     else                                                                                                            \
-      memw_update_vec_kernel<C, MT, false><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram,   \
-                                                                  coef, A_state, (f16*)a_act, err);                 \
+      e = launch_pdl(memw_update_vec_kernel<C, MT, false>, grid, dim3(256), sh, st, nodes, dm.M, dm.dk, dm.d, dm.P, \
+                     kv, phik, gram, coef, A_state, (f16*)a_act, err);                                              \
   }
 #define ARMT_MEMWV_M(C)                  \
   {                                      \
@@ -507,7 +520,7 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     else ARMT_MEMWV_M(8)
 #undef ARMT_MEMWV_M
 #undef ARMT_MEMWV_CASE
-    return cudaGetLastError();
+    return e;
   }
   if (chunks <= 4) ARMT_MEMW_M(4)
   else if (chunks <= 12) ARMT_MEMW_M(12)

@@ -121,6 +121,7 @@ __global__ void init_first_layer_kernel(const NodeEntry* nodes, int T, int Tp, i
 // tile's 32 x 64 values form one contiguous run of 2048 floats.
 __global__ void init_first_layer_blocked_kernel(const NodeEntry* nodes, int T, int Tp, int d, const bf16* emb,
                                                 const float* mem_emb, float* h, f16* xb) {
+  grid_dependency_sync();
   __shared__ float tile[32][65];
   const NodeEntry nd = nodes[blockIdx.z];
   if (nd.y != 0) return;
@@ -149,7 +150,8 @@ cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int 
   if (dm.bf16) {
     if (!xb || dm.d % 4) return cudaErrorInvalidValue;
     dim3 grid(rows_blocked(Tp) / 32, (dm.d + 63) / 64, n);
-    init_first_layer_blocked_kernel<<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const bf16*)emb, mem_emb, h, xb);
+    return launch_pdl(init_first_layer_blocked_kernel, grid, dim3(256), 0, st, nodes, T, Tp, dm.d, (const bf16*)emb,
+                      mem_emb, h, xb);
   } else {
     dim3 grid(Tp, n);
     init_first_layer_kernel<float><<<grid, 256, 0, st>>>(nodes, T, Tp, dm.d, (const float*)emb, mem_emb, h);
@@ -198,6 +200,7 @@ template <typename TP>
 __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu, int P,
                                  const float* qm, const float* z_state, TP* phi, float* inv_den,
                                  float eps, unsigned* err) {
+  grid_dependency_sync();
   extern __shared__ float r_sh[];   // [8 warps][2 dk]
   const NodeEntry nd = nodes[blockIdx.y];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -237,8 +240,8 @@ cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int 
   dim3 grid((Tp + 7) / 8, n);
   const size_t sh = 8 * 2 * dm.dk * sizeof(float);
   if (dm.bf16)
-    dpfp_read_kernel<f16><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
-                                                 (f16*)phi, inv_den, dm.mem_eps, err);
+    return launch_pdl(dpfp_read_kernel<f16>, grid, dim3(256), sh, st, nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
+                      (f16*)phi, inv_den, dm.mem_eps, err);
   else
     dpfp_read_kernel<float><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
                                                    (float*)phi, inv_den, dm.mem_eps, nullptr);

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
+  grid_dependency_sync();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // an earlier kernel of this forward already gave up on a wait: do nothing
   // (the forward's result is reported as failed), so a systematic failure
@@ -669,8 +670,7 @@ cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const Tc
   using SM = Smem<BN>;
   const int total = p.n_nodes * p.m_tiles * p.n_tiles;
   const int grid = total < sm_count ? total : sm_count;
-  tc_gemm_kernel<BN, EPI><<<grid, NUM_THREADS, SM::TOTAL, st>>>(ta, tb, p);
-  return cudaGetLastError();
+  return launch_pdl(tc_gemm_kernel<BN, EPI>, dim3(grid), dim3(NUM_THREADS), SM::TOTAL, st, ta, tb, p);
 }
 
 template <int BN, int EPI>
