@@ -145,6 +145,14 @@ __device__ __forceinline__ void resid_add32(float* Hs, int row, int col, int d, 
   }
 }
 
+// The 32 residual values of columns col .. col+31 (col % 4 == 0) of this
+// thread's row in the row-blocked layout: 8 groups of 4, 128 floats apart.
+__device__ __forceinline__ void load_h8(const float* Hs, int row, int col, int d, float4* dst) {
+  const float4* H4 = reinterpret_cast<const float4*>(Hs + h_blocked_offset(row, col, d));
+#pragma unroll
+  for (int q = 0; q < 8; ++q) dst[q] = H4[q * 32];
+}
+
 // Epilogue of one accumulator tile for this thread's row.  Every tcgen05.ld
 // is executed by the whole warp (warp-uniform loops); only the stores are
 // guarded by the row/column bounds.
@@ -161,43 +169,77 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
                                              bool valid, int nb, int half) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
-  if constexpr (EPI == TC_EPI_F32 || EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+  if constexpr (EPI == TC_EPI_F32) {
     float rs = 1.f;
-    if (EPI != TC_EPI_F32 && p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
-    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
-    if (EPI == TC_EPI_F32 && p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
-    float ss = 0.f;
+    if (p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
 #pragma unroll 1
     for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
       tmem_ld32(tbase + c * 32, v);
       const int col = nb * BN + c * 32;
       if (!valid || col >= p.N) continue;
+      float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+      if (p.rsq) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] *= rs;
+      }
+      store_f32x32(C, v, p.N - col);
+    }
+  } else if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+    // h += acc * rs.  The residual of the next 32-column chunk is loaded while
+    // the current one is processed (the epilogue is bound by that load's
+    // latency, not by bandwidth).
+    float rs = 1.f;
+    if (p.rowscale && valid) rs = p.rowscale[(long long)slot * p.rs_slot_stride + row];
+    const bool to_out = EPI == TC_EPI_RESID_ACT && p.out && nd.y == p.out_layer && row < p.seg_len;
+    float* Hs = p.h + (long long)slot * p.h_slot_stride;
+    constexpr int NCH = BN / 64;   // chunks per half tile
+    const int c0 = half * NCH;
+    auto full_chunk = [&](int c) { return valid && nb * BN + (c + 1) * 32 <= p.N; };
+    float4 hn[8];
+    if (full_chunk(c0)) load_h8(Hs, row, nb * BN + c0 * 32, p.ldh, hn);
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCH; ++k) {
+      const int c = c0 + k;
+      float4 hc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) hc[q] = hn[q];
+      if (k + 1 < NCH && full_chunk(c + 1)) load_h8(Hs, row, nb * BN + (c + 1) * 32, p.ldh, hn);
+      float v[32];
+      tmem_ld32(tbase + c * 32, v);
+      const int col = nb * BN + c * 32;
+      if (!valid || col >= p.N) continue;
       const int nv = p.N - col;
-      if (EPI == TC_EPI_F32) {
-        float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-        if (p.rsq) {
+      if (nv >= 32) {
+        float4* H4 = reinterpret_cast<float4*>(Hs + h_blocked_offset(row, col, p.ldh));
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= rs;
+        for (int q = 0; q < 8; ++q) {
+          float4 o = hc[q];
+          o.x = fmaf(v[4 * q], rs, o.x);
+          o.y = fmaf(v[4 * q + 1], rs, o.y);
+          o.z = fmaf(v[4 * q + 2], rs, o.z);
+          o.w = fmaf(v[4 * q + 3], rs, o.w);
+          H4[q * 32] = o;
+          v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
         }
-        store_f32x32(C, v, nv);
       } else {
-        resid_add32(p.h + (long long)slot * p.h_slot_stride, row, col, p.ldh, v, rs, nv);
-        if (p.rsq) {
+        resid_add32(Hs, row, col, p.ldh, v, rs, nv);
+      }
+      if (p.rsq) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
-        }
-        if (EPI == TC_EPI_RESID_ACT) {
-          f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-          store_act32(X, v, nv);
-          if (to_out) {
-            bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
-            store_bf16_32(O, v, nv);
-          }
+        for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
+      }
+      if (EPI == TC_EPI_RESID_ACT) {
+        f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
+        store_act32(X, v, nv);
+        if (to_out) {
+          bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
+          store_bf16_32(O, v, nv);
         }
       }
     }
-    if (EPI != TC_EPI_F32 && p.rsq && valid)
+    if (p.rsq && valid)
       p.rsq[(long long)slot * p.rsq_slot_stride + (long long)(2 * nb + half) * p.rsq_pitch + row] = ss;
   } else if constexpr (EPI == TC_EPI_QKV_ROPE) {
     // heads of head_dim columns; pairs (j, j + hd/2) live in chunks (c1, c1 + hd/64)
@@ -235,9 +277,12 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
             v2[i] *= rs;
           }
         }
-        f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
-        store_act32(C + col1, v1, p.N - col1);
-        if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+        // value heads go only to V^T when it is requested (its reader takes V^T)
+        if (!(p.vt && !rot)) {
+          f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
+          store_act32(C + col1, v1, p.N - col1);
+          if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+        }
         if (p.vt && !rot) {
           // value head: dims pc*32.. and hd/2 + pc*32.. of this row, transposed
           const int vh = head - p.rope_heads;

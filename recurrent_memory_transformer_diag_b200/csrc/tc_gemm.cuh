@@ -27,8 +27,9 @@ struct TcGemmParams {
   float* h; long long h_slot_stride; int ldh;   // residual, row-blocked (h_blocked_offset), ldh = row length
   const float* rowscale; long long rs_slot_stride;
   const float2* rope; int rope_pitch; int rope_heads; int head_dim;   // rope [hd/2][rope_pitch]
-  // QKV epilogue: also write the value heads (heads >= rope_heads) transposed,
-  // vt[slot][head - rope_heads][dim][row] with rows vt_pitch apart (optional)
+  // QKV epilogue: write the value heads (heads >= rope_heads) transposed,
+  // vt[slot][head - rope_heads][dim][row] with rows vt_pitch apart, instead of
+  // into C (optional; without it they go to C like q and k)
   f16* vt; int vt_pitch; int n_vheads;
   int f_out;                // SWIGLU: number of valid output features
   // RMSNorm folded into the GEMMs.  Residual epilogues write, per row and per
