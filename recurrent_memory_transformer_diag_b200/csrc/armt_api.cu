@@ -133,7 +133,9 @@ void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeE
     w.count = (int)tab.size() - first;
     w.any_first_layer = false;
     w.any_last_layer = false;
+    w.first_layer_pos = -1;
     for (int k = first; k < (int)tab.size(); ++k) {
+      if (tab[k].y == 0) w.first_layer_pos = k - first;   // a wave holds at most one layer-0 node
       w.any_first_layer |= tab[k].y == 0;
       w.any_last_layer |= tab[k].y == L - 1;
     }
@@ -221,7 +223,9 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   void* a_read = A;
 
   if (wv.any_first_layer)
-    L("init", [&] { return launch_init_first_layer(dm, nodes, n, T, Tp, emb, w.mem_emb, ws.h, nullptr, st); });
+    L("init", [&] {   // only the wave's layer-0 node
+      return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, nullptr, st);
+    });
 
   // ---- memory read: q = h Wq_mem^T, phi = DPFP(q), h += phi A^T / (z.phi + eps)
   {
@@ -344,7 +348,9 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   };
 
   if (wv.any_first_layer)
-    L("init", [&] { return launch_init_first_layer(dm, nodes, n, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st); });
+    L("init", [&] {   // only the wave's layer-0 node
+      return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st);
+    });
 
   // ---- memory read
   L("tc_qmem", [&] {

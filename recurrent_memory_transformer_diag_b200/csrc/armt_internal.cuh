@@ -74,6 +74,7 @@ struct Wave {
   int first;   // index of the wave's first entry in the device node table
   int count;   // nodes in the wave
   bool any_first_layer;
+  int first_layer_pos;   // index within the wave of the (single) layer-0 node, -1 if none
   bool any_last_layer;
 };
 

@@ -95,14 +95,20 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
+    // z_j . phi_j = z_0 . phi_j + sum_{j'<j} gamma_j' G[j'][j]: lane j (< M <= 32)
+    // carries row j; at step j lane j's value is final, gamma_j is broadcast
+    // and the later lanes add its term
+    float zp = lane < M ? zp0[lane] : 0.f;
     for (int j = 0; j < M; ++j) {
-      float zp = zp0[j];
-      for (int jp = 0; jp < j; ++jp) zp = fmaf(gam[jp], G[jp * M + j], zp);
-      const float gm = fminf(fmaxf(1.f - zp / (G[j * M + j] + eps), 0.f), 1.f);
-      gam[j] = gm;
-      coef[(long long)slot * M + j] = 1.f / (zp + eps);
-      gamma[(long long)slot * M + j] = gm;
+      const float gm_l = fminf(fmaxf(1.f - zp / (G[(lane < M ? lane : 0) * (M + 1)] + eps), 0.f), 1.f);
+      const float gm = __shfl_sync(0xffffffffu, gm_l, j);
+      if (lane == j) {
+        gam[j] = gm;
+        coef[(long long)slot * M + j] = 1.f / (zp + eps);
+        gamma[(long long)slot * M + j] = gm;
+      }
+      if (lane > j && lane < M) zp = fmaf(gm, G[j * M + lane], zp);
     }
   }
   __syncthreads();
