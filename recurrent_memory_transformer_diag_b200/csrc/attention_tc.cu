@@ -81,6 +81,28 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// A packed pair of fp32 (sm_100a's f32x2 FMA: two lanes per instruction) and
+// the three-input max.  (Packed row sums cost more in register pairing than
+// they save.)
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the FMA pipe, for the share of the probabilities that bypasses the
 // MUFU unit: x = j + f with j = round(x) (the 1.5 * 2^23 shift puts j in the
 // low mantissa bits of t) and f in [-1/2, 1/2]; 2^f by a degree-3 polynomial
@@ -488,15 +510,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
         if (diag) {   // causal mask on the tile that holds the diagonal
 #pragma unroll
-          for (int i = 0; i < BKEY; ++i) {
-            float v = __uint_as_float(sr[i]);
-            if (k0 + i > row) v = -INFINITY;
-            sr[i] = __float_as_uint(v);
-            m8[i & 7] = fmaxf(m8[i & 7], v);
+          for (int i = 0; i < BKEY; i += 2) {
+            const float v0 = k0 + i > row ? -INFINITY : __uint_as_float(sr[i]);
+            const float v1 = k0 + i + 1 > row ? -INFINITY : __uint_as_float(sr[i + 1]);
+            sr[i] = __float_as_uint(v0);
+            sr[i + 1] = __float_as_uint(v1);
+            m8[(i >> 1) & 7] = max3f(m8[(i >> 1) & 7], v0, v1);
           }
-        } else {
+        } else {   // two new values per three-input max
 #pragma unroll
-          for (int i = 0; i < BKEY; ++i) m8[i & 7] = fmaxf(m8[i & 7], __uint_as_float(sr[i]));
+          for (int i = 0; i < BKEY; i += 2)
+            m8[(i >> 1) & 7] = max3f(m8[(i >> 1) & 7], __uint_as_float(sr[i]), __uint_as_float(sr[i + 1]));
         }
         const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                                fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
@@ -515,20 +539,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // previous O (the exponentials overlap that product)
         // (pairs i with i % POLY_EVERY == POLY_EVERY - 1 on the FMA pipe, the
         // rest on MUFU); row sum in fp32
+        // (scale and shift of a pair in one f32x2 FMA); row sum in fp32
         uint32_t pk[BKEY / 2];
-        float l2[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t sc2 = f2pack(p.scale_log2, p.scale_log2), nm2 = f2pack(-m_used, -m_used);
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int i = 0; i < BKEY / 2; ++i) {
-          const float x0 = fmaf(__uint_as_float(sr[2 * i]), p.scale_log2, -m_used);
-          const float x1 = fmaf(__uint_as_float(sr[2 * i + 1]), p.scale_log2, -m_used);
+          float x0, x1;
+          f2unpack(fma_f32x2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sc2, nm2), x0, x1);
           const bool poly = POLY_EVERY > 0 && i % (POLY_EVERY > 0 ? POLY_EVERY : 1) == POLY_EVERY - 1;
           const float e0 = poly ? ex2_poly(x0) : ex2_approx(x0);
           const float e1 = poly ? ex2_poly(x1) : ex2_approx(x1);
-          l2[i & 3] += e0 + e1;
+          l4[i & 3] += e0 + e1;
           const __half2 h2 = __floats2half2_rn(e0, e1);
           pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        l += (l2[0] + l2[1]) + (l2[2] + l2[3]);
+        l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
         // the previous step's O must be complete: its MMA read the P buffer,
         // and O is read (head done) or rescaled below
         if (!first) {
