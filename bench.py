@@ -160,13 +160,22 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of x over all ranks (the timed region's duration of the
+    slowest replica); x itself on one rank."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(tokens_per_rank: int, ms_max: float, world: int) -> float:
+    """Whole-job tokens/s of `world` independent replicas, each processing
+    tokens_per_rank tokens, timed by the slowest one (ms_max)."""
+    return world * tokens_per_rank / (ms_max / 1e3)
 
 
 # ---------------------------------------------------------------------------- CPU oracle
@@ -266,14 +275,14 @@ def run_ours(args, cfg, S):
     clk = clocks.stop()
     ms = max_over_ranks(ms, world)
     tokens = S * T
-    value = world * tokens / (ms / 1e3)
+    value = replica_throughput(tokens, ms, world)
     launches_per_step = m.launch_count(S)
 
     extra = {}
     # ---- the library's own sequential schedule on the same kernels
     if not args.no_seq and args.schedule == "diagonal":
         ms_seq = max_over_ranks(timed(max(2, args.steps // 2), "sequential"), world)
-        extra["sequential_tokens_per_s"] = world * tokens / (ms_seq / 1e3)
+        extra["sequential_tokens_per_s"] = replica_throughput(tokens, ms_seq, world)
         extra["sequential_ms_per_step"] = ms_seq
         extra["speedup_vs_sequential"] = ms_seq / ms
         m.set_schedule(args.schedule)
@@ -331,7 +340,7 @@ def run_ours(args, cfg, S):
         e1.record(stream)
         torch.cuda.synchronize()
         ms_e2e = max_over_ranks(e0.elapsed_time(e1) / n_e2e, world)
-        e2e = {"value": world * tokens / (ms_e2e / 1e3), "unit": "tokens/s",
+        e2e = {"value": replica_throughput(tokens, ms_e2e, world), "unit": "tokens/s",
                "h2d_bytes_per_step": tokens * d * esz,
                "d2h_bytes_per_step": tokens * d * esz + L * d * P * 4 + L * P * 4,
                "ms_per_step": ms_e2e}
