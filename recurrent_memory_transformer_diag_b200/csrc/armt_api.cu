@@ -134,8 +134,14 @@ void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeE
     w.any_first_layer = false;
     w.any_last_layer = false;
     w.first_layer_pos = -1;
+    w.first_layer_seg = -1;
+    w.last_layer_seg = -1;
     for (int k = first; k < (int)tab.size(); ++k) {
-      if (tab[k].y == 0) w.first_layer_pos = k - first;   // a wave holds at most one layer-0 node
+      if (tab[k].y == 0) {   // a wave holds at most one layer-0 node
+        w.first_layer_pos = k - first;
+        w.first_layer_seg = tab[k].x;
+      }
+      if (tab[k].y == L - 1) w.last_layer_seg = tab[k].x;   // and at most one last-layer node
       w.any_first_layer |= tab[k].y == 0;
       w.any_last_layer |= tab[k].y == L - 1;
     }
@@ -625,7 +631,11 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
 extern "C" armt_status armt_destroy(armt_ctx* ctx) {
   if (!ctx) return ARMT_OK;
   if (ctx->graph_exec) cudaGraphExecDestroy(ctx->graph_exec);
+  if (ctx->host_graph_exec) cudaGraphExecDestroy(ctx->host_graph_exec);
   if (ctx->capture_stream) cudaStreamDestroy(ctx->capture_stream);
+  if (ctx->copy_in_stream) cudaStreamDestroy(ctx->copy_in_stream);
+  if (ctx->copy_out_stream) cudaStreamDestroy(ctx->copy_out_stream);
+  for (cudaEvent_t ev : ctx->host_events) cudaEventDestroy(ev);
   free_weights(ctx->w);
   free_workspace(ctx->ws);
   dfree(ctx->st_emb); dfree(ctx->st_out); dfree(ctx->st_A); dfree(ctx->st_z);
@@ -741,6 +751,107 @@ extern "C" armt_status armt_forward(armt_ctx* ctx, const void* emb, int S, int s
   return forward_impl(ctx, emb, S, seg_len, out_hidden, out_A, out_z, (cudaStream_t)stream);
 }
 
+namespace {
+
+bool host_page_locked(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+// Host-buffer forward on page-locked buffers as one graph over three streams:
+// the embeddings of segment s are copied in on one stream and the wave that
+// starts segment s (its layer-0 node) waits for that copy only; the hidden
+// rows of segment s are copied out on another stream as soon as the wave
+// holding its last-layer node has run; A and z follow the last wave.  The
+// copies thus overlap the forward instead of bracketing it.
+armt_status forward_host_overlapped(armt_ctx* ctx, const void* emb_host, int S, int T, void* out_host,
+                                    float* A_host, float* z_host, cudaStream_t st) {
+  const Dims& dm = ctx->dm;
+  armt_status s = ensure_table(ctx, S, st);
+  if (s != ARMT_OK) return s;
+  armt_ctx::GraphKey key;
+  key.S = S; key.T = T; key.sched = (int)ctx->cfg.schedule;
+  key.emb = emb_host; key.out = out_host; key.A = A_host; key.z = z_host;
+  const armt_ctx::GraphKey& k0 = ctx->host_key;
+  const bool same = ctx->host_graph_exec && k0.S == key.S && k0.T == key.T && k0.sched == key.sched &&
+                    k0.emb == key.emb && k0.out == key.out && k0.A == key.A && k0.z == key.z;
+  if (!same) {
+    if (ctx->host_graph_exec) {
+      cudaGraphExecDestroy(ctx->host_graph_exec);
+      ctx->host_graph_exec = nullptr;
+    }
+    if (!ctx->copy_in_stream) ARMT_TRY(cudaStreamCreateWithFlags(&ctx->copy_in_stream, cudaStreamNonBlocking), "copy stream");
+    if (!ctx->copy_out_stream) ARMT_TRY(cudaStreamCreateWithFlags(&ctx->copy_out_stream, cudaStreamNonBlocking), "copy stream");
+    const size_t need = 2 * (size_t)S + 3;
+    while (ctx->host_events.size() < need) {
+      cudaEvent_t ev;
+      ARMT_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming), "event");
+      ctx->host_events.push_back(ev);
+    }
+    cudaEvent_t* ev_in = ctx->host_events.data();        // [S]
+    cudaEvent_t* ev_out = ev_in + S;                      // [S]
+    cudaEvent_t ev_fork = ev_out[S], ev_join_in = ev_out[S + 1], ev_join_out = ev_out[S + 2];
+    cudaStream_t s1 = ctx->capture_stream, s2 = ctx->copy_in_stream, s3 = ctx->copy_out_stream;
+    const size_t as = act_size(dm);
+    const size_t seg_bytes = (size_t)T * dm.d * as;
+    ARMT_TRY(cudaStreamBeginCapture(s1, cudaStreamCaptureModeThreadLocal), "begin capture");
+    cudaError_t e = cudaSuccess;
+    const char* where = "host forward capture";
+    auto C = [&](cudaError_t r, const char* w) { if (e == cudaSuccess && r != cudaSuccess) { e = r; where = w; } };
+    C(cudaEventRecord(ev_fork, s1), "fork");
+    C(cudaStreamWaitEvent(s2, ev_fork, 0), "fork");
+    C(cudaStreamWaitEvent(s3, ev_fork, 0), "fork");
+    for (int sg = 0; sg < S && e == cudaSuccess; ++sg) {
+      C(cudaMemcpyAsync((char*)ctx->st_emb + sg * seg_bytes, (const char*)emb_host + sg * seg_bytes, seg_bytes,
+                        cudaMemcpyHostToDevice, s2), "copy emb in");
+      C(cudaEventRecord(ev_in[sg], s2), "copy emb in");
+    }
+    C(cudaMemsetAsync(ctx->st_A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), s1), "zero A");
+    C(cudaMemsetAsync(ctx->st_z, 0, (size_t)dm.L * dm.P * sizeof(float), s1), "zero z");
+    if (dm.bf16) C(cudaMemsetAsync(ctx->ws.a_act, 0, (size_t)dm.L * dm.d * dm.P * as, s1), "zero A copy");
+    Launcher L;
+    for (const Wave& wv : ctx->waves) {
+      if (e != cudaSuccess) break;
+      if (wv.first_layer_seg >= 0) C(cudaStreamWaitEvent(s1, ev_in[wv.first_layer_seg], 0), "wait emb");
+      if (dm.bf16) enqueue_wave_tc(ctx, wv, T, ctx->st_emb, ctx->st_out, ctx->st_A, ctx->st_z, s1, L);
+      else enqueue_wave(ctx, wv, T, ctx->st_emb, ctx->st_out, ctx->st_A, ctx->st_z, s1, L);
+      C(L.err, L.where);
+      if (wv.last_layer_seg >= 0) {
+        const int sg = wv.last_layer_seg;
+        C(cudaEventRecord(ev_out[sg], s1), "segment done");
+        C(cudaStreamWaitEvent(s3, ev_out[sg], 0), "segment done");
+        C(cudaMemcpyAsync((char*)out_host + sg * seg_bytes, (const char*)ctx->st_out + sg * seg_bytes, seg_bytes,
+                          cudaMemcpyDeviceToHost, s3), "copy out");
+      }
+    }
+    C(cudaMemcpyAsync(A_host, ctx->st_A, (size_t)dm.L * dm.d * dm.P * 4, cudaMemcpyDeviceToHost, s1), "copy A");
+    C(cudaMemcpyAsync(z_host, ctx->st_z, (size_t)dm.L * dm.P * 4, cudaMemcpyDeviceToHost, s1), "copy z");
+    C(cudaEventRecord(ev_join_in, s2), "join");
+    C(cudaStreamWaitEvent(s1, ev_join_in, 0), "join");
+    C(cudaEventRecord(ev_join_out, s3), "join");
+    C(cudaStreamWaitEvent(s1, ev_join_out, 0), "join");
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ce = cudaStreamEndCapture(s1, &graph);
+    if (e == cudaSuccess) e = ce;
+    if (e == cudaSuccess) e = cudaGraphInstantiate(&ctx->host_graph_exec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    if (e != cudaSuccess) {
+      ctx->host_graph_exec = nullptr;
+      return cuda_fail(ctx, e, where);
+    }
+    ctx->host_key = key;
+  }
+  ARMT_TRY(cudaGraphLaunch(ctx->host_graph_exec, st), "graph launch");
+  ARMT_TRY(cudaStreamSynchronize(st), "host forward sync");
+  return ARMT_OK;
+}
+
+}  // namespace
+
 extern "C" armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int seg_len,
                                          void* out_hidden_host, float* out_A_host, float* out_z_host,
                                          void* stream) {
@@ -762,6 +873,9 @@ extern "C" armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, in
     }
   }
   const size_t tok = (size_t)S * seg_len;
+  if (ctx->use_graph && host_page_locked(emb_host) && host_page_locked(out_hidden_host) &&
+      host_page_locked(out_A_host) && host_page_locked(out_z_host))
+    return forward_host_overlapped(ctx, emb_host, S, seg_len, out_hidden_host, out_A_host, out_z_host, st);
   ARMT_TRY(cudaMemcpyAsync(ctx->st_emb, emb_host, tok * dm.d * as, cudaMemcpyHostToDevice, st), "copy emb in");
   s = forward_impl(ctx, ctx->st_emb, S, seg_len, ctx->st_out, ctx->st_A, ctx->st_z, st);
   if (s != ARMT_OK) return s;

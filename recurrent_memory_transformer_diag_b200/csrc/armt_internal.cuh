@@ -75,6 +75,8 @@ struct Wave {
   int count;   // nodes in the wave
   bool any_first_layer;
   int first_layer_pos;   // index within the wave of the (single) layer-0 node, -1 if none
+  int first_layer_seg;   // its segment, -1 if none
+  int last_layer_seg;    // segment of the wave's (single) last-layer node, -1 if none
   bool any_last_layer;
 };
 
@@ -151,6 +153,12 @@ struct armt_ctx {
   // host-buffer forward staging
   void* st_emb = nullptr; void* st_out = nullptr; float* st_A = nullptr; float* st_z = nullptr;
   size_t st_tokens = 0;
+  // host-buffer forward with page-locked buffers: one graph whose per-segment
+  // input copies, waves and per-segment output copies run on three streams
+  cudaGraphExec_t host_graph_exec = nullptr;
+  GraphKey host_key;
+  cudaStream_t copy_in_stream = nullptr, copy_out_stream = nullptr;
+  std::vector<cudaEvent_t> host_events;
 };
 
 namespace armt {
