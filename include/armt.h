@@ -147,10 +147,15 @@ armt_status armt_forward(armt_ctx* ctx, const void* emb, int S, int seg_len,
                          void* out_hidden, float* out_A, float* out_z, void* stream);
 
 /* Same forward with HOST buffers (same shapes and types as armt_forward):
- * copies emb to the device, runs the forward and copies the results back,
- * all on `stream`; returns after the stream has finished (synchronous).
- * Pinned host memory gives full PCIe/C2C bandwidth; pageable memory works.
- * The device staging buffers are allocated on the first call and kept.
+ * copies emb to the device, runs the forward and copies the results back;
+ * returns after `stream` has finished (synchronous).  When all four host
+ * buffers are page-locked (and graphs are on), the copies are per segment and
+ * overlap the forward: segment s's embeddings are copied in just before the
+ * wave that starts segment s and its hidden rows copied out right after the
+ * wave that finishes it, on two library-owned copy streams joined into one
+ * graph launched on `stream`; A and z follow the last wave.  Pageable memory
+ * works too (copy in, forward, copy out on `stream`).  The device staging
+ * buffers are allocated on the first call and kept.
  * Errors: as armt_forward, plus OOM. */
 armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int seg_len,
                               void* out_hidden_host, float* out_A_host, float* out_z_host,
