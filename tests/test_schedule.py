@@ -88,3 +88,17 @@ def test_checker_catches_planted_errors():
     assert any("backwards" in e for e in sch.check_schedule(swapped, deps))
     merged = [waves[0] + waves[1]] + waves[2:]
     assert any("inside group" in e for e in sch.check_schedule(merged, deps))
+
+
+@pytest.mark.parametrize("S,L", [(S, L) for S in range(1, 13) for L in range(1, 13)])
+def test_each_wave_starts_and_finishes_at_most_one_segment(S, L):
+    """A wave holds at most one layer-0 node (the segment whose embeddings it
+    first needs) and at most one last-layer node (the segment whose hidden
+    states it completes); segment s starts in wave s and finishes in wave
+    s + L - 1.  The per-segment host copies are ordered by exactly this."""
+    for i, wave in enumerate(sch.diagonal_waves(S, L)):
+        starts = [s for s, l in wave if l == 0]
+        ends = [s for s, l in wave if l == L - 1]
+        assert len(starts) <= 1 and len(ends) <= 1
+        assert starts == ([i] if i < S else [])
+        assert ends == ([i - (L - 1)] if 0 <= i - (L - 1) < S else [])
