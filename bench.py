@@ -73,10 +73,8 @@ def kind_bytes(cfg, n_nodes: int, T: int):
     Tp = T + cfg.n_mem
     d, P, M, dk = cfg.d_model, cfg.phi_dim, cfg.n_mem, cfg.d_key
     per = {
-        "memw_update": d * P * (4 + 4 + 2),          # read A, write A, write its bf16 copy
+        "memw_update": d * P * (4 + 4 + 2),          # read A, write A, write its fp16 copy
         "memw_phi": M * P * 4 + P * 8,
-        "norm_attn": Tp * d * (4 + 2),
-        "norm_mlp": Tp * d * (4 + 2),
         "dpfp_read": Tp * dk * 4 + Tp * P * 2,
         "tc_kvmem": (dk + d) * d * 2 + M * d * 2 + M * (dk + d) * 4,   # weight-read bound (M = 16 rows)
     }
@@ -287,6 +285,15 @@ def run_ours(args, cfg, S):
         extra["speedup_vs_sequential"] = ms_seq / ms
         m.set_schedule(args.schedule)
 
+    # ---- sequence-length sweep at this shape (same context, same kernels): the
+    # diagonal and sequential schedules at S segments each; and the "ideal even
+    # load" throughput, every node run at the per-node cost of a full wave (the
+    # marginal cost of one more segment once S >= L, measured between the two
+    # largest S of the sweep)
+    if world == 1 and not args.no_sweep:
+        extra["sweep"] = seq_len_sweep(args, m, emb, out, A, z, S, T, L, stream)
+        m.set_schedule(args.schedule)
+
     # ---- per-kernel device times (un-graphed forward, CUDA events around each launch)
     prof = m.profile_forward(emb, S, T, out, A, z)
     n_nodes = S * L
@@ -353,6 +360,12 @@ def run_ours(args, cfg, S):
                "sample": f"first segment ({T} tokens + {cfg.n_mem} memory tokens, all {L} layers) of the "
                          f"workload, fp64 numpy oracle, {secs:.1f} s"}
 
+    # ---- segment-length sweep: the same token count split into segments of
+    # 512 and 2048 tokens (a context per length; skill page, "Practical
+    # Guidance", segment length tuning)
+    if world == 1 and not args.no_sweep and extra.get("sweep") is not None:
+        extra["sweep"]["seg_len"] = seg_len_sweep(args, cfg, weights, emb, S * T, T, ms, extra, stream)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -360,7 +373,10 @@ def run_ours(args, cfg, S):
         "config": {"workload": workload_name(cfg, S, args.schedule), "segments": S, "seg_len": T,
                    "batch": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs (emb 512 MB at 1B) and weights exceed the 126 MB L2; no flush needed",
-                   "weights": "random init N(0,0.02) (bf16-rounded), embeddings N(0,1)"},
+                   "weights": "random init N(0,0.02) (bf16-rounded), embeddings N(0,1)",
+                   "precision": ("bf16 weights held exactly in fp16, fp16 MMA operands, fp32 accumulate, "
+                                 "fp32 residual stream and memory state; bf16 embeddings in, bf16 hidden out"
+                                 if cfg.dtype == "bf16" else "fp32 throughout")},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
         "clocks": clk, "kernels": kernels, **extra,
@@ -371,6 +387,76 @@ def run_ours(args, cfg, S):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def _time_forward(m, emb, out, A, z, S, T, schedule, n_steps, n_warm, stream):
+    """Mean ms of n_steps graph-launched forwards of S segments after n_warm warm-ups."""
+    import torch
+    m.set_schedule(schedule)
+    for _ in range(n_warm):
+        m.forward(emb, S, T, out, A, z)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_steps):
+        m.forward(emb, S, T, out, A, z)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    m.device_status()
+    return e0.elapsed_time(e1) / n_steps
+
+
+SWEEP_SEGMENTS = (4, 16, 32, 64, 128)
+
+
+def seq_len_sweep(args, m, emb, out, A, z, S_max, T, L, stream):
+    rows = []
+    for S in [s for s in SWEEP_SEGMENTS if s <= S_max]:
+        md = _time_forward(m, emb, out, A, z, S, T, "diagonal", 3, 2, stream)
+        mq = _time_forward(m, emb, out, A, z, S, T, "sequential", 2, 1, stream)
+        rows.append({"segments": S, "tokens": S * T, "diagonal_tokens_per_s": S * T / (md / 1e3),
+                     "sequential_tokens_per_s": S * T / (mq / 1e3), "diagonal_ms": md, "sequential_ms": mq,
+                     "speedup": mq / md})
+    res = {"rows": rows}
+    big = [r for r in rows if r["segments"] >= L]
+    if len(big) >= 2:
+        a, b = big[-2], big[-1]
+        per_seg = (b["diagonal_ms"] - a["diagonal_ms"]) / (b["segments"] - a["segments"])
+        res["ideal_even_load"] = {
+            "tokens_per_s": T / (per_seg / 1e3), "ms_per_full_wave": per_seg,
+            "how": (f"every node at the per-node cost of a full {L}-node wave: the marginal diagonal time of one "
+                    f"more segment between S={a['segments']} and S={b['segments']} (each adds one full wave)"),
+        }
+        for r in rows:
+            r["frac_of_ideal"] = r["diagonal_tokens_per_s"] / res["ideal_even_load"]["tokens_per_s"]
+    return res
+
+
+def seg_len_sweep(args, cfg, weights, emb, tokens, T0, ms0, extra, stream):
+    import torch
+    from recurrent_memory_transformer_diag_b200 import Armt
+    rows = [{"seg_len": T0, "segments": tokens // T0, "diagonal_tokens_per_s": tokens / (ms0 / 1e3),
+             "sequential_tokens_per_s": extra.get("sequential_tokens_per_s"),
+             "speedup": extra.get("speedup_vs_sequential")}]
+    for Tx in (512, 2048):
+        if Tx == T0 or tokens % Tx:
+            continue
+        Sx = tokens // Tx
+        c2 = cfg.with_(seg_len=Tx, n_segments=Sx)
+        m2 = Armt(c2, max_segments=Sx)
+        try:
+            m2.load_weights(weights)
+            out2 = torch.empty(tokens, cfg.d_model, dtype=emb.dtype, device="cuda")
+            A2 = torch.empty(cfg.n_layers, cfg.d_model, cfg.phi_dim, dtype=torch.float32, device="cuda")
+            z2 = torch.empty(cfg.n_layers, cfg.phi_dim, dtype=torch.float32, device="cuda")
+            md = _time_forward(m2, emb, out2, A2, z2, Sx, Tx, "diagonal", 3, 2, stream)
+            mq = _time_forward(m2, emb, out2, A2, z2, Sx, Tx, "sequential", 2, 1, stream)
+            rows.append({"seg_len": Tx, "segments": Sx, "diagonal_tokens_per_s": tokens / (md / 1e3),
+                         "sequential_tokens_per_s": tokens / (mq / 1e3), "speedup": mq / md})
+            del out2, A2, z2
+        finally:
+            m2.close()
+    return rows
 
 
 def read_traffic(kernel: str):
@@ -403,6 +489,7 @@ def main():
     ap.add_argument("--no-seq", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     args = ap.parse_args()
     from recurrent_memory_transformer_diag_b200.inputs import CONFIGS
     cfg = CONFIGS[args.config]

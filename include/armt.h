@@ -235,11 +235,16 @@ armt_status armt_memory_write(int M, int d, int d_key, int nu, float eps,
  * It allocates nothing: its scratch is a fixed 1 MiB array in the library's
  * device image (held by every device that loads the library, until the
  * process exits), enough for 4 + M*(d_key + d) + M*P + M*M + 2*M floats
- * (P = 2*d_key*nu), e.g. M = 16 rows at d = 3072, d_key = 128, nu = 3.
- * Larger sizes return ARMT_ERR_SHAPE without launching anything.
+ * (P = 2*d_key*nu; each of the five parts after the first rounded up to a
+ * multiple of 4 floats so that it starts on a 16-byte boundary), e.g.
+ * M = 16 rows at d = 3072, d_key = 128, nu = 3.  Larger sizes return
+ * ARMT_ERR_SHAPE without launching anything.
  *
  * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * that device current) and caches it; make that first call before any
+ * stream capture.  The cached address stays valid for the life of the
+ * device's primary context: after cudaDeviceReset on a device, this entry
+ * point must not be called again on that device in the same process.
  * All calls share the one array, so calls whose work overlaps on the GPU
  * (other streams, other host threads) race: order them on one stream.
  * Arguments, layouts and errors otherwise as armt_memory_write. */

@@ -498,7 +498,11 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     else ARMT_MEMW_CASE(C, 32)          \
   }
   if (dm.M > 32) return cudaErrorInvalidValue;
-  const bool aligned = (reinterpret_cast<uintptr_t>(A_state) & 15) == 0 && (reinterpret_cast<uintptr_t>(a_act) & 7) == 0;
+  // the 16-byte kernel reads A rows and the phi rows as float4 and writes the
+  // fp16 copy 8 bytes at a time: every base it offsets must be aligned to that
+  const bool aligned = (reinterpret_cast<uintptr_t>(A_state) & 15) == 0 &&
+                       (reinterpret_cast<uintptr_t>(phik) & 15) == 0 &&
+                       (reinterpret_cast<uintptr_t>(a_act) & 7) == 0;
   if (dm.P % 4 == 0 && dm.P <= 1024 && aligned) {   // 16-byte path
     const int c4 = (dm.P / 4 + 31) / 32;
     const size_t sh_pf = memw_update_pf_smem(dm);

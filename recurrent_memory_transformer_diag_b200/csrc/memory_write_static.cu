@@ -47,10 +47,14 @@ cudaError_t scratch_on_current_device(float** out) {
   return cudaSuccess;
 }
 
+// Every sub-buffer starts on a 16-byte boundary (a multiple of 4 floats):
+// the update kernel reads the DPFP features as float4.
+size_t pad4(size_t n) { return (n + 3) & ~(size_t)3; }
+
 // Floats of scratch one call needs: node entry (4), projected [k | v] rows,
-// DPFP features, Gram matrix, coefficients and gammas.
+// DPFP features, Gram matrix, coefficients and gammas, each padded to 4.
 size_t scratch_floats(int M, int d, int d_key, int P) {
-  return 4 + (size_t)M * (d_key + d) + (size_t)M * P + (size_t)M * M + 2 * (size_t)M;
+  return 4 + pad4((size_t)M * (d_key + d)) + pad4((size_t)M * P) + pad4((size_t)M * M) + pad4(M) + pad4(M);
 }
 
 armt_status to_status(cudaError_t e) {
@@ -81,10 +85,10 @@ extern "C" armt_status armt_memory_write_static(int M, int d, int d_key, int nu,
   cudaStream_t st = (cudaStream_t)stream;
   NodeEntry* node = reinterpret_cast<NodeEntry*>(scratch);   // (segment 0, layer 0, slot 0)
   float* kv = scratch + 4;
-  float* phik = kv + (size_t)M * (d_key + d);
-  float* gram = phik + (size_t)M * dm.P;
-  float* coef = gram + (size_t)M * M;
-  float* gamma = coef + M;
+  float* phik = kv + pad4((size_t)M * (d_key + d));
+  float* gram = phik + pad4((size_t)M * dm.P);
+  float* coef = gram + pad4((size_t)M * M);
+  float* gamma = coef + pad4(M);
   // The array keeps the previous call's contents: the node entry must read as
   // zeros; everything else is fully written below before it is read.
   e = cudaMemsetAsync(node, 0, sizeof(NodeEntry), st);

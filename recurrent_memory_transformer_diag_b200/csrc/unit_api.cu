@@ -70,8 +70,12 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = setup_memory_kernels(dm);
   if (e != cudaSuccess) return to_status(e);
-  const size_t n_w = (size_t)(d_key + d) * d, n_kv = (size_t)M * (d_key + d), n_ph = (size_t)M * dm.P;
-  const size_t bytes = (n_w + n_kv + n_ph + 2 * (size_t)M + (size_t)M * M) * sizeof(float) + sizeof(NodeEntry);
+  // sub-buffers padded to 4 floats: each starts on a 16-byte boundary (the
+  // update kernel reads the DPFP features as float4)
+  auto pad4 = [](size_t n) { return (n + 3) & ~(size_t)3; };
+  const size_t n_w = pad4((size_t)(d_key + d) * d), n_kv = pad4((size_t)M * (d_key + d)),
+               n_ph = pad4((size_t)M * dm.P), n_m = pad4(M);
+  const size_t bytes = (n_w + n_kv + n_ph + 2 * n_m + (size_t)M * M) * sizeof(float) + sizeof(NodeEntry);
   char* scratch = nullptr;
   e = cudaMallocAsync((void**)&scratch, bytes, st);
   if (e != cudaSuccess) return to_status(e);
@@ -80,8 +84,8 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
   float* kv = w_kv + n_w;
   float* phik = kv + n_kv;
   float* coef = phik + n_ph;
-  float* gamma = coef + M;
-  float* gram = gamma + M;
+  float* gamma = coef + n_m;
+  float* gram = gamma + n_m;
   static const NodeEntry one = {0, 0, 0, 0};
   e = cudaMemcpyAsync(node, &one, sizeof(NodeEntry), cudaMemcpyHostToDevice, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(w_kv, wk, (size_t)d_key * d * 4, cudaMemcpyDeviceToDevice, st);

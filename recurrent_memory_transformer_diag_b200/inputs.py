@@ -15,7 +15,8 @@ targets):
 * ``3b``    bf16:  L=28, d=3072, 24x128 / 8 KV,     ffn 8192, M=16, T=2048, S=32
 
 Value distributions: linear weights and memory-token embeddings N(0, 0.02),
-input embeddings N(0, 1), RMSNorm gains 1.  In bf16 workloads every tensor is
+input embeddings N(0, 1), RMSNorm gains 1 (optionally 1 + 0.1 N(0, 1) in
+tests).  In bf16 workloads every tensor is
 rounded (round-to-nearest-even) to a bf16-representable fp32 value here, so
 that the oracle computes on exactly the values the GPU loads.
 
@@ -96,14 +97,6 @@ class ArmtConfig:
             "wv_mem": (L, d, d),
         }
 
-    def linear_flops_per_row(self) -> int:
-        """Multiply-add flops (x2) of every dense projection, per processed row."""
-        d, H, KV, hd, F, dk, P = (self.d_model, self.n_heads, self.n_kv_heads,
-                                  self.head_dim, self.d_ffn, self.d_key, self.phi_dim)
-        per_layer = (H + 2 * KV) * hd * d + d * H * hd + 3 * F * d
-        mem_read = dk * d + P * d
-        return 2 * self.n_layers * (per_layer + mem_read)
-
 
 CONFIGS: Dict[str, ArmtConfig] = {
     "tiny": ArmtConfig("tiny", n_layers=2, d_model=64, n_heads=4, n_kv_heads=4, head_dim=16,
@@ -135,8 +128,13 @@ def _round(t, dtype: str) -> np.ndarray:
     return np.ascontiguousarray(t.numpy())
 
 
-def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02) -> Dict[str, np.ndarray]:
-    """All weights of ``cfg`` as host fp32 arrays, nn.Linear layout [out, in]."""
+def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02,
+                 gain_std: float = 0.0) -> Dict[str, np.ndarray]:
+    """All weights of ``cfg`` as host fp32 arrays, nn.Linear layout [out, in].
+
+    RMSNorm gains are 1 by default; ``gain_std > 0`` draws them as
+    1 + gain_std * N(0, 1) instead (a test input that makes a slip in how the
+    gains reach the projections visible)."""
     import torch
     out = {}
     shapes = cfg.weight_shapes()
@@ -144,6 +142,8 @@ def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02) ->
         shape = shapes[name]
         if name in ("attn_norm", "mlp_norm"):
             t = torch.ones(*shape, dtype=torch.float32)
+            if gain_std > 0:
+                t = t + _randn(shape, seed * 1000 + k, gain_std)
         else:
             t = _randn(shape, seed * 1000 + k, std)
         out[name] = _round(t, cfg.dtype)

@@ -38,3 +38,14 @@ def test_bf16_workloads_are_bf16_representable():
     for a in (make_weights(cfg)["w_up"], make_embeddings(cfg, 1)):
         t = torch.from_numpy(a)
         np.testing.assert_array_equal(t.to(torch.bfloat16).to(torch.float32).numpy(), a)
+
+
+def test_optional_gains_are_drawn_around_one():
+    cfg = CONFIGS["small"]
+    w = make_weights(cfg, gain_std=0.1)
+    for name in ("attn_norm", "mlp_norm"):
+        g = w[name]
+        assert 0.07 < float(g.std()) < 0.13 and abs(float(g.mean()) - 1.0) < 0.02
+    assert not np.array_equal(w["attn_norm"], w["mlp_norm"])
+    base = make_weights(cfg)
+    np.testing.assert_array_equal(w["wq"], base["wq"])     # only the gains change

@@ -22,6 +22,9 @@ def _compare(cfg, got, ref, tol):
     hr, Ar, zr = ref
     assert np.isfinite(h).all() and np.isfinite(A).all() and np.isfinite(z).all()
     errs = {"hidden": rel_l2(h, hr)}
+    T = cfg.seg_len
+    for s in range(h.shape[0] // T):   # per segment: a wrong segment cannot hide under the average
+        errs[f"hidden[seg {s}]"] = rel_l2(h[s * T:(s + 1) * T], hr[s * T:(s + 1) * T])
     for l in range(cfg.n_layers):
         errs[f"A[{l}]"] = rel_l2(A[l], Ar[l])
         errs[f"z[{l}]"] = rel_l2(z[l], zr[l])

@@ -5,7 +5,6 @@ Lemma 3.1 of the Diagonal Batching paper (Pith review of arXiv 2506.05229,
 (node (s, l) <- (s, l-1), (s-1, l)), grouping by s + l gives S + L - 1
 groups, the minimum, because the longest dependency path has S + L - 1 nodes.
 """
-import itertools
 import json
 import os
 
@@ -16,16 +15,32 @@ from oracle import schedule as sch
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-def _longest_path_bruteforce(S, L):
-    """Longest path (in nodes) of the PRMT grid by enumerating monotone lattice
-    paths: every path from (0,0) to (S-1,L-1) taking unit steps."""
+def _longest_path_by_enumeration(deps):
+    """Nodes on the longest path of the dependency DAG, found by walking every
+    path from every node (exhaustive; no use of the grid's structure)."""
+    succ = {n: [] for n in deps}
+    for n, preds in deps.items():
+        for p in preds:
+            succ[p].append(n)
     best = 0
-    n = (S - 1) + (L - 1)
-    for steps in itertools.product((0, 1), repeat=n):
-        if sum(steps) != L - 1:
-            continue
-        best = max(best, n + 1)
-    return best if (S, L) != (1, 1) else 1
+
+    def walk(n, length):
+        nonlocal best
+        best = max(best, length)
+        for m in succ[n]:
+            walk(m, length + 1)
+
+    for n in deps:
+        walk(n, 1)
+    return best
+
+
+def test_path_enumeration_separates_the_two_graphs():
+    """The enumeration is not a restatement of S + L - 1: on the original-RMT
+    graph (every layer of segment s waits for the last layer of s - 1) the
+    longest path is the whole S x L sequence."""
+    assert _longest_path_by_enumeration(sch.prmt_dependencies(3, 4)) == 3 + 4 - 1
+    assert _longest_path_by_enumeration(sch.rmt_dependencies(3, 4)) == 3 * 4
 
 
 @pytest.mark.parametrize("S,L", [(S, L) for S in range(1, 13) for L in range(1, 13)])
@@ -42,8 +57,8 @@ def test_diagonal_waves_valid_and_minimal(S, L):
     levels = sch.earliest_groups(deps)
     assert max(levels.values()) + 1 == len(waves)
     assert all(levels[(s, l)] == s + l for (s, l) in deps)   # earliest feasible group = s + l
-    if S + L <= 14:
-        assert _longest_path_bruteforce(S, L) == S + L - 1
+    if S + L <= 11:
+        assert _longest_path_by_enumeration(deps) == S + L - 1
 
 
 @pytest.mark.parametrize("S,L", [(1, 1), (3, 5), (12, 12)])

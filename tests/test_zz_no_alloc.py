@@ -26,7 +26,11 @@ def _case(M, d, dk, nu, seed):
     return m1, m2, wk, wv, A0, z0
 
 
-@pytest.mark.parametrize("M,d,dk,nu", [(16, 2048, 64, 3), (4, 64, 16, 2), (16, 3072, 128, 3)])
+# The last three shapes make M*(dk+d) (the projected rows that precede the
+# DPFP features in the scratch) not a multiple of 4 floats, so the feature
+# rows start only where the scratch layout pads them to 16 bytes.
+@pytest.mark.parametrize("M,d,dk,nu", [(16, 2048, 64, 3), (4, 64, 16, 2), (16, 3072, 128, 3),
+                                       (1, 64, 2, 1), (3, 65, 2, 2), (5, 130, 8, 2)])
 def test_static_write_matches_allocating_write_on_two_calls(M, d, dk, nu):
     import torch
     from recurrent_memory_transformer_diag_b200 import memory_write, memory_write_static
@@ -50,6 +54,59 @@ def test_static_write_matches_allocating_write_on_two_calls(M, d, dk, nu):
     torch.cuda.synchronize()
     assert rel_l2(A.cpu().numpy(), A_ref.cpu().numpy()) < 1e-5
     assert rel_l2(z.cpu().numpy(), z_ref.cpu().numpy()) < 1e-5
+
+
+def _default_pool_used():
+    """(current, high-water) bytes in use in the device's default memory pool,
+    the pool cudaMallocAsync draws from."""
+    import torch
+    from cuda.bindings import runtime as rt
+    err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
+    assert err == rt.cudaError_t.cudaSuccess
+    out = []
+    for attr in (rt.cudaMemPoolAttr.cudaMemPoolAttrUsedMemCurrent, rt.cudaMemPoolAttr.cudaMemPoolAttrUsedMemHigh):
+        err, v = rt.cudaMemPoolGetAttribute(pool, attr)
+        assert err == rt.cudaError_t.cudaSuccess
+        out.append(int(v))
+    return out
+
+
+def _reset_pool_high_water():
+    import torch
+    from cuda.bindings import driver as dr, runtime as rt
+    err, pool = rt.cudaDeviceGetDefaultMemPool(torch.cuda.current_device())
+    assert err == rt.cudaError_t.cudaSuccess
+    err, = rt.cudaMemPoolSetAttribute(pool, rt.cudaMemPoolAttr.cudaMemPoolAttrUsedMemHigh, dr.cuuint64_t(0))
+    assert err == rt.cudaError_t.cudaSuccess
+
+
+def test_static_write_takes_nothing_from_the_allocators():
+    """Neither the stream-ordered pool nor torch's allocator grows during the
+    no-allocation write, even transiently (the pool's high-water mark is reset
+    first); the allocating write, run the same way, does raise the mark."""
+    import torch
+    from recurrent_memory_transformer_diag_b200 import memory_write, memory_write_static
+    M, d, dk, nu = 16, 2048, 64, 3
+    m1, m2, wk, wv, A0, z0 = _case(M, d, dk, nu, seed=7)
+    dev = lambda x: torch.from_numpy(x).cuda()
+    m1_d, m2_d, wk_d, wv_d, A, z = dev(m1), dev(m2), dev(wk), dev(wv), dev(A0), dev(z0)
+    memory_write_static(m1_d, wk_d, wv_d, A, z, nu, 1e-5)   # first call on the device: set-up
+    torch.cuda.synchronize()
+    torch_before = torch.cuda.memory_allocated()
+    _reset_pool_high_water()
+    used0, _ = _default_pool_used()
+    memory_write_static(m2_d, wk_d, wv_d, A, z, nu, 1e-5)
+    memory_write_static(m1_d, wk_d, wv_d, A, z, nu, 1e-5)
+    torch.cuda.synchronize()
+    used1, high1 = _default_pool_used()
+    assert used1 == used0 and high1 <= used0
+    assert torch.cuda.memory_allocated() == torch_before
+    # positive control: the check sees the allocating entry point's scratch
+    _reset_pool_high_water()
+    memory_write(m2_d, wk_d, wv_d, A, z, nu, 1e-5)
+    torch.cuda.synchronize()
+    _, high2 = _default_pool_used()
+    assert high2 > used0
 
 
 def test_static_write_rejects_sizes_beyond_its_scratch():
