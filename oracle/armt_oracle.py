@@ -52,6 +52,14 @@ both cited in the Pith review's reference list):
    random-init model diverge geometrically over the segments (fp64: hidden
    RMS x2 and |A| x10 per segment at the 1B shape), so no finite-precision
    forward over 128 segments could be compared with it.
+   Two variants of the write, both off by default (the ARMT family the
+   Pith review names, ref. 28, and the delta rule, ref. 38, have them; the
+   pages print neither):
+     gated write:      A <- A + beta_j (v_j - vbar_j) phi_j^T with
+                       beta_j = sigmoid(w_beta[l] . m_j), z as above;
+     unclamped gamma:  gamma_j = 1 - (z . phi_j) / (|phi_j|^2 + eps).
+   And the state a forward starts from may be given (A0, z0) instead of 0:
+   a long input streamed over several calls carries the state across them.
 5. DPFP_nu(x): r = [relu(x); relu(-x)] (length 2 d_k);
    phi[(n-1) 2 d_k + j] = r_j * r_{(j-n) mod 2 d_k}, n = 1..nu  (P = 2 d_k nu).
 6. Output: rows 0..T-1 of node (s, L-1) are the final hidden states of
@@ -128,20 +136,29 @@ def mem_read(x: np.ndarray, wq_mem: np.ndarray, A: np.ndarray, z: np.ndarray,
     return (phi @ A.T) / (phi @ z + eps)[:, None]
 
 
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
 def mem_write(m: np.ndarray, wk_mem: np.ndarray, wv_mem: np.ndarray, A: np.ndarray,
-              z: np.ndarray, nu: int, eps: float) -> Tuple[np.ndarray, np.ndarray]:
+              z: np.ndarray, nu: int, eps: float, w_beta: Optional[np.ndarray] = None,
+              clamp_gamma: bool = True) -> Tuple[np.ndarray, np.ndarray]:
     """Delta-rule update of (A, z) from memory rows m [M, d], row after row;
-    returns the new (A, z)."""
+    returns the new (A, z).  ``w_beta`` [d] gates each row's write of A by
+    sigmoid(w_beta . m_j); ``clamp_gamma=False`` leaves gamma unclamped."""
     k = m @ wk_mem.T                              # [M, dk]
     v = m @ wv_mem.T                              # [M, d]
     phi = dpfp(k, nu)                             # [M, P]
+    beta = sigmoid(m @ w_beta) if w_beta is not None else np.ones(m.shape[0])
     A = A.copy()
     z = z.copy()
     for j in range(m.shape[0]):
         zphi = phi[j] @ z
         vbar = (A @ phi[j]) / (zphi + eps)
-        gamma = min(max(1.0 - zphi / (phi[j] @ phi[j] + eps), 0.0), 1.0)
-        A += np.outer(v[j] - vbar, phi[j])
+        gamma = 1.0 - zphi / (phi[j] @ phi[j] + eps)
+        if clamp_gamma:
+            gamma = min(max(gamma, 0.0), 1.0)
+        A += beta[j] * np.outer(v[j] - vbar, phi[j])
         z += gamma * phi[j]
     return A, z
 
@@ -174,7 +191,9 @@ def node_forward(x: np.ndarray, w: Dict[str, np.ndarray], l: int, A: np.ndarray,
     x = decoder_layer(x, w, l, cfg)
     if memory:
         m = rms_norm(x[cfg.seg_len:], np.ones(x.shape[1]), cfg.rms_eps)
-        A, z = mem_write(m, w["wk_mem"][l], w["wv_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps)
+        w_beta = w["w_beta"][l] if getattr(cfg, "write_gate", False) else None
+        A, z = mem_write(m, w["wk_mem"][l], w["wv_mem"][l], A, z, cfg.dpfp_nu, cfg.mem_eps,
+                         w_beta=w_beta, clamp_gamma=getattr(cfg, "gamma_clamp", True))
     return x, A, z
 
 
@@ -183,9 +202,12 @@ def node_forward(x: np.ndarray, w: Dict[str, np.ndarray], l: int, A: np.ndarray,
 # ---------------------------------------------------------------------------
 
 def forward(cfg, weights: Dict[str, np.ndarray], emb: np.ndarray,
-            order: Optional[Iterable[Tuple[int, int]]] = None, memory: bool = True):
+            order: Optional[Iterable[Tuple[int, int]]] = None, memory: bool = True,
+            A0: Optional[np.ndarray] = None, z0: Optional[np.ndarray] = None):
     """Run every node of S = len(emb) / T segments in ``order`` (default:
-    segment-major).  Each node must come after its two predecessors.
+    segment-major).  Each node must come after its two predecessors.  The
+    memory state starts from (A0, z0) when given (the state a previous call
+    left), else from 0.
 
     Returns (hidden [S*T, d], A [L, d, P], z [L, P]) in fp64.
     """
@@ -196,8 +218,9 @@ def forward(cfg, weights: Dict[str, np.ndarray], emb: np.ndarray,
     w = {k: np.asarray(v, dtype=F64) for k, v in weights.items()}
     if order is None:
         order = [(s, l) for s in range(S) for l in range(L)]
-    A = np.zeros((L, d, P), dtype=F64)
-    z = np.zeros((L, P), dtype=F64)
+    A = np.zeros((L, d, P), dtype=F64) if A0 is None else np.array(A0, dtype=F64)
+    z = np.zeros((L, P), dtype=F64) if z0 is None else np.array(z0, dtype=F64)
+    assert A.shape == (L, d, P) and z.shape == (L, P)
     hidden = np.zeros((S * T, d), dtype=F64)
     cur: Dict[int, np.ndarray] = {}     # output of the latest layer run, per segment
     done_layer = np.full(S, -1)         # latest layer run, per segment

@@ -88,8 +88,11 @@ def _layer(x, W, l, cfg):
     return [[x[t][i] + dn[t][i] for i in range(len(x[t]))] for t in range(T)]
 
 
-def forward(cfg, weights, emb, memory=True):
-    """Segment-major recurrence; returns (hidden [S*T][d], A [L][d][P], z [L][P])."""
+def forward(cfg, weights, emb, memory=True, A0=None, z0=None):
+    """Segment-major recurrence; returns (hidden [S*T][d], A [L][d][P], z [L][P]).
+    The write variants follow cfg.write_gate (row j's change of A times
+    1 / (1 + exp(-w_beta . m_j))) and cfg.gamma_clamp; (A0, z0) is the state
+    to start from (zeros when not given)."""
     W = {}
     for name, arr in weights.items():
         if arr.ndim == 1:
@@ -104,6 +107,11 @@ def forward(cfg, weights, emb, memory=True):
     S = len(emb) // T
     A = [[[0.0] * P for _ in range(d)] for _ in range(L)]
     z = [[0.0] * P for _ in range(L)]
+    if A0 is not None:
+        A = [[[float(A0[l][i][p]) for p in range(P)] for i in range(d)] for l in range(L)]
+        z = [[float(z0[l][p]) for p in range(P)] for l in range(L)]
+    gate = getattr(cfg, "write_gate", False)
+    clamp = getattr(cfg, "gamma_clamp", True)
     hidden = []
     for s in range(S):
         x = _mat(emb[s * T:(s + 1) * T]) + [list(r) for r in W["mem_emb"]]
@@ -124,11 +132,16 @@ def forward(cfg, weights, emb, memory=True):
                     phi = _dpfp(kk[j], cfg.dpfp_nu)
                     zphi = sum(z[l][p] * phi[p] for p in range(P))
                     nrm = sum(p * p for p in phi)
-                    gamma = min(max(1.0 - zphi / (nrm + eps), 0.0), 1.0)
+                    gamma = 1.0 - zphi / (nrm + eps)
+                    if clamp:
+                        gamma = min(max(gamma, 0.0), 1.0)
+                    beta = 1.0
+                    if gate:
+                        beta = 1.0 / (1.0 + math.exp(-sum(W["w_beta"][l][i] * mem[j][i] for i in range(d))))
                     for i in range(d):
                         vbar = sum(A[l][i][p] * phi[p] for p in range(P)) / (zphi + eps)
                         for p in range(P):
-                            A[l][i][p] += (vv[j][i] - vbar) * phi[p]
+                            A[l][i][p] += beta * (vv[j][i] - vbar) * phi[p]
                     for p in range(P):
                         z[l][p] += gamma * phi[p]
         hidden.extend(x[:T])

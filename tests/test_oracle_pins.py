@@ -169,6 +169,49 @@ def test_orthogonal_keys_retrieved_independently():
         np.testing.assert_allclose(r[j], (wv @ k[j]) * n2 / (n2 + eps), rtol=1e-12)
 
 
+def test_gated_write_with_zero_gate_vector_halves_the_write_of_A():
+    """w_beta = 0 gives beta = 1/2 for every row: into A = 0, z = 0 one row
+    writes A = v phi^T / 2, while z (gamma = 1) is not gated: z = phi."""
+    dk, nu, eps = 3, 2, 1e-5
+    k = np.array([[0.7, -0.4, 1.1]])
+    P = 2 * dk * nu
+    A, z = oracle.mem_write(k, np.eye(dk), np.eye(dk), np.zeros((dk, P)), np.zeros(P), nu, eps,
+                            w_beta=np.zeros(dk))
+    phi = oracle.dpfp(k[0], nu)
+    np.testing.assert_allclose(A, 0.5 * np.outer(k[0], phi), rtol=0, atol=1e-15)
+    np.testing.assert_allclose(z, phi, rtol=0, atol=1e-15)
+
+
+def test_gated_write_saturates_to_the_plain_write():
+    """A gate vector that makes w_beta . m very large gives beta = 1 (the
+    plain write); very negative gives beta = 0 (A unchanged, z still written)."""
+    dk, nu, eps = 2, 2, 1e-5
+    k = np.array([[0.3, -0.9]])
+    P = 2 * dk * nu
+    A0 = 0.1 * np.arange(dk * P, dtype=float).reshape(dk, P)
+    z0 = np.abs(np.sin(np.arange(P, dtype=float)))
+    plain = oracle.mem_write(k, np.eye(dk), np.eye(dk), A0, z0, nu, eps)
+    hi = oracle.mem_write(k, np.eye(dk), np.eye(dk), A0, z0, nu, eps, w_beta=np.array([1e3, -1e3]))
+    lo = oracle.mem_write(k, np.eye(dk), np.eye(dk), A0, z0, nu, eps, w_beta=np.array([-1e3, 1e3]))
+    np.testing.assert_allclose(hi[0], plain[0], rtol=1e-14)
+    np.testing.assert_array_equal(lo[0], A0)
+    np.testing.assert_allclose(lo[1], plain[1], rtol=1e-14)
+
+
+def test_unclamped_gamma_goes_negative():
+    """With z = 2 phi(k), gamma = 1 - 2|phi|^2/(|phi|^2+eps) ~ -1: unclamped,
+    z moves back to ~phi (clamped it stays, test_gamma_clamped_at_zero)."""
+    dk, nu, eps = 2, 2, 1e-5
+    k = np.array([[0.3, -0.9]])
+    P = 2 * dk * nu
+    phi = oracle.dpfp(k[0], nu)
+    z0 = 2 * phi
+    n2 = phi @ phi
+    _, z = oracle.mem_write(k, np.eye(dk), np.eye(dk), np.zeros((dk, P)), z0, nu, eps, clamp_gamma=False)
+    np.testing.assert_allclose(z, z0 + (1.0 - 2 * n2 / (n2 + eps)) * phi, rtol=1e-13)
+    np.testing.assert_allclose(z, phi, rtol=4 * eps / n2)     # z0 - phi up to the eps terms
+
+
 def test_read_of_empty_state_is_zero():
     x = RNG.standard_normal((5, 8))
     r = oracle.mem_read(x, RNG.standard_normal((2, 8)), np.zeros((8, 8)), np.zeros(8), 2, 1e-5)
@@ -275,6 +318,53 @@ def test_oracle_matches_bruteforce_gqa_and_odd_shapes():
     np.testing.assert_allclose(h, np.array(hn), rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(A, np.array(An), rtol=1e-11, atol=1e-13)
     np.testing.assert_allclose(z, np.array(zn), rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("gate,clamp", [(True, True), (False, False), (True, False)])
+def test_oracle_variants_match_pure_python_bruteforce(gate, clamp):
+    cfg = _micro(write_gate=gate, gamma_clamp=clamp, n_segments=4)
+    w = _micro_weights(cfg, seed=5)
+    emb = RNG.standard_normal((cfg.n_segments * cfg.seg_len, cfg.d_model))
+    h, A, z = oracle.forward(cfg, w, emb)
+    hn, An, zn = naive_armt.forward(cfg, w, emb)
+    np.testing.assert_allclose(h, np.array(hn), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(A, np.array(An), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(z, np.array(zn), rtol=1e-11, atol=1e-13)
+    base = oracle.forward(_micro(n_segments=4), w, emb)
+    assert not np.allclose(A, base[1])      # the variant changes the state
+
+
+def test_oracle_initial_state_matches_pure_python_bruteforce():
+    cfg = _micro()
+    w = _micro_weights(cfg, seed=9)
+    P = cfg.phi_dim
+    rng = np.random.default_rng(2)
+    A0 = 0.2 * rng.standard_normal((cfg.n_layers, cfg.d_model, P))
+    z0 = np.abs(rng.standard_normal((cfg.n_layers, P)))
+    emb = RNG.standard_normal((cfg.n_segments * cfg.seg_len, cfg.d_model))
+    h, A, z = oracle.forward(cfg, w, emb, A0=A0, z0=z0)
+    hn, An, zn = naive_armt.forward(cfg, w, emb, A0=A0, z0=z0)
+    np.testing.assert_allclose(h, np.array(hn), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(A, np.array(An), rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(z, np.array(zn), rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("name,split", [("tiny", 1), ("tiny", 3), ("small", 2)])
+def test_streaming_in_two_calls_equals_one_call(name, split):
+    """Resume: S1 segments, then the next S2 segments from the carried state,
+    equal S1 + S2 segments in one call, bit for bit (the same operations in
+    the same order)."""
+    cfg = CONFIGS[name]
+    S = 4 if name == "small" else cfg.n_segments
+    T = cfg.seg_len
+    w = make_weights(cfg)
+    emb = make_embeddings(cfg, S)
+    h, A, z = oracle.forward(cfg, w, emb)
+    h1, A1, z1 = oracle.forward(cfg, w, emb[:split * T])
+    h2, A2, z2 = oracle.forward(cfg, w, emb[split * T:], A0=A1, z0=z1)
+    np.testing.assert_array_equal(np.concatenate([h1, h2]), h)
+    np.testing.assert_array_equal(A2, A)
+    np.testing.assert_array_equal(z2, z)
 
 
 @pytest.mark.parametrize("name", ["tiny", "small"])
@@ -403,7 +493,7 @@ def test_planted_transposed_weight_is_caught(monkeypatch):
 
 
 def test_planted_gamma_sign_is_caught(monkeypatch):
-    def bad_write(m, wk, wv, A, z, nu, eps):
+    def bad_write(m, wk, wv, A, z, nu, eps, **kw):
         k = m @ wk.T
         v = m @ wv.T
         phi = ao.dpfp(k, nu)
@@ -420,7 +510,7 @@ def test_planted_gamma_sign_is_caught(monkeypatch):
 
 
 def test_planted_batched_write_is_caught(monkeypatch):
-    def batched_write(m, wk, wv, A, z, nu, eps):
+    def batched_write(m, wk, wv, A, z, nu, eps, **kw):
         k = m @ wk.T
         v = m @ wv.T
         phi = ao.dpfp(k, nu)
@@ -443,3 +533,27 @@ def test_planted_missing_write_norm_is_caught(monkeypatch):
         return x, A, z
     monkeypatch.setattr(ao, "node_forward", node_no_norm)
     assert _fails(test_oracle_matches_pure_python_bruteforce)
+
+
+def test_planted_gate_on_z_is_caught(monkeypatch):
+    """A gate that also scaled the z update would be a different reading:
+    the brute force (gate on A only) catches it."""
+    orig = ao.mem_write
+
+    def gate_on_z(m, wk, wv, A, z, nu, eps, w_beta=None, clamp_gamma=True):
+        A1, z1 = orig(m, wk, wv, A, z, nu, eps, w_beta=w_beta, clamp_gamma=clamp_gamma)
+        if w_beta is None:
+            return A1, z1
+        return A1, z + ao.sigmoid(m @ w_beta).mean() * (z1 - z)
+    _run_pins(monkeypatch, "mem_write", gate_on_z)
+    assert _fails(lambda: test_oracle_variants_match_pure_python_bruteforce(True, True))
+
+
+def test_planted_ignored_initial_state_is_caught(monkeypatch):
+    orig = ao.forward
+
+    def ignores_state(cfg, weights, emb, order=None, memory=True, A0=None, z0=None):
+        return orig(cfg, weights, emb, order=order, memory=memory)
+    monkeypatch.setattr(ao, "forward", ignores_state)
+    monkeypatch.setattr(oracle, "forward", ignores_state)
+    assert _fails(lambda: test_streaming_in_two_calls_equals_one_call("tiny", 1))
