@@ -366,6 +366,11 @@ def run_ours(args, cfg, S):
     if world == 1 and not args.no_sweep and extra.get("sweep") is not None:
         extra["sweep"]["seg_len"] = seg_len_sweep(args, cfg, weights, emb, S * T, T, ms, extra, stream)
 
+    # ---- the full-attention decoder over the same tokens on the same kernels
+    # (no memory tokens, one segment): the baseline the pages compare with
+    if world == 1 and not args.no_sweep:
+        extra["full_attention"] = full_attention(cfg, weights, emb, S * T, ms, stream)
+
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -457,6 +462,25 @@ def seg_len_sweep(args, cfg, weights, emb, tokens, T0, ms0, extra, stream):
         finally:
             m2.close()
     return rows
+
+
+def full_attention(cfg, weights, emb, tokens, ms_armt, stream):
+    import torch
+    from recurrent_memory_transformer_diag_b200 import Armt
+    c2 = cfg.with_(n_mem=0, seg_len=tokens, n_segments=1)
+    m2 = Armt(c2, max_segments=1)
+    try:
+        m2.load_weights(weights)
+        out2 = torch.empty(tokens, cfg.d_model, dtype=emb.dtype, device="cuda")
+        A2 = torch.empty(cfg.n_layers, cfg.d_model, cfg.phi_dim, dtype=torch.float32, device="cuda")
+        z2 = torch.empty(cfg.n_layers, cfg.phi_dim, dtype=torch.float32, device="cuda")
+        msf = _time_forward(m2, emb, out2, A2, z2, 1, tokens, "diagonal", 3, 2, stream)
+        del out2, A2, z2
+    finally:
+        m2.close()
+    return {"tokens_per_s": tokens / (msf / 1e3), "ms": msf, "armt_diagonal_speedup": msf / ms_armt,
+            "workload": f"LLaMA-{cfg.name}-shaped decoder, full causal attention over {tokens} tokens "
+                        f"(no memory tokens, one segment), same kernels"}
 
 
 def read_traffic(kernel: str):

@@ -53,18 +53,24 @@ typedef enum {
   ARMT_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
   ARMT_ERR_DEVICE_TIMEOUT = 6,  /* a kernel's bounded wait ran out (reported by armt_device_status) */
   ARMT_ERR_UNSUPPORTED = 7,     /* valid but not implemented shape (e.g. head_dim not 16..128 step 16) */
-  ARMT_ERR_NUMERIC_RANGE = 8    /* an fp16 operand copy overflowed (reported by armt_device_status) */
+  ARMT_ERR_NUMERIC_RANGE = 8    /* reserved: no kernel of this version reports it (the memory read
+                                   multiplies the fp32 state at tf32 precision, with fp32 range) */
 } armt_status;
 
 /* ARMT_FP32: fp32 weights and activations, SIMT kernels.
  * ARMT_BF16: weights rounded to bf16 (round to nearest even) on load; the
  *   tensor-core path stores these bf16 values in fp16 (exact for every value
- *   of magnitude >= 2^-17) and keeps the GEMM/attention activations and the
- *   memory-read operands in fp16, which the tcgen05 tensor cores multiply at
- *   the bf16 rate with 3 more mantissa bits; accumulation, residual stream
- *   and memory state are fp32; embeddings in and hidden states out are bf16.
- * ARMT_F16: fp16 operands; accepted by armt_grouped_gemm only. */
-typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1, ARMT_F16 = 2 } armt_dtype;
+ *   of magnitude >= 2^-17), the products of the bf16 QKV / gate / up weights
+ *   with the (bf16) RMSNorm gains folded into them at fp16 precision, and
+ *   keeps the GEMM/attention activations in fp16,
+ *   which the tcgen05 tensor cores multiply at the bf16 rate with 3 more
+ *   mantissa bits; the memory read multiplies the fp32 features and the fp32
+ *   state A at tf32 precision (fp32 range); accumulation, residual stream and
+ *   memory state are fp32; embeddings in and hidden states out are bf16.
+ * ARMT_F16: fp16 operands; accepted by armt_grouped_gemm only.
+ * ARMT_TF32: fp32 operands multiplied at tf32 precision on the tensor cores;
+ *   accepted by armt_grouped_gemm only. */
+typedef enum { ARMT_FP32 = 0, ARMT_BF16 = 1, ARMT_F16 = 2, ARMT_TF32 = 3 } armt_dtype;
 
 typedef enum { ARMT_SCHED_DIAGONAL = 0, ARMT_SCHED_SEQUENTIAL = 1 } armt_schedule;
 
@@ -72,7 +78,13 @@ typedef enum { ARMT_SCHED_DIAGONAL = 0, ARMT_SCHED_SEQUENTIAL = 1 } armt_schedul
  * stacking the weights (Pith review, "Assumptions & free parameters").
  *   dtype: ARMT_FP32 or ARMT_BF16 (see armt_dtype).  The associative
  *          memory state A, z and the residual stream are fp32 in both modes.
- *   max_seg_len, max_segments: size the workspace allocated at create. */
+ *   max_seg_len, max_segments: size the workspace allocated at create.
+ *   write_gate, gamma_unclamped: ARMT write variants (0 = off, the default
+ *          reading; a zero-initialised struct gets it).  write_gate scales
+ *          memory row j's write of A by beta_j = sigmoid(w_beta[l] . m_j)
+ *          (m_j the RMS-normalised memory row; weights.w_beta required);
+ *          gamma_unclamped leaves gamma_j = 1 - z.phi_j / (|phi_j|^2 + eps)
+ *          unclamped (by default it is clamped to [0, 1]). */
 typedef struct {
   int n_layers;     /* L */
   int d_model;      /* d */
@@ -80,7 +92,12 @@ typedef struct {
   int n_kv_heads;   /* KV heads, H % KV == 0 */
   int head_dim;     /* hd, even */
   int d_ffn;        /* F */
-  int n_mem;        /* M memory tokens per segment, 1..32 */
+  int n_mem;        /* M memory tokens per segment, 0..32.  0: no memory tokens
+                       and no associative memory (the read and write are not
+                       run; A and z stay 0): every segment is a plain causal
+                       decoder forward, and S = 1 with seg_len = N is the
+                       full-attention decoder over N tokens on the same
+                       kernels (the baseline the pages compare ARMT with) */
   int d_key;        /* memory key dimension d_k */
   int dpfp_nu;      /* DPFP order nu */
   float rope_theta;
@@ -90,11 +107,15 @@ typedef struct {
   armt_schedule schedule;
   int max_seg_len;
   int max_segments;
+  int write_gate;       /* 0 / 1 */
+  int gamma_unclamped;  /* 0 / 1 */
 } armt_config;
 
 /* Host fp32 weights, row-major, nn.Linear layout [out, in].  The library
  * copies them (rounding to bf16, round-to-nearest-even, in bf16 mode); the
- * caller keeps ownership and may free them after armt_load_weights returns. */
+ * caller keeps ownership and may free them after armt_load_weights returns.
+ * With n_mem = 0 the memory weights (mem_emb, wq_mem, wk_mem, wv_mem,
+ * w_beta) are not read and may be NULL. */
 typedef struct {
   const float* mem_emb;    /* [M, d]        memory-token embeddings */
   const float* attn_norm;  /* [L, d]        RMSNorm gain before attention */
@@ -109,6 +130,7 @@ typedef struct {
   const float* wq_mem;     /* [L, d_k, d]   memory read query */
   const float* wk_mem;     /* [L, d_k, d]   memory write key */
   const float* wv_mem;     /* [L, d, d]     memory write value */
+  const float* w_beta;     /* [L, d]        write-gate vector (read only when cfg.write_gate) */
 } armt_weights;
 
 /* Create a context on the current CUDA device and allocate its workspace for
@@ -146,6 +168,18 @@ armt_status armt_set_graph(armt_ctx* ctx, int enable);
 armt_status armt_forward(armt_ctx* ctx, const void* emb, int S, int seg_len,
                          void* out_hidden, float* out_A, float* out_z, void* stream);
 
+/* armt_forward with the memory state carried in: when carry_state is 1,
+ * A and z (device, [L, d, P] and [L, P] fp32) hold the state to start from,
+ * e.g. the A and z a previous call left after its last segment, and are
+ * updated in place; running S1 segments and then the next S2 segments this
+ * way gives the same hidden states and final state as one call over
+ * S1 + S2 segments (skill page, "Practical Guidance", memory state
+ * management: the per-layer state stays on the GPU between calls).  With
+ * carry_state 0 it is armt_forward (A and z start from 0).
+ * Errors: as armt_forward; INVALID_ARG for carry_state not 0 or 1. */
+armt_status armt_forward_ex(armt_ctx* ctx, const void* emb, int S, int seg_len,
+                            void* out_hidden, float* A, float* z, int carry_state, void* stream);
+
 /* Same forward with HOST buffers (same shapes and types as armt_forward):
  * copies emb to the device, runs the forward and copies the results back;
  * returns after `stream` has finished (synchronous).  When all four host
@@ -162,9 +196,8 @@ armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int se
                               void* stream);
 
 /* Wait for `stream`, then report and clear the device-side error word that
- * kernels set when a bounded wait runs out (ARMT_ERR_DEVICE_TIMEOUT) or an
- * fp16 operand copy overflows (ARMT_ERR_NUMERIC_RANGE); ARMT_OK otherwise
- * (ARMT_ERR_CUDA if the stream itself failed). */
+ * kernels set when a bounded wait runs out (ARMT_ERR_DEVICE_TIMEOUT);
+ * ARMT_OK otherwise (ARMT_ERR_CUDA if the stream itself failed). */
 armt_status armt_device_status(armt_ctx* ctx, void* stream);
 
 /* Kernel launches one armt_forward enqueues for (S, current schedule):
@@ -205,8 +238,9 @@ const char* armt_last_error(armt_ctx* ctx);
 /* Grouped GEMM over G groups: for g < G,
  *   C[g] (m x n, row-major, fp32) = A[g] (m x k, row-major) * B[bidx[g]]^T
  * with B stored [num_b, n, k] row-major (nn.Linear layout), A and B both bf16
- * (ARMT_BF16) or both fp16 (ARMT_F16) on the tcgen05 tensor-core kernel, or
- * fp32 (ARMT_FP32) on the SIMT kernel.
+ * (ARMT_BF16), both fp16 (ARMT_F16) or both fp32 read at tf32 precision
+ * (ARMT_TF32) on the tcgen05 tensor-core kernel, or fp32 (ARMT_FP32) on the
+ * SIMT kernel.
  * A is [G, m, k], C is [G, m, n]; bidx is a HOST array of G indices < num_b.
  * This is the per-wave "grouped layer" product (skill page, "GroupedGEMM
  * Operations"), each group indexing its own layer's weights.
@@ -224,6 +258,17 @@ armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, int k,
 armt_status armt_memory_write(int M, int d, int d_key, int nu, float eps,
                               const float* m, const float* wk, const float* wv,
                               float* A, float* z, void* stream);
+
+/* Test hook for failure detection (no counterpart in the paper): runs the
+ * grouped GEMM kernel on one tile with its TMA producer told to issue no
+ * copies, so the tensor-core issuer's wait for the first pipeline stage can
+ * never complete.  The kernel's bounded wait (about one second) runs out, it
+ * records the timeout in its error word, every warp leaves its wait, the CTA
+ * frees its tensor memory and exits; the context stays usable.  Returns
+ * ARMT_ERR_DEVICE_TIMEOUT when that happened (the expected result),
+ * ARMT_OK if the wait somehow completed, ARMT_ERR_CUDA / ARMT_ERR_OOM
+ * otherwise.  Synchronous on stream; allocates its own small buffers. */
+armt_status armt_test_bounded_wait(void* stream);
 
 /* The same delta-rule memory write as armt_memory_write, for callers that
  * cannot allocate device memory at call time (a host framework that has

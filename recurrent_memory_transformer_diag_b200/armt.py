@@ -19,7 +19,7 @@ from .inputs import ArmtConfig
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libarmt.so")
 
-ARMT_FP32, ARMT_BF16, ARMT_F16 = 0, 1, 2
+ARMT_FP32, ARMT_BF16, ARMT_F16, ARMT_TF32 = 0, 1, 2, 3
 SCHED = {"diagonal": 0, "sequential": 1}
 
 STATUS = {
@@ -34,6 +34,7 @@ EXPORTS = (
     "armt_forward_host", "armt_device_status", "armt_launch_count", "armt_destroy",
     "armt_status_string", "armt_last_error", "armt_grouped_gemm", "armt_memory_write",
     "armt_kernel_kinds", "armt_kernel_kind_name", "armt_profile_forward", "armt_memory_write_static",
+    "armt_forward_ex", "armt_test_bounded_wait",
 )
 
 
@@ -49,11 +50,12 @@ class _Config(ctypes.Structure):
                                             "d_ffn", "n_mem", "d_key", "dpfp_nu")] + \
                [("rope_theta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("mem_eps", ctypes.c_float),
                 ("dtype", ctypes.c_int), ("schedule", ctypes.c_int),
-                ("max_seg_len", ctypes.c_int), ("max_segments", ctypes.c_int)]
+                ("max_seg_len", ctypes.c_int), ("max_segments", ctypes.c_int),
+                ("write_gate", ctypes.c_int), ("gamma_unclamped", ctypes.c_int)]
 
 
 _WEIGHT_FIELDS = ("mem_emb", "attn_norm", "mlp_norm", "wq", "wk", "wv", "wo", "w_gate", "w_up",
-                  "w_down", "wq_mem", "wk_mem", "wv_mem")
+                  "w_down", "wq_mem", "wk_mem", "wv_mem", "w_beta")
 
 
 class _Weights(ctypes.Structure):
@@ -78,6 +80,7 @@ def lib() -> ctypes.CDLL:
     L.armt_set_schedule.argtypes = [vp, c_int]
     L.armt_set_graph.argtypes = [vp, c_int]
     L.armt_forward.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, vp]
+    L.armt_forward_ex.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, c_int, vp]
     L.armt_forward_host.argtypes = [vp, vp, c_int, c_int, vp, vp, vp, vp]
     L.armt_device_status.argtypes = [vp, vp]
     L.armt_launch_count.argtypes = [vp, c_int, ctypes.POINTER(c_int)]
@@ -90,6 +93,7 @@ def lib() -> ctypes.CDLL:
                                     ctypes.POINTER(c_int), vp, vp]
     L.armt_memory_write.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
     L.armt_memory_write_static.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
+    L.armt_test_bounded_wait.argtypes = [vp]
     L.armt_kernel_kinds.argtypes = []
     L.armt_kernel_kind_name.argtypes = [c_int]
     L.armt_kernel_kind_name.restype = ctypes.c_char_p
@@ -133,6 +137,8 @@ def make_c_config(cfg: ArmtConfig, max_segments: Optional[int] = None, max_seg_l
     c.schedule = SCHED[schedule]
     c.max_seg_len = max_seg_len or cfg.seg_len
     c.max_segments = max_segments or cfg.n_segments
+    c.write_gate = int(bool(getattr(cfg, "write_gate", False)))
+    c.gamma_unclamped = int(not getattr(cfg, "gamma_clamp", True))
     return c
 
 
@@ -167,7 +173,7 @@ class Armt:
 
     # -- calls
     def load_weights(self, weights: Dict[str, np.ndarray]):
-        keep = {k: np.ascontiguousarray(weights[k], dtype=np.float32) for k in _WEIGHT_FIELDS}
+        keep = {k: np.ascontiguousarray(weights[k], dtype=np.float32) for k in _WEIGHT_FIELDS if k in weights}
         w = _Weights(**{k: v.ctypes.data for k, v in keep.items()})
         _check(lib().armt_load_weights(self._h, ctypes.byref(w)), "armt_load_weights", self._h)
 
@@ -181,6 +187,14 @@ class Armt:
         """Device buffers (torch tensors): see armt_forward in include/armt.h."""
         _check(lib().armt_forward(self._h, _ptr(emb), n_segments, seg_len, _ptr(out_hidden), _ptr(out_A),
                                   _ptr(out_z), _stream_handle(stream)), "armt_forward", self._h)
+
+    def forward_ex(self, emb, n_segments: int, seg_len: int, out_hidden, A, z, carry_state: bool,
+                   stream=None):
+        """armt_forward_ex: with carry_state, A and z (device) hold the state to
+        start from and are updated in place (streaming a long input across calls)."""
+        _check(lib().armt_forward_ex(self._h, _ptr(emb), n_segments, seg_len, _ptr(out_hidden), _ptr(A),
+                                     _ptr(z), int(bool(carry_state)), _stream_handle(stream)),
+               "armt_forward_ex", self._h)
 
     def forward_host(self, emb, n_segments: int, seg_len: int, out_hidden, out_A, out_z, stream=None):
         """Host buffers (numpy arrays or pinned CPU tensors): see armt_forward_host."""
@@ -208,10 +222,14 @@ class Armt:
         return n.value
 
 
-def grouped_gemm(A, B, bidx, C, stream=None):
-    """C[g] = A[g] @ B[bidx[g]]^T on device tensors; bf16/fp16 -> tcgen05 kernel, fp32 -> SIMT."""
+def grouped_gemm(A, B, bidx, C, stream=None, tf32: bool = False):
+    """C[g] = A[g] @ B[bidx[g]]^T on device tensors; bf16/fp16 -> tcgen05 kernel, fp32 -> SIMT
+    (fp32 with tf32=True -> tcgen05 kind::tf32)."""
     import torch
     dtype = {torch.bfloat16: ARMT_BF16, torch.float16: ARMT_F16}.get(A.dtype, ARMT_FP32)
+    if tf32:
+        assert A.dtype == torch.float32 and B.dtype == torch.float32
+        dtype = ARMT_TF32
     G, m, k = A.shape
     num_b, n, _ = B.shape
     idx = (ctypes.c_int * G)(*[int(i) for i in bidx])

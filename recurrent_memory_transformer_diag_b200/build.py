@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libarmt.so")
 SOURCES = ["armt_api.cu", "unit_api.cu", "simt_kernels.cu", "memory_kernels.cu", "tc_gemm.cu",
-           "attention_mma.cu", "attention_tc.cu", "memory_write_static.cu"]
+           "attention_tc.cu", "memory_write_static.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
          "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]

@@ -81,14 +81,14 @@ void free_weights(Weights& w) {
 void free_workspace(Workspace& ws) {
   dfree(ws.h); dfree(ws.xb); dfree(ws.qm); dfree(ws.phi); dfree(ws.inv_den); dfree(ws.qkv);
   dfree(ws.attn); dfree(ws.gu); dfree(ws.u); dfree(ws.kv); dfree(ws.phik); dfree(ws.coef);
-  dfree(ws.gamma); dfree(ws.a_act); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err); dfree(ws.rsq); dfree(ws.gram); dfree(ws.vt);
+  dfree(ws.gamma); dfree(ws.beta); dfree(ws.rope); dfree(ws.nodes); dfree(ws.err); dfree(ws.rsq); dfree(ws.gram); dfree(ws.vt);
   ws = Workspace();
 }
 
 armt_status validate_config(const armt_config* c, const char** why) {
   if (!c) { *why = "null config"; return ARMT_ERR_INVALID_ARG; }
   if (c->n_layers < 1 || c->d_model < 1 || c->n_heads < 1 || c->n_kv_heads < 1 || c->head_dim < 2 ||
-      c->d_ffn < 1 || c->n_mem < 1 || c->d_key < 1 || c->dpfp_nu < 1 || c->max_seg_len < 1 ||
+      c->d_ffn < 1 || c->n_mem < 0 || c->d_key < 1 || c->dpfp_nu < 1 || c->max_seg_len < 1 ||
       c->max_segments < 1) {
     *why = "every size must be positive"; return ARMT_ERR_INVALID_ARG;
   }
@@ -102,6 +102,9 @@ armt_status validate_config(const armt_config* c, const char** why) {
     *why = "eps must be >= 0 (rms) / > 0 (memory), rope_theta > 0"; return ARMT_ERR_INVALID_ARG;
   }
   if (c->dpfp_nu > 2 * c->d_key) { *why = "dpfp_nu must be <= 2 * d_key"; return ARMT_ERR_INVALID_ARG; }
+  if ((c->write_gate != 0 && c->write_gate != 1) || (c->gamma_unclamped != 0 && c->gamma_unclamped != 1)) {
+    *why = "write_gate and gamma_unclamped must be 0 or 1"; return ARMT_ERR_INVALID_ARG;
+  }
   if (c->head_dim != 16 && c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) {
     *why = "head_dim must be 16, 32, 64 or 128"; return ARMT_ERR_UNSUPPORTED;
   }
@@ -234,7 +237,8 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     });
 
   // ---- memory read: q = h Wq_mem^T, phi = DPFP(q), h += phi A^T / (z.phi + eps)
-  {
+  // (no memory tokens: no associative memory, the layer alone)
+  if (dm.M > 0) {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = Tp; g.N = dm.dk; g.K = dm.d;
     g.A = ws.h; g.a_slot_stride = hs; g.lda = dm.d;
@@ -243,8 +247,8 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     g.epi = EPI_STORE_F32;
     L("gemm_qmem", [&] { return launch_simt_gemm(g, st); });
   }
-  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, ws.err, st); });
-  {
+  if (dm.M > 0) L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
+  if (dm.M > 0) {
     GemmArgs g{};
     g.nodes = nodes; g.n_nodes = n; g.M = Tp; g.N = dm.d; g.K = dm.P;
     g.A = ws.phi; g.a_slot_stride = (long long)Tp * dm.P; g.lda = dm.P;
@@ -301,20 +305,25 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
   }
 
   // ---- memory write from the RMS-normalised M memory rows of the layer output
-  L("norm_mem", [&] { return launch_rmsnorm(dm, nodes, n, Tp, T, dm.M, ws.h, ws.xb, dm.rms_eps, st); });
-  {
+  if (dm.M > 0) L("norm_mem", [&] { return launch_rmsnorm(dm, nodes, n, Tp, T, dm.M, ws.h, ws.xb, dm.rms_eps, st); });
+  if (dm.M > 0) {
+    const int ldkv = kv_ld(dm);
     GemmArgs g{};
-    g.nodes = nodes; g.n_nodes = n; g.M = dm.M; g.N = dm.dk + dm.d; g.K = dm.d;
+    g.nodes = nodes; g.n_nodes = n; g.M = dm.M; g.N = ldkv; g.K = dm.d;
     g.A = (const float*)ws.xb + (long long)T * dm.d; g.a_slot_stride = hs; g.lda = dm.d;
-    g.B = w.w_kvm; g.b_layer_stride = (long long)(dm.dk + dm.d) * dm.d; g.ldb = dm.d;
-    g.C = ws.kv; g.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); g.ldc = dm.dk + dm.d;
+    g.B = w.w_kvm; g.b_layer_stride = (long long)ldkv * dm.d; g.ldb = dm.d;
+    g.C = ws.kv; g.c_slot_stride = (long long)dm.M * ldkv; g.ldc = ldkv;
     g.epi = EPI_STORE_F32;
     L("gemm_kvmem", [&] { return launch_simt_gemm(g, st); });
   }
-  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
-  L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, nullptr, nullptr, st);
-  });
+  if (dm.M > 0) {
+    L("memw_phi", [&] {
+      return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, ws.beta, st);
+    });
+    L("memw_update", [&] {
+      return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, ws.beta, A, st);
+    });
+  }
 
   if (wv.any_last_layer)
     L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
@@ -325,9 +334,9 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
 // bf16-rounded values in fp16 containers and the GEMM activations are fp16
 // (same tensor-core rate as bf16, 3 more mantissa bits: rounding the
 // normalised activations to bf16 alone costs ~1 % relative error over 16
-// layers), as are the memory-read operands phi and the copy of A.  A value
-// past the fp16 range sets ERR_FP16_RANGE in the error word.  Residual
-// stream, accumulation and the memory state are fp32.
+// layers).  The memory read multiplies the fp32 features and the fp32 state
+// A itself at tf32 precision (fp16's mantissa, fp32's range), so no copy of
+// A is kept.  Residual stream, accumulation and the memory state are fp32.
 void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
                      cudaStream_t st, Launcher& L) {
   const Dims& dm = ctx->dm;
@@ -357,25 +366,37 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     L("init", [&] {   // only the wave's layer-0 node
       return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st);
     });
+  // no memory tokens: no associative memory.  The QKV epilogue's RMSNorm row
+  // scale then needs the layer-0 input's sums of squares, which the memory
+  // read's residual epilogue would otherwise have written.
+  if (dm.M == 0 && wv.any_first_layer)
+    L("init", [&] {
+      return launch_row_sumsq(dm, nodes + wv.first_layer_pos, 1, Tp, ws.h, ws.rsq, (long long)Tp * rsq_parts,
+                              rsq_parts, Tp, st);
+    });
 
   // ---- memory read
+  if (dm.M > 0) {
   L("tc_qmem", [&] {
     TcGemmOperands op{ws.xb, Tp, slots, w.w_qm, dm.dk, dm.L};
     TcGemmParams p; base(p, Tp, dm.dk, dm.d);
     p.C = ws.qm; p.c_slot_stride = (long long)Tp * dm.dk; p.ldc = dm.dk;
     return launch_tc_gemm(op, p, TC_EPI_F32, tc_pick_bn(dm.dk), sms, st);
   });
-  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, ws.err, st); });
+  L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
   L("tc_read", [&] {
-    // h += phi A^T / (z.phi + eps); new h -> fp16 operand copy + norm partials
-    TcGemmOperands op{ws.phi, Tp, slots, ws.a_act, dm.d, dm.L};
+    // h += phi A^T / (z.phi + eps) on kind::tf32 (phi and A fp32); new h ->
+    // fp16 operand copy + norm partials
+    TcGemmOperands op{ws.phi, Tp, slots, A, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, dm.P);
+    p.ab_tf32 = 1;
     p.h = ws.h; p.h_slot_stride = hs_blk; p.ldh = dm.d;
     p.rowscale = ws.inv_den; p.rs_slot_stride = Tp;
     p.C = ws.xb; p.c_slot_stride = hs; p.ldc = dm.d;
     norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
+  }
 
   // ---- attention block (RMSNorm folded: row scale applied in the QKV epilogue)
   L("tc_qkv_rope", [&] {
@@ -389,10 +410,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     norm_partials(p);
     return launch_tc_gemm(op, p, TC_EPI_QKV_ROPE, 256, sms, st);
   });
-  L("attention", [&] {
-    return ws.vt ? launch_attention_tc(dm, nodes, n, Tp, slots, ws.qkv, ws.vt, ws.attn, ws.err, st)
-                 : launch_attention_mma(dm, nodes, n, Tp, ws.qkv, ws.attn, st);
-  });
+  L("attention", [&] { return launch_attention_tc(dm, nodes, n, Tp, slots, ws.qkv, ws.vt, ws.attn, ws.err, st); });
   L("tc_o", [&] {
     TcGemmOperands op{ws.attn, Tp, slots, w.w_o, dm.d, dm.L};
     TcGemmParams p; base(p, Tp, dm.d, Hh);
@@ -425,18 +443,22 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   // ---- memory write: [k | v] = RMSNorm(m) [Wk_mem; Wv_mem]^T for the M memory
   // rows (rows T..T'-1 of the fp16 copy of the layer output the down GEMM
   // wrote; the RMS row scale comes from the down GEMM's partial sums)
+  if (dm.M == 0) return;
   L("tc_kvmem", [&] {
-    TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, dm.dk + dm.d, dm.L};
+    const int ldkv = kv_ld(dm);
+    TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, ldkv, dm.L};
     op.a_pitch = Tp;
-    TcGemmParams p; base(p, dm.M, dm.dk + dm.d, dm.d);
-    p.C = ws.kv; p.c_slot_stride = (long long)dm.M * (dm.dk + dm.d); p.ldc = dm.dk + dm.d;
+    TcGemmParams p; base(p, dm.M, ldkv, dm.d);
+    p.C = ws.kv; p.c_slot_stride = (long long)dm.M * ldkv; p.ldc = ldkv;
     norm_partials(p);
     p.rsq_row0 = T;
     return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, st);
   });
-  L("memw_phi", [&] { return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, st); });
+  L("memw_phi", [&] {
+    return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, ws.beta, st);
+  });
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, A, ws.a_act, ws.err, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, ws.beta, A, st);
   });
 
 }
@@ -455,14 +477,13 @@ armt_status ensure_table(armt_ctx* ctx, int S, cudaStream_t st) {
   return ARMT_OK;
 }
 
+// carry_state: A and z already hold the state to start from (else zeroed first)
 armt_status enqueue_forward(armt_ctx* ctx, const void* emb, int S, int T, void* out, float* A, float* z,
-                            cudaStream_t st, Launcher& L) {
+                            cudaStream_t st, Launcher& L, bool carry_state = false) {
   const Dims& dm = ctx->dm;
-  if (!L.dry) {
+  if (!L.dry && !carry_state) {
     ARMT_TRY(cudaMemsetAsync(A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), st), "zero A");
     ARMT_TRY(cudaMemsetAsync(z, 0, (size_t)dm.L * dm.P * sizeof(float), st), "zero z");
-    if (dm.bf16)
-      ARMT_TRY(cudaMemsetAsync(ctx->ws.a_act, 0, (size_t)dm.L * dm.d * dm.P * act_size(dm), st), "zero A copy");
   }
   for (const Wave& wv : ctx->waves) {
     if (dm.bf16) enqueue_wave_tc(ctx, wv, T, emb, out, A, z, st, L);
@@ -484,19 +505,20 @@ armt_status check_forward_args(armt_ctx* ctx, const void* emb, int S, int seg_le
 }
 
 armt_status forward_impl(armt_ctx* ctx, const void* emb, int S, int T, void* out, float* A, float* z,
-                         cudaStream_t st) {
+                         cudaStream_t st, bool carry_state = false) {
   armt_status s = ensure_table(ctx, S, st);
   if (s != ARMT_OK) return s;
   if (!ctx->use_graph) {
     Launcher L;
-    return enqueue_forward(ctx, emb, S, T, out, A, z, st, L);
+    return enqueue_forward(ctx, emb, S, T, out, A, z, st, L, carry_state);
   }
   armt_ctx::GraphKey key;
-  key.S = S; key.T = T; key.sched = (int)ctx->cfg.schedule;
+  key.S = S; key.T = T; key.sched = (int)ctx->cfg.schedule; key.carry = carry_state ? 1 : 0;
   key.emb = emb; key.out = out; key.A = A; key.z = z;
   const armt_ctx::GraphKey& k0 = ctx->graph_key;
   const bool same = ctx->graph_exec && k0.S == key.S && k0.T == key.T && k0.sched == key.sched &&
-                    k0.emb == key.emb && k0.out == key.out && k0.A == key.A && k0.z == key.z;
+                    k0.carry == key.carry && k0.emb == key.emb && k0.out == key.out && k0.A == key.A &&
+                    k0.z == key.z;
   if (!same) {
     if (ctx->graph_exec) {
       cudaGraphExecDestroy(ctx->graph_exec);
@@ -504,7 +526,7 @@ armt_status forward_impl(armt_ctx* ctx, const void* emb, int S, int T, void* out
     }
     ARMT_TRY(cudaStreamBeginCapture(ctx->capture_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
     Launcher L;
-    armt_status es = enqueue_forward(ctx, emb, S, T, out, A, z, ctx->capture_stream, L);
+    armt_status es = enqueue_forward(ctx, emb, S, T, out, A, z, ctx->capture_stream, L, carry_state);
     cudaGraph_t graph = nullptr;
     cudaError_t ce = cudaStreamEndCapture(ctx->capture_stream, &graph);
     if (es != ARMT_OK) {
@@ -540,7 +562,7 @@ extern "C" const char* armt_status_string(armt_status s) {
     case ARMT_ERR_CUDA: return "CUDA error";
     case ARMT_ERR_DEVICE_TIMEOUT: return "device-side bounded wait timed out";
     case ARMT_ERR_UNSUPPORTED: return "unsupported shape";
-    case ARMT_ERR_NUMERIC_RANGE: return "a value exceeded the fp16 range of an operand copy";
+    case ARMT_ERR_NUMERIC_RANGE: return "numeric range (reserved)";
   }
   return "unknown status";
 }
@@ -563,6 +585,8 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   dm.P = 2 * dm.dk * dm.nu; dm.nqkv = (dm.H + 2 * dm.KV) * dm.hd;
   dm.theta = cfg->rope_theta; dm.rms_eps = cfg->rms_eps; dm.mem_eps = cfg->mem_eps;
   dm.bf16 = cfg->dtype == ARMT_BF16;
+  dm.write_gate = cfg->write_gate != 0;
+  dm.clamp_gamma = cfg->gamma_unclamped == 0;
 
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->sm_count, cudaDevAttrMultiProcessorCount, ctx->device);
@@ -582,7 +606,7 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   A(&ws.h, (size_t)ws.slots * rows_blocked(ws.tp_max) * dm.d * 4);   // >= rows * d (row-blocked slots)
   A(&ws.xb, rows * dm.d * as);
   A(&ws.qm, rows * dm.dk * 4);
-  A(&ws.phi, rows * dm.P * as);
+  A(&ws.phi, rows * dm.P * 4);
   A(&ws.inv_den, rows * 4);
   if (dm.bf16) A(&ws.rsq, rows * 2 * ((dm.d + 255) / 256) * 4);
   A(&ws.qkv, rows * dm.nqkv * as);
@@ -591,12 +615,12 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
     A(&ws.vt, (size_t)ws.slots * dm.KV * dm.hd * attention_tc_vt_pitch(ws.tp_max) * 2);
   if (!dm.bf16) A(&ws.gu, rows * 2 * dm.F * as);
   A(&ws.u, rows * dm.F * as);
-  A(&ws.kv, (size_t)ws.slots * dm.M * (dm.dk + dm.d) * 4);
+  A(&ws.kv, (size_t)ws.slots * dm.M * kv_ld(dm) * 4);
   A(&ws.phik, (size_t)ws.slots * dm.M * dm.P * 4);
   A(&ws.coef, (size_t)ws.slots * dm.M * 4);
   A(&ws.gram, (size_t)ws.slots * dm.M * dm.M * 4);
   A(&ws.gamma, (size_t)ws.slots * dm.M * 4);
-  if (dm.bf16) A(&ws.a_act, (size_t)dm.L * dm.d * dm.P * as);
+  A(&ws.beta, (size_t)ws.slots * dm.M * 4);
   A(&ws.rope, (size_t)ws.tp_max * (dm.hd / 2) * sizeof(float2));
   A(&ws.nodes, ntab * sizeof(NodeEntry));
   A(&ws.err, sizeof(unsigned));
@@ -614,7 +638,6 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   }
   if (e == cudaSuccess) e = setup_memory_kernels(dm);
   if (e == cudaSuccess && dm.bf16) e = setup_tc_gemm();
-  if (e == cudaSuccess && dm.bf16) e = setup_attention_mma();
   if (e == cudaSuccess && dm.bf16 && attention_tc_supported(dm)) e = setup_attention_tc();
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&ctx->capture_stream, cudaStreamNonBlocking);
   if (e != cudaSuccess) {
@@ -658,8 +681,10 @@ extern "C" armt_status armt_set_graph(armt_ctx* ctx, int enable) {
 
 extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) {
   if (!ctx) return ARMT_ERR_INVALID_ARG;
-  if (!wt || !wt->mem_emb || !wt->attn_norm || !wt->mlp_norm || !wt->wq || !wt->wk || !wt->wv || !wt->wo ||
-      !wt->w_gate || !wt->w_up || !wt->w_down || !wt->wq_mem || !wt->wk_mem || !wt->wv_mem)
+  const bool mem = ctx->dm.M > 0;   // the memory weights are read only with memory tokens
+  if (!wt || !wt->attn_norm || !wt->mlp_norm || !wt->wq || !wt->wk || !wt->wv || !wt->wo || !wt->w_gate ||
+      !wt->w_up || !wt->w_down ||
+      (mem && (!wt->mem_emb || !wt->wq_mem || !wt->wk_mem || !wt->wv_mem || (ctx->dm.write_gate && !wt->w_beta))))
     return fail(ctx, ARMT_ERR_INVALID_ARG, "null weight pointer");
   const Dims& dm = ctx->dm;
   free_weights(ctx->w);
@@ -674,11 +699,14 @@ extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) 
   const int f_pad = dm.bf16 ? (F + 127) / 128 * 128 : F;
   A(&w.w_gu, (size_t)L * 2 * f_pad * d * as);
   A(&w.w_down, (size_t)L * d * F * as);
-  A(&w.w_qm, (size_t)L * dm.dk * d * as);
-  A(&w.w_kvm, (size_t)L * (dm.dk + d) * d * as);
+  const int ldkv = kv_ld(dm);
+  if (mem) {
+    A(&w.w_qm, (size_t)L * dm.dk * d * as);
+    A(&w.w_kvm, (size_t)L * ldkv * d * as);
+  }
   // staging for one layer's largest block (fp32)
   const size_t blk = std::max({(size_t)dm.nqkv * d, (size_t)d * Hh, 2 * (size_t)f_pad * d, (size_t)d * F,
-                               (size_t)(dm.dk + d) * d});
+                               (size_t)ldkv * d});
   float* stage = nullptr;
   A(&stage, blk * 4);
   if (e != cudaSuccess) {
@@ -688,18 +716,31 @@ extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) 
   }
   std::vector<float> host(blk);
   cudaStream_t st = 0;
-  auto put = [&](void* dst_base, size_t layer_elems, int l, size_t n_elems) {
+  // folded: the block holds products W diag(g) (bf16 mode: of the bf16-rounded
+  // W and g, exact in fp32), stored at fp16 precision; others are bf16 values
+  auto put = [&](void* dst_base, size_t layer_elems, int l, size_t n_elems, bool folded = false) {
     if (e != cudaSuccess) return;
     e = cudaMemcpy(stage, host.data(), n_elems * 4, cudaMemcpyHostToDevice);
     if (e == cudaSuccess)
       e = launch_convert(stage, (char*)dst_base + (size_t)l * layer_elems * as, n_elems,
-                         dm.bf16 ? CONVERT_BF16_AS_F16 : CONVERT_COPY_F32, st);
+                         dm.bf16 ? (folded ? CONVERT_F16 : CONVERT_BF16_AS_F16) : CONVERT_COPY_F32, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   };
-  // rows of W scaled by the RMSNorm gain on the input dimension: (x*g) W^T = x (W diag g)^T
+  // bf16 round to nearest even of an fp32 value (host); identity in fp32 mode
+  auto to_model = [&](float x) {
+    if (!dm.bf16) return x;
+    uint32_t b;
+    memcpy(&b, &x, 4);
+    b = (b + 0x7FFFu + ((b >> 16) & 1u)) & 0xFFFF0000u;
+    memcpy(&x, &b, 4);
+    return x;
+  };
+  // rows of W scaled by the RMSNorm gain on the input dimension: (x*g) W^T = x (W diag g)^T.
+  // bf16 mode: the product of the bf16-rounded W and g (16 significant bits,
+  // exact in fp32) is stored as fp16, 3 bits finer than rounding it to bf16.
   auto scaled_rows = [&](float* dst, const float* src, int rows, const float* gain) {
     for (int r = 0; r < rows; ++r)
-      for (int k = 0; k < d; ++k) dst[(size_t)r * d + k] = src[(size_t)r * d + k] * gain[k];
+      for (int k = 0; k < d; ++k) dst[(size_t)r * d + k] = to_model(src[(size_t)r * d + k]) * to_model(gain[k]);
   };
   for (int l = 0; l < L && e == cudaSuccess; ++l) {
     const float* ga = wt->attn_norm + (size_t)l * d;
@@ -707,7 +748,7 @@ extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) 
     scaled_rows(host.data(), wt->wq + (size_t)l * Hh * d, Hh, ga);
     scaled_rows(host.data() + (size_t)Hh * d, wt->wk + (size_t)l * KVh * d, KVh, ga);
     scaled_rows(host.data() + (size_t)(Hh + KVh) * d, wt->wv + (size_t)l * KVh * d, KVh, ga);
-    put(w.w_qkv, (size_t)dm.nqkv * d, l, (size_t)dm.nqkv * d);
+    put(w.w_qkv, (size_t)dm.nqkv * d, l, (size_t)dm.nqkv * d, true);
     memcpy(host.data(), wt->wo + (size_t)l * d * Hh, (size_t)d * Hh * 4);
     put(w.w_o, (size_t)d * Hh, l, (size_t)d * Hh);
     if (dm.bf16) {
@@ -725,16 +766,22 @@ extern "C" armt_status armt_load_weights(armt_ctx* ctx, const armt_weights* wt) 
       scaled_rows(host.data(), wt->w_gate + (size_t)l * F * d, F, gm);
       scaled_rows(host.data() + (size_t)F * d, wt->w_up + (size_t)l * F * d, F, gm);
     }
-    put(w.w_gu, 2 * (size_t)f_pad * d, l, 2 * (size_t)f_pad * d);
+    put(w.w_gu, 2 * (size_t)f_pad * d, l, 2 * (size_t)f_pad * d, true);
     memcpy(host.data(), wt->w_down + (size_t)l * d * F, (size_t)d * F * 4);
     put(w.w_down, (size_t)d * F, l, (size_t)d * F);
+    if (!mem) continue;
     memcpy(host.data(), wt->wq_mem + (size_t)l * dm.dk * d, (size_t)dm.dk * d * 4);
     put(w.w_qm, (size_t)dm.dk * d, l, (size_t)dm.dk * d);
+    // [Wk_mem; Wv_mem; w_beta; zero rows] (the gate row and its padding only for the gated write)
     memcpy(host.data(), wt->wk_mem + (size_t)l * dm.dk * d, (size_t)dm.dk * d * 4);
     memcpy(host.data() + (size_t)dm.dk * d, wt->wv_mem + (size_t)l * d * d, (size_t)d * d * 4);
-    put(w.w_kvm, (size_t)(dm.dk + d) * d, l, (size_t)(dm.dk + d) * d);
+    if (dm.write_gate) {
+      std::fill(host.begin() + (size_t)(dm.dk + d) * d, host.begin() + (size_t)ldkv * d, 0.f);
+      memcpy(host.data() + (size_t)(dm.dk + d) * d, wt->w_beta + (size_t)l * d, (size_t)d * 4);
+    }
+    put(w.w_kvm, (size_t)ldkv * d, l, (size_t)ldkv * d);
   }
-  if (e == cudaSuccess) e = cudaMemcpy(w.mem_emb, wt->mem_emb, (size_t)dm.M * d * 4, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess && mem) e = cudaMemcpy(w.mem_emb, wt->mem_emb, (size_t)dm.M * d * 4, cudaMemcpyHostToDevice);
   dfree(stage);
   if (e != cudaSuccess) {
     free_weights(ctx->w);
@@ -749,6 +796,14 @@ extern "C" armt_status armt_forward(armt_ctx* ctx, const void* emb, int S, int s
   armt_status s = check_forward_args(ctx, emb, S, seg_len, out_hidden, out_A, out_z);
   if (s != ARMT_OK) return s;
   return forward_impl(ctx, emb, S, seg_len, out_hidden, out_A, out_z, (cudaStream_t)stream);
+}
+
+extern "C" armt_status armt_forward_ex(armt_ctx* ctx, const void* emb, int S, int seg_len, void* out_hidden,
+                                       float* A, float* z, int carry_state, void* stream) {
+  armt_status s = check_forward_args(ctx, emb, S, seg_len, out_hidden, A, z);
+  if (s != ARMT_OK) return s;
+  if (carry_state != 0 && carry_state != 1) return fail(ctx, ARMT_ERR_INVALID_ARG, "carry_state must be 0 or 1");
+  return forward_impl(ctx, emb, S, seg_len, out_hidden, A, z, (cudaStream_t)stream, carry_state == 1);
 }
 
 namespace {
@@ -812,7 +867,6 @@ armt_status forward_host_overlapped(armt_ctx* ctx, const void* emb_host, int S, 
     }
     C(cudaMemsetAsync(ctx->st_A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), s1), "zero A");
     C(cudaMemsetAsync(ctx->st_z, 0, (size_t)dm.L * dm.P * sizeof(float), s1), "zero z");
-    if (dm.bf16) C(cudaMemsetAsync(ctx->ws.a_act, 0, (size_t)dm.L * dm.d * dm.P * as, s1), "zero A copy");
     Launcher L;
     for (const Wave& wv : ctx->waves) {
       if (e != cudaSuccess) break;
@@ -893,8 +947,7 @@ extern "C" armt_status armt_device_status(armt_ctx* ctx, void* stream) {
   ARMT_TRY(cudaMemcpy(&flag, ctx->ws.err, sizeof(unsigned), cudaMemcpyDeviceToHost), "read error word");
   if (flag) {
     ARMT_TRY(cudaMemset(ctx->ws.err, 0, sizeof(unsigned)), "clear error word");
-    if (flag & ERR_WAIT_TIMEOUT_MASK) return fail(ctx, ARMT_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait timed out");
-    return fail(ctx, ARMT_ERR_NUMERIC_RANGE, "an fp16 operand copy exceeded the fp16 range");
+    return fail(ctx, ARMT_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait timed out");
   }
   return ARMT_OK;
 }

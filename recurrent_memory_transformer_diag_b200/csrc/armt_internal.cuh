@@ -20,7 +20,6 @@ typedef __half f16;
 
 // Bits of the device error word (Workspace::err).
 constexpr unsigned ERR_WAIT_TIMEOUT_MASK = 0x77u; // bits 0-2 (GEMM), 4-6 (attention): a bounded wait ran out
-constexpr unsigned ERR_FP16_RANGE = 8u;           // an fp16 operand copy exceeded the fp16 range
 
 // Residual stream layout on the tensor-core path ("row-blocked"): rows in
 // blocks of 32, each block stored as [d/4 column groups][32 rows][4 columns].
@@ -89,7 +88,7 @@ struct Workspace {
                             // [slots][rows_blocked(T')][d] (tensor-core path)
   void* xb = nullptr;       // [slots][T'][d] GEMM operand copy of h (fp32, or fp16 on the tensor-core path)
   float* qm = nullptr;      // [slots][T'][dk] memory-read query
-  void* phi = nullptr;      // [slots][T'][P] DPFP features (fp32, or fp16 on the tensor-core path)
+  float* phi = nullptr;     // [slots][T'][P] DPFP features, fp32 (tf32-rounded on the tensor-core path)
   float* inv_den = nullptr; // [slots][T'] 1 / (z . phi + eps)
   float* rsq = nullptr;     // [slots][2 ceil(d/256)][T'] RMSNorm partial sums (tensor-core path)
   void* qkv = nullptr;      // [slots][T'][Nqkv]  (fp32 / fp16)
@@ -97,12 +96,12 @@ struct Workspace {
   void* vt = nullptr;       // [slots][KV][hd][pitch] fp16 V^T for the tcgen05 attention
   void* gu = nullptr;       // [slots][T'][2F]    (fp32 path only)
   void* u = nullptr;        // [slots][T'][F]     (fp32 / fp16)
-  float* kv = nullptr;      // [slots][M][dk + d]
+  float* kv = nullptr;      // [slots][M][kv_ld] = k | v | gate logit (gated write)
   float* phik = nullptr;    // [slots][M][P]
   float* gram = nullptr;    // [slots][M][M] phi_j . phi_j'
   float* coef = nullptr;    // [slots][M] 1 / (z_j . phi_j + eps)
   float* gamma = nullptr;   // [slots][M]
-  void* a_act = nullptr;    // [L][d][P] fp16 copy of A (tensor-core path: the read GEMM operand)
+  float* beta = nullptr;    // [slots][M] write strength (gated write)
   float2* rope = nullptr;   // [hd/2][tp_max] (cos, sin), frequency-major
   NodeEntry* nodes = nullptr;
   int nodes_cap = 0;
@@ -120,14 +119,20 @@ struct Weights {
   void* w_gu = nullptr;      // [L][2F][d]     mlp gain folded; gate rows then up rows
   void* w_down = nullptr;    // [L][d][F]
   void* w_qm = nullptr;      // [L][dk][d]
-  void* w_kvm = nullptr;     // [L][dk+d][d]   key rows then value rows
+  void* w_kvm = nullptr;     // [L][kv_ld][d]  key rows, value rows, gate row (gated write), zero rows
 };
 
 struct Dims {
   int L, d, H, KV, hd, F, M, dk, nu, P, nqkv;
   float theta, rms_eps, mem_eps;
   bool bf16;
+  bool write_gate = false;   // beta_j = sigmoid(w_beta . m_j) scales each row's write of A
+  bool clamp_gamma = true;   // gamma_j clamped to [0, 1]
 };
+
+// Columns of a projected memory row [k (dk) | v (d) | gate logit]: the gated
+// write adds one column, padded to 16 so the projection keeps N % 16 == 0.
+inline int kv_ld(const Dims& dm) { return dm.dk + dm.d + (dm.write_gate ? 16 : 0); }
 
 }  // namespace armt
 
@@ -144,7 +149,7 @@ struct armt_ctx {
   cudaGraphExec_t graph_exec = nullptr;
   cudaStream_t capture_stream = nullptr;
   struct GraphKey {
-    int S = -1, T = -1, sched = -1;
+    int S = -1, T = -1, sched = -1, carry = 0;
     const void* emb = nullptr; void* out = nullptr; float* A = nullptr; float* z = nullptr;
   } graph_key;
   // node table of the last (S, schedule)
@@ -185,11 +190,15 @@ cudaError_t launch_simt_gemm(const GemmArgs& a, cudaStream_t st);
 // xb the fp16 copy, row-major.
 cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                                     const void* emb, const float* mem_emb, float* h, f16* xb, cudaStream_t st);
+// Tensor-core path: per-row sums of squares of the row-blocked residual into
+// the RMSNorm partials rsq[slot][part][pitch] (part 0 the row's sum, the rest 0).
+cudaError_t launch_row_sumsq(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h, float* rsq,
+                             long long rsq_slot_stride, int parts, int pitch, cudaStream_t st);
 // RMSNorm (no gain) of rows row0 .. row0+nrows-1 of every node's slot.
 cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int row0, int nrows,
                            const float* h, void* xb, float eps, cudaStream_t st);
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
-                             const float* z_state, void* phi, float* inv_den, unsigned* err, cudaStream_t st);
+                             const float* z_state, float* phi, float* inv_den, cudaStream_t st);
 // rope: [hd/2][rope_pitch] (cos, sin) of angle p * theta^(-2j/hd) at [j][p]
 cudaError_t launch_rope(const Dims& dm, const NodeEntry* nodes, int n, int Tp, void* qkv,
                         const float2* rope, int rope_pitch, cudaStream_t st);
@@ -199,32 +208,28 @@ cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
                           void* u, cudaStream_t st);
 // shared memory of memw_phi (bytes)
 size_t memw_phi_smem(const Dims& dm);
+// kv rows of kv_ld(dm) columns; beta [slots][M] written (gated write) or unused
 cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                            float* z_state, float* phik, float* gram, float* coef, float* gamma,
+                            float* z_state, float* phik, float* gram, float* coef, float* gamma, float* beta,
                             cudaStream_t st);
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                               const float* phik, const float* gram, const float* coef, float* A_state,
-                               void* a_act, unsigned* err, cudaStream_t st);
+                               const float* phik, const float* gram, const float* coef, const float* beta,
+                               float* A_state, cudaStream_t st);
 cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                           const float* h, void* out, cudaStream_t st);
 
 cudaError_t setup_memory_kernels(const Dims& dm);
 
-// tcgen05 attention (head_dim 64): reads V^T [slot][KV][hd][vt_pitch]
+// tcgen05 attention (head_dim 64 or 128): reads V^T [slot][KV][hd][vt_pitch]
 bool attention_tc_supported(const Dims& dm);
 int attention_tc_vt_pitch(int Tp);
 cudaError_t setup_attention_tc();
 cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int slots, const void* qkv,
                                 const void* vt, void* out, unsigned* err, cudaStream_t st);
 
-// warp-level tensor-core attention (mma.sync); head_dim 64 or 128
-bool attention_mma_supported(const Dims& dm);
-cudaError_t setup_attention_mma();
-cudaError_t launch_attention_mma(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const void* qkv, void* out,
-                                 cudaStream_t st);
-
 // weight conversions at load: fp32 copy, or bf16 rounding (RNE) stored as fp16
-enum ConvertMode { CONVERT_COPY_F32 = 0, CONVERT_BF16_AS_F16 = 1 };
+// weight upload: fp32 copy; fp32 -> bf16 (RNE) held in fp16; fp32 -> fp16 (RNE)
+enum ConvertMode { CONVERT_COPY_F32 = 0, CONVERT_BF16_AS_F16 = 1, CONVERT_F16 = 2 };
 cudaError_t launch_convert(const float* src, void* dst, size_t n, int mode, cudaStream_t st);
 
 }  // namespace armt

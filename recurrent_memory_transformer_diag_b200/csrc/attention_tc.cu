@@ -1,5 +1,5 @@
 // Batched causal attention on the 5th-generation tensor cores (tcgen05,
-// TMEM accumulators, TMA-fed operands), head_dim 64.
+// TMEM accumulators, TMA-fed operands), head_dim 64 or 128.
 //
 // The wave's nodes are a batch: a CTA handles one 128-row query tile of one
 // node for the H/KV query heads that share a kv head, so the node's keys and
@@ -10,22 +10,30 @@
 //
 // Two softmax warpgroups (A: warps 2..5, B: warps 6..9; one thread per query
 // row) take the even and the odd query heads of the group, so two heads are
-// in flight and share every K/V tile.  Per key tile j and warpgroup w:
-//   MMA  S_w = Q_w K_j^T          (M=128 queries, N=128 keys, K=64) -> TMEM
-//   softmax: row max, p = exp2(s - m) as fp16 P_w in shared memory (K-major,
-//            128-byte swizzle)
-//   MMA  O_w += P_w [V_j | 1]     (M=128, N=80, K=128 keys), O_w stays in TMEM;
-//        column 64 of O_w accumulates the row sums of P (a ones row is
-//        appended to V^T in shared memory), so the softmax never sums
-//        probabilities itself and the sum follows every rescaling of O
+// in flight and share every K/V tile; each has its own MMA-issuer warp (1 for
+// A, 10 for B).  Per key tile j and warpgroup w:
+//   MMA  S_w = Q_w K_j^T          (M=128 queries, N=128 keys, K=hd) -> TMEM
+//   softmax: row max, p = exp2(s - m) and its fp32 row sum in registers; P_w
+//            (fp16 pairs) written to TMEM
+//   MMA  O_w += P_w V_j           (M=128, N=hd, K=128 keys; P_w read from
+//        TMEM), O_w stays in TMEM
 // The running max m is only raised when a row's max grows by more than 8 (in
-// log2 units): then that row of O_w is rescaled in TMEM; otherwise the stale
-// max is kept (p <= 2^8 fits fp16 and the row sum uses the same max, so the
-// result is exact).  The MMA warp interleaves O_A(j), S_A(j+1), O_B(j),
-// S_B(j+1) so one warpgroup's softmax overlaps the other's tensor work.  V is
-// read as V^T (written transposed by the QKV epilogue): every operand is
-// K-major.  All mbarrier waits are bounded; on timeout the kernel sets the
-// error word, drains its copies and MMAs, frees TMEM and exits.
+// log2 units): then that row of O_w and its row sum are rescaled; otherwise
+// the stale max is kept (p <= 2^8 fits fp16 and the row sum uses the same
+// max, so the result is exact).  V is read as V^T (written transposed by the
+// QKV epilogue): every shared-memory operand is K-major.
+//
+// TMEM (512 columns).  hd = 64: S_A, S_B (128 each), O_A, O_B (64 each), P_A,
+// P_B (64 each); S(j+1) is issued before O(j), as soon as the softmax holds
+// the scores of step j in registers.  hd = 128: S_A, S_B, O_A, O_B take 128
+// columns each and P_w is written over the first 64 columns of S_w (the
+// scores are in registers by then), so S(j+1) is issued after O(j) (MMAs of
+// one issuing thread run in order) and the other warpgroup's products fill
+// the tensor core meanwhile.  Shared memory at hd = 128: one Q buffer per
+// warpgroup, three K and two V stages (224 KB).
+//
+// All mbarrier waits are bounded; on timeout the kernel sets the error word,
+// drains its copies and MMAs, frees TMEM and exits.
 #include "armt_internal.cuh"
 #include "tcgen05_ptx.cuh"
 
@@ -35,27 +43,39 @@ namespace {
 
 using namespace tc;
 
-constexpr int HD = 64;
 constexpr int BQ = 128;                 // query rows per tile
 constexpr int BKEY = 128;               // keys per tile
 constexpr int NUM_THREADS = 352;        // warp 0 TMA, warps 1 / 10 MMA for warpgroup A / B, warps 2..9 softmax
-constexpr int Q_BYTES = BQ * HD * 2;    // 16 KB
-constexpr int K_BYTES = BKEY * HD * 2;  // 16 KB
-constexpr int VT_BYTES = HD * BKEY * 2; // 16 KB loaded per stage (two 64-key blocks of 8 KB)
-constexpr int VT_BLK = HD * 128;        // V^T block in shared memory: 64 rows (dims) of 64 keys (8 KB)
-constexpr int K_STAGES = 4;             // K is needed first (S of the next step): deeper ring
-constexpr int V_STAGES = 3;             // V^T only at O, a softmax later
-constexpr int OFF_Q = 0;                               // [2 warpgroups][2 buffers]
-constexpr int OFF_K = OFF_Q + 4 * Q_BYTES;             // [K_STAGES]
-constexpr int OFF_VT = OFF_K + K_STAGES * K_BYTES;     // [V_STAGES][2 blocks of VT_BLK]
-constexpr int OFF_BAR = OFF_VT + V_STAGES * 2 * VT_BLK;
-constexpr int SMEM_TOTAL = OFF_BAR + 512 + 1024;
-static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
-// TMEM columns: S_A, S_B (fp32 scores, 128 each), O_A, O_B (fp32, 64 each),
-// P_A, P_B (fp16 probabilities packed in pairs, 64 each)
-constexpr int TM_S = 0, TM_O = 2 * BKEY, TM_P = TM_O + 2 * HD;
+constexpr int HALF_BYTES = 128 * 128;   // 128 rows x 64 dims (fp16): one 128-byte-swizzled operand block
 constexpr int TMEM_COLS = 512;
-static_assert(TM_P + 2 * (BKEY / 2) <= TMEM_COLS, "tensor memory");
+
+// Tile geometry per head_dim.  A Q or K tile is hd / 64 blocks of 128 rows x
+// 64 dims (a 128-byte swizzle row holds 64 fp16 values); a V^T stage is two
+// blocks of hd rows (dims) x 64 keys.
+template <int HD_>
+struct AttnShape {
+  static constexpr int HD = HD_;
+  static constexpr int Q_BYTES = BQ * HD * 2;          // 16 / 32 KB
+  static constexpr int K_BYTES = BKEY * HD * 2;        // 16 / 32 KB
+  static constexpr int VT_BLK = HD * 128;              // hd rows of 64 keys
+  static constexpr int VT_BYTES = 2 * VT_BLK;          // one 128-key stage
+  static constexpr int QB = HD == 64 ? 2 : 1;          // Q buffers per warpgroup (2: next head loaded ahead)
+  static constexpr int K_STAGES = HD == 64 ? 4 : 3;    // K is needed first (S of the next step): deeper ring
+  static constexpr int V_STAGES = HD == 64 ? 3 : 2;    // V^T only at O, a softmax later
+  static constexpr bool P_IN_S = HD == 128;            // P written over S (TMEM holds 2 S + 2 O of 128 columns)
+  static constexpr int OFF_Q = 0;                                // [2 warpgroups][QB buffers]
+  static constexpr int OFF_K = OFF_Q + 2 * QB * Q_BYTES;         // [K_STAGES]
+  static constexpr int OFF_VT = OFF_K + K_STAGES * K_BYTES;      // [V_STAGES][2 blocks of VT_BLK]
+  static constexpr int OFF_BAR = OFF_VT + V_STAGES * VT_BYTES;
+  static constexpr int SMEM_TOTAL = OFF_BAR + 512 + 1024;
+  static_assert(SMEM_TOTAL <= 227 * 1024, "shared memory");
+  // TMEM columns: S_A, S_B (fp32 scores, 128 each), O_A, O_B (fp32, hd each),
+  // P_A, P_B (fp16 probabilities packed in pairs, 64 each; over S at hd = 128)
+  static constexpr int TM_S = 0, TM_O = 2 * BKEY;
+  static constexpr int TM_P = P_IN_S ? TM_S : TM_O + 2 * HD;
+  static constexpr int TM_P_STRIDE = P_IN_S ? BKEY : BKEY / 2;
+  static_assert(TM_O + 2 * HD <= TMEM_COLS && TM_P + 2 * TM_P_STRIDE <= TMEM_COLS, "tensor memory");
+};
 constexpr float RESCALE_THRESHOLD = 8.f;
 // Share of the exponentials taken off the MUFU unit (every POLY_EVERY-th
 // pair by polynomial; 0 = none).  A quarter measured 3 % faster than none on
@@ -121,9 +141,15 @@ __device__ __forceinline__ float ex2_poly(float x) {
   return __uint_as_float(__float_as_uint(q) + (__float_as_uint(t) << 23));
 }
 
+template <int HD_>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm_qk, const __grid_constant__ CUtensorMap tm_vt,
                         const AttnParams p) {
+  using SH = AttnShape<HD_>;
+  constexpr int HD = SH::HD, QB = SH::QB, K_STAGES = SH::K_STAGES, V_STAGES = SH::V_STAGES;
+  constexpr int Q_BYTES = SH::Q_BYTES, K_BYTES = SH::K_BYTES, VT_BLK = SH::VT_BLK, VT_BYTES = SH::VT_BYTES;
+  constexpr int OFF_Q = SH::OFF_Q, OFF_K = SH::OFF_K, OFF_VT = SH::OFF_VT, OFF_BAR = SH::OFF_BAR;
+  constexpr int TM_S = SH::TM_S, TM_O = SH::TM_O, TM_P = SH::TM_P, TM_P_STRIDE = SH::TM_P_STRIDE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
@@ -164,7 +190,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   };
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 4; ++b) {
+    for (int b = 0; b < 2 * QB; ++b) {
       mbar_init(&q_full[b], 1);
       mbar_init(&q_empty[b], 1);
     }
@@ -265,8 +291,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int& qi = w ? qi_b : qi_a;
         int& qr = w ? qr_b : qr_a;
         int& qk = w ? qk_b : qk_a;
-        const int qb = w * 2 + (qi & 1);
-        const uint32_t par = ((qi >> 1) & 1) ^ 1;
+        const int qb = w * QB + qi % QB;
+        const uint32_t par = ((qi / QB) & 1) ^ 1;
         if (block) {
           if (!mbar_wait_warp(&q_empty[qb], par, abort_flag)) return -1;
         } else if (!__any_sync(0xffffffffu, mbar_try_wait(&q_empty[qb], par))) {
@@ -275,7 +301,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         NodeEntry nd; int g, q0, nt;
         decode(item_of(qr), nd, g, q0, nt);
         if (issuer) mbar_expect_tx(&q_full[qb], Q_BYTES);
-        if (issuer) tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES, (g * grp + w + 2 * qk) * HD, q0, nd.z);
+#pragma unroll
+        for (int h = 0; h < HD / 64; ++h)   // 64-dim blocks of the head
+          if (issuer)
+            tma_load_3d(&tm_qk, &q_full[qb], smem + OFF_Q + qb * Q_BYTES + h * HALF_BYTES,
+                        (g * grp + w + 2 * qk) * HD + h * 64, q0, nd.z);
         armed |= 1u << qb;
         ++qi;
         if (++qk >= (w ? heads_b : heads_a)) { qk = 0; ++qr; }
@@ -288,7 +318,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         NodeEntry nd; int g, q0, nt;
         decode(c.u, nd, g, q0, nt);
         if (issuer) mbar_expect_tx(&v_full[vs], VT_BYTES);
-        uint8_t* vt = smem + OFF_VT + vs * 2 * VT_BLK;
+        uint8_t* vt = smem + OFF_VT + vs * VT_BYTES;
         const int vt_outer = nd.z * p.KV + g;
         if (issuer) tma_load_3d(&tm_vt, &v_full[vs], vt, j * BKEY, 0, vt_outer);
         if (issuer) tma_load_3d(&tm_vt, &v_full[vs], vt + VT_BLK, j * BKEY + 64, 0, vt_outer);
@@ -313,7 +343,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             NodeEntry nd; int g, q0, nt;
             decode(c.u, nd, g, q0, nt);
             if (issuer) mbar_expect_tx(&k_full[ks], K_BYTES);
-            if (issuer) tma_load_3d(&tm_qk, &k_full[ks], smem + OFF_K + ks * K_BYTES, (p.H + g) * HD, j * BKEY, nd.z);
+#pragma unroll
+            for (int h = 0; h < HD / 64; ++h)
+              if (issuer)
+                tma_load_3d(&tm_qk, &k_full[ks], smem + OFF_K + ks * K_BYTES + h * HALF_BYTES, (p.H + g) * HD + h * 64,
+                            j * BKEY, nd.z);
             armed |= 16u << ks;
           }
           if (has_prev && !load_v(prev)) { ok = false; break; }
@@ -333,7 +367,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (*abort_flag) {   // let every issued copy land before the CTA exits
         const unsigned long long t0 = global_ns();
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < 2 * QB; ++b)
           if (armed & (1u << b))
             while (!mbar_try_wait(&q_full[b], 0) && !mbar_try_wait(&q_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
         for (int b = 0; b < K_STAGES; ++b)
@@ -352,21 +386,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int w = warp == 1 ? 0 : 1;
     const bool issuer = elect_one();
     const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
-    const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x 64 x 16
+    const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x hd x 16
     auto active = [&](const Cursor& c) { return w == 0 || c.t < c.nB; };
     // S_w = Q_w K_j^T for step c
     auto issue_s = [&](const Cursor& c) -> bool {
       const int hidx = (w ? c.qh0_b : c.qh0_a) + c.k, sidx = (w ? c.sw0_b : c.sw0_a) + c.t, kidx = c.kv0 + c.t;
-      const int qb = w * 2 + (hidx & 1), ks = kidx % K_STAGES;
-      if (c.j == 0 && !mbar_wait_warp(&q_full[qb], (hidx >> 1) & 1, abort_flag)) return false;
+      const int qb = w * QB + hidx % QB, ks = kidx % K_STAGES;
+      if (c.j == 0 && !mbar_wait_warp(&q_full[qb], (hidx / QB) & 1, abort_flag)) return false;
       if (!mbar_wait_warp(&k_full[ks], (kidx / K_STAGES) & 1, abort_flag)) return false;
       if (!mbar_wait_warp(&s_empty[w], (sidx & 1) ^ 1, abort_flag)) return false;
       tc_fence_after();
       const uint32_t qa = smem_u32(smem + OFF_Q + qb * Q_BYTES);
       const uint32_t ka = smem_u32(smem + OFF_K + ks * K_BYTES);
 #pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk)
-        if (issuer) mma_f16(tmem_base + TM_S + w * BKEY, sw128_desc(qa + kk * 32), sw128_desc(ka + kk * 32), idesc_s, kk > 0);
+      for (int kk = 0; kk < HD / 16; ++kk) {   // 16 dims per instruction, 4 per 64-dim block
+        const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+        if (issuer) mma_f16(tmem_base + TM_S + w * BKEY, sw128_desc(qa + off), sw128_desc(ka + off), idesc_s, kk > 0);
+      }
       if (issuer) mma_commit(&s_full[w]);
       if (c.j == c.ntiles - 1 && issuer) mma_commit(&q_empty[qb]);   // Q buffer free once these MMAs finish
       return true;
@@ -377,8 +413,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!mbar_wait_warp(&p_full[w], sidx & 1, abort_flag)) return false;
       if (!mbar_wait_warp(&v_full[vs], (kidx / V_STAGES) & 1, abort_flag)) return false;
       tc_fence_after();
-      const uint32_t pa = tmem_base + TM_P + w * (BKEY / 2);   // P_w in TMEM: 8 columns per 16 keys
-      const uint32_t va = smem_u32(smem + OFF_VT + vs * 2 * VT_BLK);
+      const uint32_t pa = tmem_base + TM_P + w * TM_P_STRIDE;   // P_w in TMEM: 8 columns per 16 keys
+      const uint32_t va = smem_u32(smem + OFF_VT + vs * VT_BYTES);
 #pragma unroll
       for (int kb = 0; kb < BKEY / 64; ++kb)
 #pragma unroll
@@ -412,9 +448,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       return true;
     };
-    // S of the next step is issued before O of the current one (the S buffer
-    // is free once the softmax has the scores in registers), so the softmax
-    // finds its next scores computed when it finishes a tile.
+    // hd = 64: S of the next step is issued before O of the current one (the
+    // S buffer is free once the softmax has the scores in registers), so the
+    // softmax finds its next scores computed when it finishes a tile.
+    // hd = 128: P_w lives in S_w's columns, so S of the next step follows O of
+    // the current one (in issue order, which the tensor core keeps).
     bool ok = true;
     if (blockIdx.x < n_items) {
       Cursor cur;
@@ -424,12 +462,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       while (ok) {
         Cursor nxt = cur;
         const bool more = advance(nxt);
+        if (SH::P_IN_S) {
+          if (active(cur) && !issue_o(cur)) { ok = false; break; }
+          if (!release_v(cur)) { ok = false; break; }
+        }
         if (more) {
           if (active(nxt) && !issue_s(nxt)) { ok = false; break; }
           if (!release_k(nxt)) { ok = false; break; }
         }
-        if (active(cur) && !issue_o(cur)) { ok = false; break; }
-        if (!release_v(cur)) { ok = false; break; }
+        if (!SH::P_IN_S) {
+          if (active(cur) && !issue_o(cur)) { ok = false; break; }
+          if (!release_v(cur)) { ok = false; break; }
+        }
         if (!more) break;
         cur = nxt;
       }
@@ -451,7 +495,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tm = tmem_base + lane_off + TM_S + w * BKEY;
     const uint32_t o_tm = tmem_base + lane_off + TM_O + w * HD;
-    const uint32_t p_tm = tmem_base + lane_off + TM_P + w * (BKEY / 2);
+    const uint32_t p_tm = tmem_base + lane_off + TM_P + w * TM_P_STRIDE;
     const int heads = w == 0 ? heads_a : heads_b;
     int sbase = 0;
     bool ok = true;
@@ -461,24 +505,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     float pend_l = 1.f;         // its row sum of P
     int last_sidx = 0;
     // O of a finished head (complete, waited for): normalise by the row sum,
-    // fp16 row of the head's 64 outputs
+    // fp16 row of the head's hd outputs (64 columns at a time)
     auto finalize = [&](f16* dst, float l) {
-      uint32_t orr[HD];
-      tmem_ld64_nowait(o_tm, orr);
-      tmem_wait_ld();
-      if (dst) {
-        const float inv = 1.f / l;
+#pragma unroll 1
+      for (int c = 0; c < HD / 64; ++c) {
+        uint32_t orr[64];
+        tmem_ld64_nowait(o_tm + c * 64, orr);
+        tmem_wait_ld();
+        if (dst) {
+          const float inv = 1.f / l;
 #pragma unroll
-        for (int q = 0; q < HD / 8; ++q) {
-          uint4 v;
-          uint32_t* wv = reinterpret_cast<uint32_t*>(&v);
+          for (int q = 0; q < 8; ++q) {
+            uint4 v;
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&v);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
-                                           __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
-            wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+            for (int i = 0; i < 4; ++i) {
+              __half2 h2 = __floats2half2_rn(__uint_as_float(orr[q * 8 + 2 * i]) * inv,
+                                             __uint_as_float(orr[q * 8 + 2 * i + 1]) * inv);
+              wv[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+            reinterpret_cast<uint4*>(dst + c * 64)[q] = v;
           }
-          reinterpret_cast<uint4*>(dst)[q] = v;
         }
       }
     };
@@ -568,12 +615,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pend = false;
         }
         if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access; rows that keep their max scale by 1
-          uint32_t orr[HD];
-          tmem_ld64_nowait(o_tm, orr);
-          tmem_wait_ld();
+#pragma unroll 1
+          for (int c = 0; c < HD / 64; ++c) {
+            uint32_t orr[64];
+            tmem_ld64_nowait(o_tm + c * 64, orr);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < HD; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
-          tmem_st64(o_tm, orr);
+            for (int i = 0; i < 64; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * corr);
+            tmem_st64(o_tm + c * 64, orr);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -631,23 +681,29 @@ cudaError_t make_map(CUtensorMap* map, const void* base, int inner, int rows, in
 
 }  // namespace
 
-bool attention_tc_supported(const Dims& dm) { return dm.bf16 && dm.hd == HD; }
+bool attention_tc_supported(const Dims& dm) { return dm.bf16 && (dm.hd == 64 || dm.hd == 128); }
 
 int attention_tc_vt_pitch(int Tp) { return (Tp + 7) / 8 * 8; }
 
 cudaError_t setup_attention_tc() {
   if (!get_tensor_map_encoder()) return cudaErrorNotSupported;
-  return cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       AttnShape<64>::SMEM_TOTAL);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attention_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             AttnShape<128>::SMEM_TOTAL);
+  return e;
 }
 
 cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, int Tp, int slots, const void* qkv,
                                 const void* vt, void* out, unsigned* err, cudaStream_t st) {
   if (!attention_tc_supported(dm)) return cudaErrorInvalidValue;
   CUtensorMap tm_qk, tm_vt;
-  // Q and K tiles: [slot][Tp][nqkv], box 64 dims x 128 rows
-  cudaError_t e = make_map(&tm_qk, qkv, dm.nqkv, Tp, slots, dm.nqkv, (long long)Tp * dm.nqkv, HD, BQ);
+  const int HD = dm.hd;
+  // Q and K tiles: [slot][Tp][nqkv], box 64 dims x 128 rows (hd / 64 boxes per tile)
+  cudaError_t e = make_map(&tm_qk, qkv, dm.nqkv, Tp, slots, dm.nqkv, (long long)Tp * dm.nqkv, 64, BQ);
   if (e != cudaSuccess) return e;
-  // V^T tiles: [slot * KV + g][hd][pitch], box 64 keys x 64 dims
+  // V^T tiles: [slot * KV + g][hd][pitch], box 64 keys x hd dims
   const int pitch = attention_tc_vt_pitch(Tp);
   e = make_map(&tm_vt, vt, Tp, HD, slots * dm.KV, pitch, (long long)HD * pitch, 64, HD);
   if (e != cudaSuccess) return e;
@@ -666,8 +722,12 @@ cudaError_t launch_attention_tc(const Dims& dm, const NodeEntry* nodes, int n, i
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int items = n * dm.KV * p.q_tiles;
-  return launch_pdl(attention_tc_kernel, dim3(items < sms ? items : sms), dim3(NUM_THREADS), SMEM_TOTAL, st, tm_qk,
-                    tm_vt, p);
+  const dim3 grid(items < sms ? items : sms);
+  if (HD == 128)
+    return launch_pdl(attention_tc_kernel<128>, grid, dim3(NUM_THREADS), AttnShape<128>::SMEM_TOTAL, st, tm_qk,
+                      tm_vt, p);
+  return launch_pdl(attention_tc_kernel<64>, grid, dim3(NUM_THREADS), AttnShape<64>::SMEM_TOTAL, st, tm_qk, tm_vt,
+                    p);
 }
 
 }  // namespace armt

@@ -10,15 +10,17 @@
 // each seeing the state (A, z) left by the previous rows:
 //   vbar_j  = A phi_j / (z . phi_j + eps)
 //   gamma_j = clamp(1 - (z . phi_j) / (|phi_j|^2 + eps), 0, 1)
-//   A      += (v_j - vbar_j) phi_j^T
+//   A      += beta_j (v_j - vbar_j) phi_j^T
 //   z      += gamma_j phi_j
+// with beta_j = 1, or, for the gated write, beta_j = sigmoid(w_beta . m_j)
+// (the projection's extra output column); gamma_j may also be left unclamped.
 //
 // Work split.  With z_j the normaliser before row j and G the Gram matrix
 // G[j'][j] = phi_j' . phi_j:  z_j . phi_j = z_0 . phi_j + sum_{j'<j} gamma_j' G[j'][j]
 // (memw_phi: one block per node, a scalar recurrence after the M dot
 // products).  Row i of A: with a the row before the write,
 //   (A_j phi_j)[i] = a . phi_j + sum_{j'<j} delta_j' G[j'][j],
-//   delta_j = v_j[i] - (A_j phi_j)[i] / (z_j . phi_j + eps),
+//   delta_j = beta_j (v_j[i] - (A_j phi_j)[i] / (z_j . phi_j + eps)),
 //   new row = a + sum_j delta_j phi_j
 // so memw_update streams A once, row by row (one read, one write per node).
 #include "armt_internal.cuh"
@@ -31,14 +33,14 @@ __device__ __forceinline__ float warp_sum_m(float v) {
   return v;
 }
 
-// kv: [slot][M][dk + d] (k first), phik: [slot][M][P], gram: [slot][M][M],
-// coef/gamma: [slot][M].  One block per node: one warp per memory row for the
-// features (phi kept in shared memory for the Gram matrix), warps over row
-// pairs for the Gram matrix, one thread for the M-step recurrence, all
-// threads for the z update.
-__global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, int P, int nu,
+// kv: [slot][M][ldkv] rows [k (dk) | v (d) | gate logit (gated write)],
+// phik: [slot][M][P], gram: [slot][M][M], coef/gamma/beta: [slot][M].  One
+// block per node: one warp per memory row for the features (phi kept in
+// shared memory for the Gram matrix), warps over row pairs for the Gram
+// matrix, one warp for the M-step recurrence, all threads for the z update.
+__global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, int P, int nu, int ldkv,
                                 const float* kv, float* z_state, float* phik, float* gram, float* coef,
-                                float* gamma, float eps) {
+                                float* gamma, float* beta, int clamp_gamma, float eps) {
   grid_dependency_sync();
   extern __shared__ float sh[];
   const int nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -55,7 +57,8 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
   for (int p = threadIdx.x; p < P; p += blockDim.x) zs[p] = z[p];
   __syncthreads();
   for (int j = warp; j < M; j += nw) {
-    const float* k = kv + ((long long)slot * M + j) * (dk + d);
+    const float* k = kv + ((long long)slot * M + j) * ldkv;
+    if (beta && lane == 0) beta[(long long)slot * M + j] = 1.f / (1.f + __expf(-k[dk + d]));
     float* rw = r + warp * n2;
     for (int c = lane; c < dk; c += 32) {
       const float kc = k[c];
@@ -101,7 +104,8 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
     // and the later lanes add its term
     float zp = lane < M ? zp0[lane] : 0.f;
     for (int j = 0; j < M; ++j) {
-      const float gm_l = fminf(fmaxf(1.f - zp / (G[(lane < M ? lane : 0) * (M + 1)] + eps), 0.f), 1.f);
+      const float g_raw = 1.f - zp / (G[(lane < M ? lane : 0) * (M + 1)] + eps);
+      const float gm_l = clamp_gamma ? fminf(fmaxf(g_raw, 0.f), 1.f) : g_raw;
       const float gm = __shfl_sync(0xffffffffu, gm_l, j);
       if (lane == j) {
         gam[j] = gm;
@@ -127,19 +131,19 @@ size_t memw_phi_smem(const Dims& dm) {
 }
 
 cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                            float* z_state, float* phik, float* gram, float* coef, float* gamma,
+                            float* z_state, float* phik, float* gram, float* coef, float* gamma, float* beta,
                             cudaStream_t st) {
   const int nw = dm.M < 32 ? dm.M : 32;
   return launch_pdl(memw_phi_kernel, dim3(n), dim3(nw * 32), memw_phi_smem(dm), st, nodes, dm.M, dm.dk, dm.d, dm.P,
-                    dm.nu, kv, z_state, phik, gram, coef, gamma, dm.mem_eps);
+                    dm.nu, kv_ld(dm), kv, z_state, phik, gram, coef, gamma, dm.write_gate ? beta : nullptr,
+                    dm.clamp_gamma ? 1 : 0, dm.mem_eps);
 }
 
 constexpr int MEMW_ROWS_PER_BLOCK = 64;
 
-// A_state: [L][d][P] fp32 in place; a_act: optional fp16 copy [L][d][P] (a
-// value past the fp16 range sets the error word).
+// A_state: [L][d][P] fp32 in place.
 // grid (ceil(d / MEMW_ROWS_PER_BLOCK), nodes), 8 warps, one A row per warp per
-// iteration; phi, G and coef are staged once per block.
+// iteration; phi, G, coef and beta are staged once per block.
 // Transposed warp reduction of MT per-lane partial sums: afterwards lane l
 // holds the warp-wide total of index j = l >> (5 - log2 MT).  Each stage
 // halves the values a lane keeps and exchanges the other half with its
@@ -180,9 +184,9 @@ constexpr int MEMW_R = 2;
 
 template <int MAXC, int MT>
 __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
-                                                          const float* kv, const float* phik,
-                                                          const float* gram, const float* coef, float* A_state,
-                                                          f16* a_act, unsigned* err) {
+                                                          int ldkv, const float* kv, const float* phik,
+                                                          const float* gram, const float* coef, const float* beta,
+                                                          float* A_state) {
   grid_dependency_sync();
   constexpr int R = MEMW_R;
   extern __shared__ float sh[];
@@ -198,12 +202,12 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* dl = dots + warp * R * M;
-  bool over = false;
   constexpr int SHIFT = 5 - log2_const<MT>();
   const float cj = lane < M ? cf[lane] : 0.f;
+  const float bj = (beta && lane < M) ? beta[(long long)slot * M + lane] : 1.f;
   const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
   const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
-  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * ldkv + dk;
   for (int i0 = i_begin + warp; i0 < i_end; i0 += 8 * R) {
     float a[R][MAXC];
     float v[R];
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
       const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
+        const float dj = __shfl_sync(0xffffffffu, bj * (v[r] - sv[r] * cj), j);
         if (lane == j) dl[r * M + j] = dj;
         sv[r] = fmaf(dj, gj, sv[r]);
       }
@@ -273,18 +277,12 @@ __global__ void __launch_bounds__(256) memw_update_kernel(const NodeEntry* nodes
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           if (!has[r]) continue;
-          const long long off = ((long long)layer * d + i0 + 8 * r) * P + p;
-          A_state[off] = acc[r];
-          if (a_act) {
-            a_act[off] = __float2half_rn(acc[r]);
-            over |= fabsf(acc[r]) > 65504.f;
-          }
+          A_state[((long long)layer * d + i0 + 8 * r) * P + p] = acc[r];
         }
       }
     }
     __syncwarp();
   }
-  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
 // Same computation with 16-byte accesses (P % 4 == 0): lane l owns the
@@ -305,9 +303,9 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 
 template <int C4, int MT, bool PF>
 __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry* nodes, int M, int dk, int d, int P,
-                                                                 const float* kv, const float* phik,
+                                                                 int ldkv, const float* kv, const float* phik,
                                                                  const float* gram, const float* coef,
-                                                                 float* A_state, f16* a_act, unsigned* err) {
+                                                                 const float* beta, float* A_state) {
   grid_dependency_sync();
   constexpr int R = MEMW_R;
   extern __shared__ float sh[];
@@ -329,12 +327,12 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
   __syncthreads();
   const float4* ph4 = reinterpret_cast<const float4*>(ph);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  bool over = false;
   constexpr int SHIFT = 5 - log2_const<MT>();
   const float cj = lane < M ? cf[lane] : 0.f;
+  const float bj = (beta && lane < M) ? beta[(long long)slot * M + lane] : 1.f;
   const int i_begin = blockIdx.x * MEMW_ROWS_PER_BLOCK;
   const int i_end = min(d, i_begin + MEMW_ROWS_PER_BLOCK);
-  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * (dk + d) + dk;
+  const float* kvj = kv + ((long long)slot * M + (lane < M ? lane : 0)) * ldkv + dk;
   // rows i0n + 8 r of this warp -> buffer b (each lane copies the 16-byte
   // groups it later reads itself)
   auto issue_rows = [&](int i0n, int b) {
@@ -419,7 +417,7 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
         const float gj = (lane > j && lane < M) ? G[j * M + lane] : 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-          const float dj = __shfl_sync(0xffffffffu, v[r] - sv[r] * cj, j);
+          const float dj = __shfl_sync(0xffffffffu, bj * (v[r] - sv[r] * cj), j);
           dreg[r][j] = dj;
           sv[r] = fmaf(dj, gj, sv[r]);
         }
@@ -452,23 +450,13 @@ __global__ void __launch_bounds__(256, 2) memw_update_vec_kernel(const NodeEntry
 #pragma unroll
         for (int r = 0; r < R; ++r) {
           if (!has[r]) continue;
-          const long long off = ((long long)layer * d + i0 + 8 * r) * P + 4 * q;
-          *reinterpret_cast<float4*>(A_state + off) = acc[r];
-          if (a_act) {
-            const __half2 lo = __floats2half2_rn(acc[r].x, acc[r].y), hi = __floats2half2_rn(acc[r].z, acc[r].w);
-            uint2 pk;
-            pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-            pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-            *reinterpret_cast<uint2*>(a_act + off) = pk;
-            over |= fmaxf(fmaxf(fabsf(acc[r].x), fabsf(acc[r].y)), fmaxf(fabsf(acc[r].z), fabsf(acc[r].w))) > 65504.f;
-          }
+          *reinterpret_cast<float4*>(A_state + ((long long)layer * d + i0 + 8 * r) * P + 4 * q) = acc[r];
         }
       }
     }
     __syncwarp();
   }
   if (PF) cp_async_wait<0>();
-  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
 static size_t memw_update_smem(const Dims& dm) {
@@ -483,14 +471,16 @@ static size_t memw_update_pf_smem(const Dims& dm) {
 constexpr size_t MEMW_PF_SMEM_MAX = 110 * 1024;
 
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
-                               const float* phik, const float* gram, const float* coef, float* A_state,
-                               void* a_act, unsigned* err, cudaStream_t st) {
+                               const float* phik, const float* gram, const float* coef, const float* beta,
+                               float* A_state, cudaStream_t st) {
+  const int ldkv = kv_ld(dm);
+  if (!dm.write_gate) beta = nullptr;
   dim3 grid((dm.d + MEMW_ROWS_PER_BLOCK - 1) / MEMW_ROWS_PER_BLOCK, n);
   const size_t sh = memw_update_smem(dm);
   const int chunks = (dm.P + 31) / 32;
 #define ARMT_MEMW_CASE(C, MT)                                                                             \
-  memw_update_kernel<C, MT><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, kv, phik, gram, coef, \
-                                                   A_state, (f16*)a_act, err);
+  memw_update_kernel<C, MT><<<grid, 256, sh, st>>>(nodes, dm.M, dm.dk, dm.d, dm.P, ldkv, kv, phik, gram, coef, \
+                                                   beta, A_state);
 #define ARMT_MEMW_M(C)                  \
   {                                     \
     if (dm.M <= 4) ARMT_MEMW_CASE(C, 4) \
@@ -498,11 +488,10 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
     else ARMT_MEMW_CASE(C, 32)          \
   }
   if (dm.M > 32) return cudaErrorInvalidValue;
-  // the 16-byte kernel reads A rows and the phi rows as float4 and writes the
-  // fp16 copy 8 bytes at a time: every base it offsets must be aligned to that
+  // the 16-byte kernel reads and writes A rows and reads the phi rows as
+  // float4: both bases must be 16-byte aligned
   const bool aligned = (reinterpret_cast<uintptr_t>(A_state) & 15) == 0 &&
-                       (reinterpret_cast<uintptr_t>(phik) & 15) == 0 &&
-                       (reinterpret_cast<uintptr_t>(a_act) & 7) == 0;
+                       (reinterpret_cast<uintptr_t>(phik) & 15) == 0;
   if (dm.P % 4 == 0 && dm.P <= 1024 && aligned) {   // 16-byte path
     const int c4 = (dm.P / 4 + 31) / 32;
     const size_t sh_pf = memw_update_pf_smem(dm);
@@ -512,10 +501,10 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
   {                                                                                                                 \
     if (pf)                                                                                                         \
       e = launch_pdl(memw_update_vec_kernel<C, MT, true>, grid, dim3(256), sh_pf, st, nodes, dm.M, dm.dk, dm.d,   \
-                     dm.P, kv, phik, gram, coef, A_state, (f16*)a_act, err);                                        \
+                     dm.P, ldkv, kv, phik, gram, coef, beta, A_state);                                              \
     else                                                                                                            \
       e = launch_pdl(memw_update_vec_kernel<C, MT, false>, grid, dim3(256), sh, st, nodes, dm.M, dm.dk, dm.d, dm.P, \
-                     kv, phik, gram, coef, A_state, (f16*)a_act, err);                                              \
+                     ldkv, kv, phik, gram, coef, beta, A_state);                                                    \
   }
 #define ARMT_MEMWV_M(C)                  \
   {                                      \

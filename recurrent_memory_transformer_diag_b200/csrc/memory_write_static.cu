@@ -108,7 +108,7 @@ extern "C" armt_status armt_memory_write_static(int M, int d, int d_key, int nu,
     g.epi = EPI_STORE_F32;
     e = launch_simt_gemm(g, st);
   }
-  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, st);
-  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, A, nullptr, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, nullptr, A, st);
   return to_status(e);
 }

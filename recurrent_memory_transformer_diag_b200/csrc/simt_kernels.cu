@@ -159,6 +159,36 @@ cudaError_t launch_init_first_layer(const Dims& dm, const NodeEntry* nodes, int 
   return cudaGetLastError();
 }
 
+// Row sums of squares of the row-blocked residual (tensor-core path) as the
+// RMSNorm partials of the QKV epilogue: part 0 holds the whole row's sum, the
+// other parts 0 (used for the layer-0 input when no memory read runs first).
+// One warp per 32-row block: lane r walks row r's column groups, so the warp
+// reads each block's 32 x 4 floats of a group as one contiguous 512 bytes.
+__global__ void row_sumsq_kernel(const NodeEntry* nodes, int Tp, int d, const float* h, float* rsq,
+                                 long long rsq_slot_stride, int parts, int pitch) {
+  grid_dependency_sync();
+  const NodeEntry nd = nodes[blockIdx.y];
+  const int r = blockIdx.x * 32 + threadIdx.x;
+  const float4* hb = reinterpret_cast<const float4*>(h + (long long)nd.z * rows_blocked(Tp) * d +
+                                                     (long long)blockIdx.x * 32 * d) + threadIdx.x;
+  float ss = 0.f;
+  for (int g = 0; g < d / 4; ++g) {
+    const float4 v = hb[(long long)g * 32];
+    ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+  }
+  if (r >= Tp) return;
+  float* out = rsq + (long long)nd.z * rsq_slot_stride + r;
+  out[0] = ss;
+  for (int q = 1; q < parts; ++q) out[(long long)q * pitch] = 0.f;
+}
+
+cudaError_t launch_row_sumsq(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* h, float* rsq,
+                             long long rsq_slot_stride, int parts, int pitch, cudaStream_t st) {
+  if (dm.d % 4) return cudaErrorInvalidValue;
+  return launch_pdl(row_sumsq_kernel, dim3(rows_blocked(Tp) / 32, n), dim3(32), 0, st, nodes, Tp, dm.d, h, rsq,
+                    rsq_slot_stride, parts, pitch);
+}
+
 // ---------------------------------------------------------------------------
 // RMSNorm (gain folded into the next projection): xb = h * rsqrt(mean h^2 + eps)
 // One warp per row.
@@ -196,10 +226,18 @@ cudaError_t launch_rmsnorm(const Dims& dm, const NodeEntry* nodes, int n, int Tp
 // DPFP: r = [relu(q); relu(-q)], phi[(n-1) 2dk + j] = r_j r_{(j-n) mod 2dk}.
 // One warp per row.
 // ---------------------------------------------------------------------------
-template <typename TP>
+// fp32 value rounded to tf32 (10-bit mantissa, round to nearest, ties away):
+// the precision at which the tensor-core read multiplies it.
+__device__ __forceinline__ float round_tf32(float v) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(v));
+  return __uint_as_float(r);
+}
+
+template <bool TF32>
 __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu, int P,
-                                 const float* qm, const float* z_state, TP* phi, float* inv_den,
-                                 float eps, unsigned* err) {
+                                 const float* qm, const float* z_state, float* phi, float* inv_den,
+                                 float eps) {
   grid_dependency_sync();
   extern __shared__ float r_sh[];   // [8 warps][2 dk]
   const NodeEntry nd = nodes[blockIdx.y];
@@ -217,34 +255,32 @@ __global__ void dpfp_read_kernel(const NodeEntry* nodes, int Tp, int dk, int nu,
   __syncwarp();
   const int n2 = 2 * dk;
   const float* z = z_state + (long long)nd.y * P;
-  TP* out = phi + roff * P;
+  float* out = phi + roff * P;
   float dot = 0.f;
-  bool over = false;
   for (int n = 1; n <= nu; ++n) {      // block n: r_j * r_{(j - n) mod 2dk} (nu <= 2 dk)
     for (int j = lane; j < n2; j += 32) {
       const int jj = j - n < 0 ? j - n + n2 : j - n;
       const int p = (n - 1) * n2 + j;
-      const float f = r[j] * r[jj];
-      over |= f > 65504.f;
-      st(out, p, f);
-      dot = fmaf(rounded<TP>(f), z[p], dot);   // the stored (operand-precision) value
+      const float f = TF32 ? round_tf32(r[j] * r[jj]) : r[j] * r[jj];
+      out[p] = f;
+      dot = fmaf(f, z[p], dot);   // the stored (operand-precision) value
     }
   }
   dot = warp_sum(dot);
   if (lane == 0) inv_den[roff] = 1.f / (dot + eps);
-  if (err && __any_sync(0xffffffffu, over) && lane == 0) atomicOr(err, ERR_FP16_RANGE);
 }
 
+// phi [slot][T'][P] fp32; on the tensor-core path (bf16 mode) rounded to tf32,
+// the operand precision of the read product.
 cudaError_t launch_dpfp_read(const Dims& dm, const NodeEntry* nodes, int n, int Tp, const float* qm,
-                             const float* z_state, void* phi, float* inv_den, unsigned* err, cudaStream_t st) {
+                             const float* z_state, float* phi, float* inv_den, cudaStream_t st) {
   dim3 grid((Tp + 7) / 8, n);
   const size_t sh = 8 * 2 * dm.dk * sizeof(float);
   if (dm.bf16)
-    return launch_pdl(dpfp_read_kernel<f16>, grid, dim3(256), sh, st, nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
-                      (f16*)phi, inv_den, dm.mem_eps, err);
-  else
-    dpfp_read_kernel<float><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
-                                                   (float*)phi, inv_den, dm.mem_eps, nullptr);
+    return launch_pdl(dpfp_read_kernel<true>, grid, dim3(256), sh, st, nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state,
+                      phi, inv_den, dm.mem_eps);
+  dpfp_read_kernel<false><<<grid, 256, sh, st>>>(nodes, Tp, dm.dk, dm.nu, dm.P, qm, z_state, phi, inv_den,
+                                                 dm.mem_eps);
   return cudaGetLastError();
 }
 
@@ -414,9 +450,16 @@ __global__ void convert_bf16_as_f16_kernel(const float* src, f16* dst, size_t n)
     dst[i] = __float2half_rn(__bfloat162float(__float2bfloat16_rn(src[i])));
 }
 
+// fp32 -> fp16 (round to nearest even)
+__global__ void convert_f16_kernel(const float* src, f16* dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __float2half_rn(src[i]);
+}
+
 cudaError_t launch_convert(const float* src, void* dst, size_t n, int mode, cudaStream_t st) {
   if (mode == CONVERT_COPY_F32) return cudaMemcpyAsync(dst, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st);
-  convert_bf16_as_f16_kernel<<<1184, 256, 0, st>>>(src, (f16*)dst, n);
+  if (mode == CONVERT_F16) convert_f16_kernel<<<1184, 256, 0, st>>>(src, (f16*)dst, n);
+  else convert_bf16_as_f16_kernel<<<1184, 256, 0, st>>>(src, (f16*)dst, n);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,11 @@
 // outer TMA coordinate, so a tile of node g loads B with coordinate l(g).
 //
 // Operands are 16-bit, both fp16 or both bf16 (a runtime instruction-
-// descriptor field).
+// descriptor field), or both fp32 multiplied at tf32 precision (kind::tf32,
+// a template variant: 32 fp32 words fill the same 128-byte swizzle row as 64
+// 16-bit values, and one K = 8 instruction covers the same 32 bytes as one
+// K = 16 instruction of kind::f16, so the shared-memory layout, descriptors
+// and pipeline are identical).
 //
 // Kernel structure (persistent, one CTA per SM, 320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile BNx64 (16-bit, 128-byte
@@ -318,10 +322,11 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
   }
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool TF32 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const TcGemmParams p) {
+  constexpr int BKE = TF32 ? BK / 2 : BK;   // elements per 128-byte k-block
   using SM = Smem<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -387,10 +392,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           armed &= ~(1u << stage);
           uint8_t* sa = smem + stage * SM::STAGE_BYTES;
-          if (issuer) mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
-          if (issuer) tma_load_3d(&tmA, &full[stage], sa, kb * BK, p.row0 + mb * BM, a_outer);
-          if (issuer) tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BK, nb * BN, nd.y);
-          armed |= 1u << stage;
+          if (!p.debug_no_loads) {
+            if (issuer) mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
+            if (issuer) tma_load_3d(&tmA, &full[stage], sa, kb * BKE, p.row0 + mb * BM, a_outer);
+            if (issuer) tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BKE, nb * BN, nd.y);
+            armed |= 1u << stage;
+          }
           if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
         }
       }
@@ -414,7 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     {
       // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
       const bool issuer = elect_one();
-      const uint32_t IDESC = idesc_f16(BN, p.ab_bf16);
+      const uint32_t IDESC = TF32 ? idesc_tf32(BN) : idesc_f16(BN, p.ab_bf16);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -430,9 +437,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t sa = smem_u32(smem + stage * SM::STAGE_BYTES);
           const uint32_t sb = sa + SM::A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            if (issuer) mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
-                     (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {   // 32 bytes of the k-block per instruction
+            if constexpr (TF32) {
+              if (issuer) mma_tf32(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+                                   (kb > 0 || kk > 0) ? 1u : 0u);
+            } else {
+              if (issuer) mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
+                                  (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           if (issuer) mma_commit(&empty[stage]);
           if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
@@ -709,18 +721,18 @@ PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder() {
 
 namespace {
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool TF32 = false>
 cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, int sm_count,
                           cudaStream_t st) {
   using SM = Smem<BN>;
   const int total = p.n_nodes * p.m_tiles * p.n_tiles;
   const int grid = total < sm_count ? total : sm_count;
-  return launch_pdl(tc_gemm_kernel<BN, EPI>, dim3(grid), dim3(NUM_THREADS), SM::TOTAL, st, ta, tb, p);
+  return launch_pdl(tc_gemm_kernel<BN, EPI, TF32>, dim3(grid), dim3(NUM_THREADS), SM::TOTAL, st, ta, tb, p);
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool TF32 = false>
 cudaError_t configure() {
-  return cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI, TF32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               Smem<BN>::TOTAL);
 }
 
@@ -790,6 +802,10 @@ cudaError_t setup_tc_gemm() {
   if (e == cudaSuccess) e = configure<256, TC_EPI_RESID_ACT>();
   if (e == cudaSuccess) e = configure<256, TC_EPI_QKV_ROPE>();
   if (e == cudaSuccess) e = configure<256, TC_EPI_SWIGLU>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_RESID_ACT, true>();
+  if (e == cudaSuccess) e = configure<256, TC_EPI_F32, true>();
+  if (e == cudaSuccess) e = configure<128, TC_EPI_F32, true>();
+  if (e == cudaSuccess) e = configure<64, TC_EPI_F32, true>();
   if (e == cudaSuccess) e = configure_pair<TC_EPI_F32>();
   if (e == cudaSuccess) e = configure_pair<TC_EPI_RESID>();
   if (e == cudaSuccess) e = configure_pair<TC_EPI_RESID_ACT>();
@@ -799,19 +815,23 @@ cudaError_t setup_tc_gemm() {
   return e;
 }
 
-// 3-D tensor map over a 16-bit array [outer][rows][inner] (inner contiguous;
-// consecutive outer indices pitch_rows rows apart), box = box_inner x
-// box_rows x 1, 128-byte swizzle, zero fill out of bounds.
+// 3-D tensor map over an array [outer][rows][inner] of 16-bit (fp16 / bf16)
+// or fp32 elements (inner contiguous; consecutive outer indices pitch_rows
+// rows apart), box = box_inner x box_rows x 1, 128-byte swizzle, zero fill
+// out of bounds.  ty: 0 = fp16, 1 = bf16, 2 = fp32.
 cudaError_t make_tmap_3d(CUtensorMap* map, const void* base, int inner, int rows, int outer, int box_inner,
-                         int box_rows, int pitch_rows, bool is_bf16) {
+                         int box_rows, int pitch_rows, int ty) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_tensor_map_encoder();
   if (!enc) return cudaErrorNotSupported;
   if (pitch_rows <= 0) pitch_rows = rows;
+  const cuuint64_t esz = ty == 2 ? 4 : 2;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)outer};
-  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)inner * pitch_rows * 2};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * esz, (cuuint64_t)inner * pitch_rows * esz};
   cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, is_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const CUtensorMapDataType dt = ty == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                         : (ty == 1 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
@@ -834,10 +854,34 @@ bool tc_gemm_supported(int m, int n, int k) {
   return k % 8 == 0 && n % 16 == 0 && get_tensor_map_encoder() != nullptr;
 }
 
+namespace {
+
+// fp32 operands on kind::tf32: k-blocks of 32 words; one-CTA kernel only
+cudaError_t launch_tc_gemm_tf32(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
+                                cudaStream_t st) {
+  constexpr int BKE = BK / 2;
+  CUtensorMap ta, tb;
+  cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BKE, BM, op.a_pitch, 2);
+  if (e == cudaSuccess) e = make_tmap_3d(&tb, op.B, p.K, op.b_rows, op.b_outer, BKE, bn, 0, 2);
+  if (e != cudaSuccess) return e;
+  p.k_blocks = (p.K + BKE - 1) / BKE;
+  p.row0 = 0;
+  p.m_tiles = (p.M + BM - 1) / BM;
+  p.n_tiles = (p.N + bn - 1) / bn;
+  if (bn == 256 && epi == TC_EPI_RESID_ACT) return launch_kernel<256, TC_EPI_RESID_ACT, true>(ta, tb, p, sm_count, st);
+  if (bn == 256 && epi == TC_EPI_F32) return launch_kernel<256, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
+  if (bn == 128 && epi == TC_EPI_F32) return launch_kernel<128, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
+  if (bn == 64 && epi == TC_EPI_F32) return launch_kernel<64, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
 int tc_pick_bn(int n) { return n >= 256 ? 256 : (n >= 128 ? 128 : 64); }
 
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st) {
+  if (p.ab_tf32) return launch_tc_gemm_tf32(op, p, epi, bn, sm_count, st);
   CUtensorMap ta, tb;
   cudaError_t e = make_tmap_3d(&ta, op.A, p.K, op.a_rows, op.a_outer, BK, BM, op.a_pitch, p.ab_bf16 != 0);
   if (e != cudaSuccess) return e;
@@ -882,7 +926,8 @@ cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, in
 }
 
 cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
-                                const NodeEntry* nodes, float* C, unsigned* err, int ab_bf16, cudaStream_t st) {
+                                const NodeEntry* nodes, float* C, unsigned* err, int ab, cudaStream_t st,
+                                int debug_no_loads) {
   int dev = 0, sms = 148;
   cudaError_t se = setup_tc_gemm();
   if (se != cudaSuccess) return se;
@@ -895,7 +940,9 @@ cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const
   p.nodes = nodes; p.n_nodes = G; p.M = m; p.N = n; p.K = k;
   p.C = C; p.c_slot_stride = (long long)m * n; p.ldc = n;
   p.err = err;
-  p.ab_bf16 = ab_bf16;
+  p.ab_bf16 = ab == 1;
+  p.ab_tf32 = ab == 2;
+  p.debug_no_loads = debug_no_loads;
   const int bn = tc_pick_bn(n);
   return launch_tc_gemm(op, p, TC_EPI_F32, bn, sms, st);
 }

@@ -22,7 +22,8 @@ struct TcGemmParams {
   int m_tiles, n_tiles, k_blocks;
   int row0;                 // first row of the range this launch covers (rows row0 .. M-1)
   int a_by_layer;           // A's outer TMA coordinate: 0 = node slot, 1 = node layer
-  int ab_bf16;              // operand type: 0 = fp16, 1 = bf16 (both operands alike)
+  int ab_bf16;              // 16-bit operand type: 0 = fp16, 1 = bf16 (both operands alike)
+  int ab_tf32;              // 1: both operands fp32, multiplied at tf32 precision (kind::tf32)
   void* C; long long c_slot_stride; int ldc;
   float* h; long long h_slot_stride; int ldh;   // residual, row-blocked (h_blocked_offset), ldh = row length
   const float* rowscale; long long rs_slot_stride;
@@ -43,11 +44,13 @@ struct TcGemmParams {
   // final hidden states (down-projection epilogue of last-layer nodes)
   void* out; int out_layer; int seg_len;
   unsigned* err;            // device error word (bounded waits)
+  int debug_no_loads;       // test hook: the producer issues no copies, so the first wait for a stage
+                            // cannot complete and the bounded-wait error path runs (never set by the forward)
 };
 
 struct TcGemmOperands {
-  const void* A; int a_rows; int a_outer;   // 16-bit [a_outer][a_rows][K] (rows a_pitch apart per outer step)
-  const void* B; int b_rows; int b_outer;   // 16-bit [b_outer][b_rows][K]
+  const void* A; int a_rows; int a_outer;   // [a_outer][a_rows][K] (rows a_pitch apart per outer step)
+  const void* B; int b_rows; int b_outer;   // [b_outer][b_rows][K]; both 16-bit, or both fp32 (ab_tf32)
   int a_pitch = 0;                          // rows between outer steps of A (0 = a_rows)
 };
 
@@ -57,7 +60,9 @@ bool tc_gemm_pairs_enabled();
 bool tc_gemm_supported(int m, int n, int k);
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st);
+// ab: 0 = fp16, 1 = bf16, 2 = fp32 operands on kind::tf32
 cudaError_t launch_tc_gemm_unit(int G, int m, int n, int k, const void* A, const void* B, int num_b,
-                                const NodeEntry* nodes, float* C, unsigned* err, int ab_bf16, cudaStream_t st);
+                                const NodeEntry* nodes, float* C, unsigned* err, int ab, cudaStream_t st,
+                                int debug_no_loads = 0);
 
 }  // namespace armt

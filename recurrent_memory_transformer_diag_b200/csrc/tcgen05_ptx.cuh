@@ -115,6 +115,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(int n, int ab_bf16, int m = 128
          ((uint32_t)(m >> 4) << 24);
 }
 
+// Instruction descriptor of kind::tf32: D fp32, A/B both tf32 (format 2; the
+// operands are fp32 words in shared memory, read at tf32 precision), both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_tf32(int n, int m = 128) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -125,6 +132,18 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
+      : "memory");
+}
+
+// K = 8 per instruction: 8 fp32 words = 32 bytes of a 128-byte swizzle row,
+// the same byte step as one K = 16 instruction of kind::f16.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
       : "memory");
 }

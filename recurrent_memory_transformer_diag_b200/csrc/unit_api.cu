@@ -21,7 +21,8 @@ armt_status to_status(cudaError_t e) {
 extern "C" armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, int k, const void* A,
                                          const void* B, int num_b, const int* bidx, float* C, void* stream) {
   if (G < 1 || m < 1 || n < 1 || k < 1 || num_b < 1 || !A || !B || !bidx || !C) return ARMT_ERR_INVALID_ARG;
-  if (dtype != ARMT_FP32 && dtype != ARMT_BF16 && dtype != ARMT_F16) return ARMT_ERR_INVALID_ARG;
+  if (dtype != ARMT_FP32 && dtype != ARMT_BF16 && dtype != ARMT_F16 && dtype != ARMT_TF32)
+    return ARMT_ERR_INVALID_ARG;
   std::vector<NodeEntry> tab(G);
   for (int g = 0; g < G; ++g) {
     if (bidx[g] < 0 || bidx[g] >= num_b) return ARMT_ERR_INVALID_ARG;
@@ -38,7 +39,8 @@ extern "C" armt_status armt_grouped_gemm(armt_dtype dtype, int G, int m, int n, 
   if (e == cudaSuccess) e = cudaMemsetAsync(derr, 0, sizeof(unsigned), st);
   if (e == cudaSuccess) {
     if (dtype != ARMT_FP32) {
-      e = launch_tc_gemm_unit(G, m, n, k, A, B, num_b, dnodes, C, derr, dtype == ARMT_BF16 ? 1 : 0, st);
+      e = launch_tc_gemm_unit(G, m, n, k, A, B, num_b, dnodes, C, derr,
+                              dtype == ARMT_BF16 ? 1 : (dtype == ARMT_TF32 ? 2 : 0), st);
     } else {
       GemmArgs g{};
       g.nodes = dnodes; g.n_nodes = G; g.M = m; g.N = n; g.K = k;
@@ -100,9 +102,40 @@ extern "C" armt_status armt_memory_write(int M, int d, int d_key, int nu, float 
     g.epi = EPI_STORE_F32;
     e = launch_simt_gemm(g, st);
   }
-  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, st);
-  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, A, nullptr, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_phi(dm, node, 1, kv, z, phik, gram, coef, gamma, nullptr, st);
+  if (e == cudaSuccess) e = launch_memw_update(dm, node, 1, kv, phik, gram, coef, nullptr, A, st);
   cudaError_t e2 = cudaFreeAsync(scratch, st);
   if (e == cudaSuccess) e = e2;
   return to_status(e);
+}
+
+// The bounded-wait error path of the grouped GEMM, on demand: one 128 x 256
+// tile with K = 1024 (16 k-blocks, more than the pipeline's stages) whose
+// producer is told to issue no copies.  The MMA warp's wait for the first
+// stage then runs out (about one second), it records the timeout in the
+// error word and raises the CTA's abort flag, the producer and epilogue warps
+// leave their waits, every warp reaches the final barrier and TMEM is freed.
+extern "C" armt_status armt_test_bounded_wait(void* stream) {
+  cudaStream_t st = (cudaStream_t)stream;
+  const int m = 128, n = 256, k = 1024;
+  const size_t bytes_a = (size_t)m * k * 2, bytes_b = (size_t)n * k * 2, bytes_c = (size_t)m * n * 4;
+  char* buf = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&buf, bytes_a + bytes_b + bytes_c + 256, st);
+  if (e != cudaSuccess) return to_status(e);
+  NodeEntry* dnode = reinterpret_cast<NodeEntry*>(buf + bytes_a + bytes_b + bytes_c);
+  unsigned* derr = reinterpret_cast<unsigned*>(dnode + 1);
+  unsigned herr = 0;
+  static const NodeEntry one = {0, 0, 0, 0};
+  e = cudaMemsetAsync(buf, 0, bytes_a + bytes_b, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dnode, &one, sizeof(NodeEntry), cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(derr, 0, sizeof(unsigned), st);
+  if (e == cudaSuccess)
+    e = launch_tc_gemm_unit(1, m, n, k, buf, buf + bytes_a, 1, dnode, reinterpret_cast<float*>(buf + bytes_a + bytes_b),
+                            derr, 0, st, /*debug_no_loads=*/1);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&herr, derr, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
+  cudaError_t e2 = cudaStreamSynchronize(st);
+  cudaFreeAsync(buf, st);
+  if (e == cudaSuccess) e = e2;
+  if (e != cudaSuccess) return to_status(e);
+  return (herr & ERR_WAIT_TIMEOUT_MASK) ? ARMT_ERR_DEVICE_TIMEOUT : ARMT_OK;
 }

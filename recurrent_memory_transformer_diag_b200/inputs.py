@@ -34,10 +34,10 @@ import numpy as np
 WEIGHT_SEED = 1234
 EMB_SEED = 5678
 
-# Order fixes each tensor's seed offset; never reorder.
+# Order fixes each tensor's seed offset; never reorder (new tensors go last).
 WEIGHT_NAMES = (
     "mem_emb", "attn_norm", "mlp_norm", "wq", "wk", "wv", "wo",
-    "w_gate", "w_up", "w_down", "wq_mem", "wk_mem", "wv_mem",
+    "w_gate", "w_up", "w_down", "wq_mem", "wk_mem", "wv_mem", "w_beta",
 )
 
 
@@ -59,6 +59,8 @@ class ArmtConfig:
     rope_theta: float = 500000.0
     rms_eps: float = 1e-5
     mem_eps: float = 1e-5
+    write_gate: bool = False     # ARMT variant: row j's write of A scaled by sigmoid(w_beta . m_j)
+    gamma_clamp: bool = True     # ARMT variant: False leaves gamma_j unclamped
 
     @property
     def phi_dim(self) -> int:
@@ -95,6 +97,7 @@ class ArmtConfig:
             "wq_mem": (L, dk, d),
             "wk_mem": (L, dk, d),
             "wv_mem": (L, d, d),
+            **({"w_beta": (L, d)} if self.write_gate else {}),
         }
 
 
@@ -139,6 +142,8 @@ def make_weights(cfg: ArmtConfig, seed: int = WEIGHT_SEED, std: float = 0.02,
     out = {}
     shapes = cfg.weight_shapes()
     for k, name in enumerate(WEIGHT_NAMES):
+        if name not in shapes:
+            continue
         shape = shapes[name]
         if name in ("attn_norm", "mlp_norm"):
             t = torch.ones(*shape, dtype=torch.float32)

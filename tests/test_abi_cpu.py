@@ -42,7 +42,8 @@ def _cfg(**kw):
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("n_layers", 0, 1), ("d_model", -1, 1), ("n_mem", 0, 1), ("max_segments", 0, 1),
+    ("n_layers", 0, 1), ("d_model", -1, 1), ("n_mem", -1, 1), ("max_segments", 0, 1),
+    ("write_gate", 2, 1), ("gamma_unclamped", -1, 1),
     ("n_kv_heads", 3, 1), ("head_dim", 15, 1), ("dtype", 7, 1), ("schedule", 5, 1),
     ("mem_eps", 0.0, 1), ("rope_theta", -1.0, 1), ("dpfp_nu", 40, 1),
     ("head_dim", 48, 7), ("n_mem", 40, 7), ("d_key", 600, 7),
@@ -67,6 +68,7 @@ def test_null_arguments(libarmt):
     idx = (ctypes.c_int * 1)(0)
     assert libarmt.armt_grouped_gemm(1, 0, 8, 16, 16, None, None, 1, idx, None, None) == 1
     assert libarmt.armt_memory_write(0, 8, 2, 1, 1e-5, None, None, None, None, None, None) == 1
+    assert libarmt.armt_forward_ex(None, None, 1, 1, None, None, None, 0, None) == 1
 
 
 def test_bf16_requires_aligned_dims(libarmt):

@@ -82,3 +82,30 @@ def test_memory_write_matches_oracle(M, d, dk, nu):
     torch.cuda.synchronize()
     assert rel_l2(At.cpu().numpy(), Ar) < 1e-5
     assert rel_l2(zt.cpu().numpy(), zr) < 1e-5
+
+
+@pytest.mark.parametrize("G,m,n,k,num_b", [
+    (2, 1040, 2048, 384, 16),   # the memory-read product at the 1B shape (K = P)
+    (3, 144, 256, 96, 2),       # ragged M, K of 3 k-blocks of 32 words
+    (2, 77, 64, 40, 1),         # N = 64 tile, ragged K (1.25 k-blocks)
+    (1, 300, 128, 768, 1),      # N = 128, the 3B P
+])
+def test_tc_grouped_gemm_tf32_matches_fp64(G, m, n, k, num_b):
+    """fp32 operands on kind::tf32: each operand enters at tf32 precision
+    (10-bit mantissa, relative error <= 2^-10 per operand whether rounded or
+    truncated), so a product term is within ~2^-9 and the rel-L2 of the sum of
+    random-sign terms stays well below 2e-3."""
+    import torch
+    from recurrent_memory_transformer_diag_b200 import grouped_gemm
+    g = torch.Generator().manual_seed(G * 7 + m + n + k)
+    A = torch.randn(G, m, k, generator=g)
+    B = torch.randn(num_b, n, k, generator=g) * 0.05
+    bidx = [(2 * i + 1) % num_b for i in range(G)]
+    C = torch.full((G, m, n), float("nan"), device="cuda")
+    grouped_gemm(A.cuda(), B.cuda(), bidx, C, tf32=True)
+    torch.cuda.synchronize()
+    got = C.cpu().numpy()
+    for i in range(G):
+        ref = A[i].double().numpy() @ B[bidx[i]].double().numpy().T
+        err = rel_l2(got[i], ref)
+        assert 0 < err < 2e-3, (i, err)     # > 0: the product really ran at reduced precision

@@ -557,3 +557,16 @@ def test_planted_ignored_initial_state_is_caught(monkeypatch):
     monkeypatch.setattr(ao, "forward", ignores_state)
     monkeypatch.setattr(oracle, "forward", ignores_state)
     assert _fails(lambda: test_streaming_in_two_calls_equals_one_call("tiny", 1))
+
+
+def test_no_memory_tokens_is_the_memoryless_forward():
+    """n_mem = 0: no memory rows are written, so the state stays 0 and every
+    read adds 0; the forward equals the memory=False hook (independent
+    causal decoder forwards per segment) bit for bit."""
+    cfg = CONFIGS["tiny"].with_(n_mem=0, n_segments=3)
+    w = make_weights(cfg)
+    emb = make_embeddings(cfg, 3)
+    a = oracle.forward(cfg, w, emb)
+    b = oracle.forward(cfg, w, emb, memory=False)
+    np.testing.assert_array_equal(a[0], b[0])
+    assert not a[1].any() and not a[2].any()

@@ -3,7 +3,9 @@
 * 1B at S = 18: every diagonal wave in the middle of the run holds the full
   16 nodes, and segments 16 and 17 reuse the activation slots of segments 0
   and 1 (a segment keeps slot s mod min(S, L)), the launch pattern of the
-  131072-token benchmark.
+  131072-token benchmark.  Run twice on the same bf16-valued weights: in fp32
+  mode (SIMT kernels, fp32 arithmetic) and in bf16 mode (the tensor-core
+  path).
 * 3B at S = 4 (head_dim 128).
 * The 1B shape at the two other segment lengths the benchmark sweeps (512 and
   2048 tokens).
@@ -12,8 +14,18 @@
   S = 2.
 
 Every comparison is per segment for the hidden states and per layer for A
-and z, relative L2 error <= 1e-2 (bf16 mode), so one wrong segment cannot
-hide under an average over the others.
+and z, so one wrong segment cannot hide under an average over the others.
+The bar is rel-L2 <= 1e-2 in bf16 mode (1e-5 in fp32 mode), except along a
+long recurrence: there the delta-rule write amplifies the rounding of every
+node's arithmetic from segment to segment, and the error grows about
+linearly with the segment index whatever kernels compute it (an fp64 run of
+the oracle with unbiased relative noise 5e-4 injected into every layer
+output drifts the same way, to 1.6e-2 by segment 17; tests/drift_study.py).
+Measured on the 1B S = 18 run, bf16: 1.9e-3 at segment 0 to 2.2e-2 at 17;
+fp32 mode: 5.5e-6 to 8.4e-5.  The envelope for segment s is the mode's bar
+or c (s + 1), whichever is larger, with c = 1.5e-3 (bf16) and 6e-6 (fp32)
+(the fitted slope with a margin); A and z per layer 5e-2 / 2e-4.  A wrong
+slot, node or state gives errors of order 1, far outside both.
 """
 import numpy as np
 import pytest
@@ -39,26 +51,62 @@ def per_part_errors(cfg, got, ref, S):
     return errs
 
 
-def check(cfg, S, gain_std=0.0, label=""):
-    w = make_weights(cfg, gain_std=gain_std)
-    emb = make_embeddings(cfg, S)
-    ref = oracle.forward(cfg, w, emb)
-    got = run_gpu(cfg, w, emb, S)
-    assert all(np.isfinite(x).all() for x in got)
-    errs = per_part_errors(cfg, got, ref, S)
+def report(label, S, errs):
     seg = {k: v for k, v in errs.items() if k.startswith("hidden")}
     worst_seg = max(seg, key=seg.get)
     worst = max(errs, key=errs.get)
-    print(f"\n{label or cfg.name} S={S}: worst segment {worst_seg} {seg[worst_seg]:.3e}, "
+    print(f"\n{label} S={S}: worst segment {worst_seg} {seg[worst_seg]:.3e}, "
           f"worst overall {worst} {errs[worst]:.3e}")
-    bad = {k: v for k, v in errs.items() if not v <= TOL}
+    print("  per segment: " + " ".join(f"{seg[f'hidden[seg {s}]']:.2e}" for s in range(S)))
+
+
+def check(cfg, S, gain_std=0.0, label="", w=None, emb=None, ref=None, tol=TOL):
+    if w is None:
+        w = make_weights(cfg, gain_std=gain_std)
+    if emb is None:
+        emb = make_embeddings(cfg, S)
+    if ref is None:
+        ref = oracle.forward(cfg, w, emb)
+    got = run_gpu(cfg, w, emb, S)
+    assert all(np.isfinite(x).all() for x in got)
+    errs = per_part_errors(cfg, got, ref, S)
+    report(label or cfg.name, S, errs)
+    bad = {k: v for k, v in errs.items() if not v <= (tol(k) if callable(tol) else tol)}
     assert not bad, bad
     return errs
 
 
-def test_1b_full_waves_and_slot_reuse_match_oracle():
+@pytest.fixture(scope="module")
+def one_b_18():
     cfg = CONFIGS["1b"]
-    check(cfg, 18)
+    S = 18
+    w = make_weights(cfg)
+    emb = make_embeddings(cfg, S)
+    return cfg, S, w, emb, oracle.forward(cfg, w, emb)
+
+
+def drift_envelope(bar, slope, state):
+    """Per-part bound along a long recurrence: hidden segment s within
+    max(bar, slope * (s + 1)); A and z within `state`."""
+    def tol(key):
+        if key.startswith("hidden"):
+            s = int(key.split()[-1].rstrip("]"))
+            return max(bar, slope * (s + 1))
+        return state
+    return tol
+
+
+def test_1b_full_waves_and_slot_reuse_fp32_mode(one_b_18):
+    """Same weights and inputs in fp32 mode (SIMT kernels, fp32 throughout):
+    the schedule, node table and slot reuse of the benchmarked launch."""
+    cfg, S, w, emb, ref = one_b_18
+    check(cfg.with_(dtype="fp32"), S, w=w, emb=emb, ref=ref, tol=drift_envelope(1e-5, 6e-6, 2e-4),
+          label="1b fp32 mode")
+
+
+def test_1b_full_waves_and_slot_reuse_bf16_mode(one_b_18):
+    cfg, S, w, emb, ref = one_b_18
+    check(cfg, S, w=w, emb=emb, ref=ref, tol=drift_envelope(1e-2, 1.5e-3, 5e-2), label="1b bf16 mode")
 
 
 def test_3b_four_segments_match_oracle():
