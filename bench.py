@@ -73,9 +73,9 @@ def kind_bytes(cfg, n_nodes: int, T: int):
     Tp = T + cfg.n_mem
     d, P, M, dk = cfg.d_model, cfg.phi_dim, cfg.n_mem, cfg.d_key
     per = {
-        "memw_update": d * P * (4 + 4 + 2),          # read A, write A, write its fp16 copy
+        "memw_update": d * P * (4 + 4),              # read A, write A (fp32 state)
         "memw_phi": M * P * 4 + P * 8,
-        "dpfp_read": Tp * dk * 4 + Tp * P * 2,
+        "dpfp_read": Tp * dk * 4 + Tp * P * 4,       # q in, phi out (fp32, tf32-rounded)
         "tc_kvmem": (dk + d) * d * 2 + M * d * 2 + M * (dk + d) * 4,   # weight-read bound (M = 16 rows)
     }
     return {k: v * n_nodes for k, v in per.items()}

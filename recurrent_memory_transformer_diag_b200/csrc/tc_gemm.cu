@@ -168,9 +168,12 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
   return rsqrtf(ss / (float)p.norm_dim + p.norm_eps);
 }
 
+// hpre: residual epilogues only, the tile's first 32-column chunk of this
+// thread's row, loaded by the caller before it waited for the accumulator
+// (so that load's latency hides behind the main loop)
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb, int half) {
+                                             bool valid, int nb, int half, const float4* hpre) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
   if constexpr (EPI == TC_EPI_F32) {
@@ -201,7 +204,8 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
     const int c0 = half * NCH;
     auto full_chunk = [&](int c) { return valid && nb * BN + (c + 1) * 32 <= p.N; };
     float4 hn[8];
-    if (full_chunk(c0)) load_h8(Hs, row, nb * BN + c0 * 32, p.ldh, hn);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) hn[q] = hpre[q];
     float ss = 0.f;
 #pragma unroll
     for (int k = 0; k < NCH; ++k) {
@@ -472,6 +476,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int buf = 0;
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = p.row0 + mb * BM + row_in_tile;
+      const bool valid = row < p.M;
+      float4 hpre[8];   // residual epilogues: first chunk of the row, loaded ahead of the wait
+      if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+        const int col = nb * BN + half * (BN / 2);
+        if (valid && col + 32 <= p.N)
+          load_h8(p.h + (long long)nd.z * p.h_slot_stride, row, col, p.ldh, hpre);
+      }
       const bool got = mbar_wait(&tfull[buf], acc_phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -479,13 +494,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
-      const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
-      const NodeEntry nd = p.nodes[node];
-      const int row = p.row0 + mb * BM + row_in_tile;
-      const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half);
+      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hpre);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -676,6 +686,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     int buf = 0;
     uint32_t acc_phase = 0;
     for (int t = cid; t < total; t += ncl) {
+      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
+      const int nb = r / p.m_tiles, mp = r - nb * p.m_tiles;
+      const NodeEntry nd = p.nodes[node];
+      const int row = p.row0 + mp * 256 + (int)rank * BM + row_in_tile;
+      const bool valid = row < p.M;
+      float4 hpre[8];
+      if constexpr (EPI == TC_EPI_RESID || EPI == TC_EPI_RESID_ACT) {
+        const int col = nb * 256 + half * 128;
+        if (valid && col + 32 <= p.N)
+          load_h8(p.h + (long long)nd.z * p.h_slot_stride, row, col, p.ldh, hpre);
+      }
       const bool got = mbar_wait_cluster(&tfull[buf], acc_phase, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) atomicOr(p.err, 4u);
@@ -683,13 +704,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int node = t / tiles_per_node, r = t - node * tiles_per_node;
-      const int nb = r / p.m_tiles, mp = r - nb * p.m_tiles;
-      const NodeEntry nd = p.nodes[node];
-      const int row = p.row0 + mp * 256 + (int)rank * BM + row_in_tile;
-      const bool valid = row < p.M;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
-      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half);
+      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half, hpre);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + (uint32_t)(buf * sizeof(uint64_t)));
