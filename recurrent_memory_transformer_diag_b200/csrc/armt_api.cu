@@ -329,6 +329,20 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
 }
 
+// The memory write of a wave (projection, features, update of A and z) runs on
+// a second stream, so that the next wave's first kernels overlap it: the
+// memory-read query of wave i+1 needs only the layer outputs of wave i; the
+// DPFP read needs z (written by the feature kernel); the read product needs
+// A (written by the update).  The layer-0 input of wave i+1 overwrites a slot
+// whose memory rows wave i's projection reads (wave i holds every slot), so
+// it waits for that projection.  Each wait is an event on the previous wave's
+// write; nothing waits when there is none yet.
+struct WriteOverlap {
+  cudaStream_t s2;
+  cudaEvent_t down, kv, phi, upd;   // recorded after: down GEMM (s1); projection, features, update (s2)
+  bool pending = false;              // a wave's write was enqueued and not yet joined
+};
+
 // Tensor-core path (bf16 mode): the dense products run on the tcgen05 grouped
 // GEMM with fused epilogues, attention on tensor cores.  Weights hold the
 // bf16-rounded values in fp16 containers and the GEMM activations are fp16
@@ -338,7 +352,7 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
 // A itself at tf32 precision (fp16's mantissa, fp32's range), so no copy of
 // A is kept.  Residual stream, accumulation and the memory state are fp32.
 void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
-                     cudaStream_t st, Launcher& L) {
+                     cudaStream_t st, Launcher& L, WriteOverlap* ov = nullptr) {
   const Dims& dm = ctx->dm;
   Workspace& ws = ctx->ws;
   const Weights& w = ctx->w;
@@ -361,11 +375,26 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.rsq = ws.rsq; p.rsq_slot_stride = (long long)Tp * rsq_parts; p.rsq_parts = rsq_parts; p.rsq_pitch = Tp;
     p.norm_dim = dm.d; p.norm_eps = dm.rms_eps;
   };
+  // stream s waits for event e of the previous wave's write (no-op without one)
+  auto after = [&](cudaStream_t s, cudaEvent_t e) {
+    if (ov && ov->pending && !L.dry && L.err == cudaSuccess) {
+      L.err = cudaStreamWaitEvent(s, e, 0);
+      if (L.err != cudaSuccess) L.where = "stream wait";
+    }
+  };
+  auto mark = [&](cudaEvent_t e, cudaStream_t s) {
+    if (ov && !L.dry && L.err == cudaSuccess) {
+      L.err = cudaEventRecord(e, s);
+      if (L.err != cudaSuccess) L.where = "event record";
+    }
+  };
 
-  if (wv.any_first_layer)
+  if (wv.any_first_layer) {
+    if (ov) after(st, ov->kv);
     L("init", [&] {   // only the wave's layer-0 node
       return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st);
     });
+  }
   // no memory tokens: no associative memory.  The QKV epilogue's RMSNorm row
   // scale then needs the layer-0 input's sums of squares, which the memory
   // read's residual epilogue would otherwise have written.
@@ -383,7 +412,9 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.C = ws.qm; p.c_slot_stride = (long long)Tp * dm.dk; p.ldc = dm.dk;
     return launch_tc_gemm(op, p, TC_EPI_F32, tc_pick_bn(dm.dk), sms, st);
   });
+  if (ov) after(st, ov->phi);
   L("dpfp_read", [&] { return launch_dpfp_read(dm, nodes, n, Tp, ws.qm, z, ws.phi, ws.inv_den, st); });
+  if (ov) after(st, ov->upd);
   L("tc_read", [&] {
     // h += phi A^T / (z.phi + eps) on kind::tf32 (phi and A fp32); new h ->
     // fp16 operand copy + norm partials
@@ -444,6 +475,15 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   // rows (rows T..T'-1 of the fp16 copy of the layer output the down GEMM
   // wrote; the RMS row scale comes from the down GEMM's partial sums)
   if (dm.M == 0) return;
+  cudaStream_t cs = st;   // the write's stream
+  if (ov) {
+    mark(ov->down, st);
+    if (!L.dry && L.err == cudaSuccess) {
+      L.err = cudaStreamWaitEvent(ov->s2, ov->down, 0);
+      if (L.err != cudaSuccess) L.where = "stream wait";
+    }
+    cs = ov->s2;
+  }
   L("tc_kvmem", [&] {
     const int ldkv = kv_ld(dm);
     TcGemmOperands op{(const char*)ws.xb + (size_t)T * dm.d * 2, dm.M, slots, w.w_kvm, ldkv, dm.L};
@@ -452,15 +492,27 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.C = ws.kv; p.c_slot_stride = (long long)dm.M * ldkv; p.ldc = ldkv;
     norm_partials(p);
     p.rsq_row0 = T;
-    return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, st);
+    return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, cs);
   });
+  if (ov) mark(ov->kv, cs);
   L("memw_phi", [&] {
-    return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, ws.beta, st);
+    return launch_memw_phi(dm, nodes, n, ws.kv, z, ws.phik, ws.gram, ws.coef, ws.gamma, ws.beta, cs);
   });
+  if (ov) mark(ov->phi, cs);
   L("memw_update", [&] {
-    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, ws.beta, A, st);
+    return launch_memw_update(dm, nodes, n, ws.kv, ws.phik, ws.gram, ws.coef, ws.beta, A, cs);
   });
+  if (ov) {
+    mark(ov->upd, cs);
+    ov->pending = true;
+  }
+}
 
+// Ties the last wave's write back into stream st.
+cudaError_t join_write(WriteOverlap* ov, cudaStream_t st) {
+  if (!ov || !ov->pending) return cudaSuccess;
+  ov->pending = false;
+  return cudaStreamWaitEvent(st, ov->upd, 0);
 }
 
 armt_status ensure_table(armt_ctx* ctx, int S, cudaStream_t st) {
@@ -477,19 +529,44 @@ armt_status ensure_table(armt_ctx* ctx, int S, cudaStream_t st) {
   return ARMT_OK;
 }
 
-// carry_state: A and z already hold the state to start from (else zeroed first)
+// The write overlap of the tensor-core path (streams and events created once).
+WriteOverlap* write_overlap(armt_ctx* ctx) {
+  if (!ctx->ov_stream) {
+    if (cudaStreamCreateWithFlags(&ctx->ov_stream, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      ctx->ov_stream = nullptr;
+      return nullptr;
+    }
+    for (cudaEvent_t* e : {&ctx->ov_ev[0], &ctx->ov_ev[1], &ctx->ov_ev[2], &ctx->ov_ev[3]})
+      if (cudaEventCreateWithFlags(e, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+      }
+  }
+  static thread_local WriteOverlap ov;
+  ov.s2 = ctx->ov_stream;
+  ov.down = ctx->ov_ev[0]; ov.kv = ctx->ov_ev[1]; ov.phi = ctx->ov_ev[2]; ov.upd = ctx->ov_ev[3];
+  ov.pending = false;
+  return &ov;
+}
+
+// carry_state: A and z already hold the state to start from (else zeroed first).
+// overlap: run each wave's memory write on the second stream (tensor-core path;
+// not in the per-kernel profile, whose events time one stream).
 armt_status enqueue_forward(armt_ctx* ctx, const void* emb, int S, int T, void* out, float* A, float* z,
-                            cudaStream_t st, Launcher& L, bool carry_state = false) {
+                            cudaStream_t st, Launcher& L, bool carry_state = false, bool overlap = false) {
   const Dims& dm = ctx->dm;
   if (!L.dry && !carry_state) {
     ARMT_TRY(cudaMemsetAsync(A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), st), "zero A");
     ARMT_TRY(cudaMemsetAsync(z, 0, (size_t)dm.L * dm.P * sizeof(float), st), "zero z");
   }
+  WriteOverlap* ov = (overlap && dm.bf16 && dm.M > 0 && !L.dry && !L.profile) ? write_overlap(ctx) : nullptr;
   for (const Wave& wv : ctx->waves) {
-    if (dm.bf16) enqueue_wave_tc(ctx, wv, T, emb, out, A, z, st, L);
+    if (dm.bf16) enqueue_wave_tc(ctx, wv, T, emb, out, A, z, st, L, ov);
     else enqueue_wave(ctx, wv, T, emb, out, A, z, st, L);
     if (L.err != cudaSuccess) return cuda_fail(ctx, L.err, L.where);
   }
+  ARMT_TRY(join_write(ov, st), "join the memory write");
   return ARMT_OK;
 }
 
@@ -510,7 +587,7 @@ armt_status forward_impl(armt_ctx* ctx, const void* emb, int S, int T, void* out
   if (s != ARMT_OK) return s;
   if (!ctx->use_graph) {
     Launcher L;
-    return enqueue_forward(ctx, emb, S, T, out, A, z, st, L, carry_state);
+    return enqueue_forward(ctx, emb, S, T, out, A, z, st, L, carry_state, ctx->overlap_write);
   }
   armt_ctx::GraphKey key;
   key.S = S; key.T = T; key.sched = (int)ctx->cfg.schedule; key.carry = carry_state ? 1 : 0;
@@ -526,7 +603,8 @@ armt_status forward_impl(armt_ctx* ctx, const void* emb, int S, int T, void* out
     }
     ARMT_TRY(cudaStreamBeginCapture(ctx->capture_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
     Launcher L;
-    armt_status es = enqueue_forward(ctx, emb, S, T, out, A, z, ctx->capture_stream, L, carry_state);
+    armt_status es = enqueue_forward(ctx, emb, S, T, out, A, z, ctx->capture_stream, L, carry_state,
+                                     ctx->overlap_write);
     cudaGraph_t graph = nullptr;
     cudaError_t ce = cudaStreamEndCapture(ctx->capture_stream, &graph);
     if (es != ARMT_OK) {
@@ -579,6 +657,10 @@ extern "C" armt_status armt_create(const armt_config* cfg, armt_ctx** out) {
   if (vs != ARMT_OK) return vs;
   armt_ctx* ctx = new armt_ctx();
   ctx->cfg = *cfg;
+  {
+    const char* v = getenv("ARMT_OVERLAP_WRITE");   // "0": memory write in line (A/B measurement)
+    ctx->overlap_write = !(v && v[0] == '0');
+  }
   Dims& dm = ctx->dm;
   dm.L = cfg->n_layers; dm.d = cfg->d_model; dm.H = cfg->n_heads; dm.KV = cfg->n_kv_heads;
   dm.hd = cfg->head_dim; dm.F = cfg->d_ffn; dm.M = cfg->n_mem; dm.dk = cfg->d_key; dm.nu = cfg->dpfp_nu;
@@ -658,6 +740,9 @@ extern "C" armt_status armt_destroy(armt_ctx* ctx) {
   if (ctx->capture_stream) cudaStreamDestroy(ctx->capture_stream);
   if (ctx->copy_in_stream) cudaStreamDestroy(ctx->copy_in_stream);
   if (ctx->copy_out_stream) cudaStreamDestroy(ctx->copy_out_stream);
+  if (ctx->ov_stream) cudaStreamDestroy(ctx->ov_stream);
+  for (cudaEvent_t ev : ctx->ov_ev)
+    if (ev) cudaEventDestroy(ev);
   for (cudaEvent_t ev : ctx->host_events) cudaEventDestroy(ev);
   free_weights(ctx->w);
   free_workspace(ctx->ws);
@@ -868,10 +953,11 @@ armt_status forward_host_overlapped(armt_ctx* ctx, const void* emb_host, int S, 
     C(cudaMemsetAsync(ctx->st_A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), s1), "zero A");
     C(cudaMemsetAsync(ctx->st_z, 0, (size_t)dm.L * dm.P * sizeof(float), s1), "zero z");
     Launcher L;
+    WriteOverlap* ov = (ctx->overlap_write && dm.bf16 && dm.M > 0) ? write_overlap(ctx) : nullptr;
     for (const Wave& wv : ctx->waves) {
       if (e != cudaSuccess) break;
       if (wv.first_layer_seg >= 0) C(cudaStreamWaitEvent(s1, ev_in[wv.first_layer_seg], 0), "wait emb");
-      if (dm.bf16) enqueue_wave_tc(ctx, wv, T, ctx->st_emb, ctx->st_out, ctx->st_A, ctx->st_z, s1, L);
+      if (dm.bf16) enqueue_wave_tc(ctx, wv, T, ctx->st_emb, ctx->st_out, ctx->st_A, ctx->st_z, s1, L, ov);
       else enqueue_wave(ctx, wv, T, ctx->st_emb, ctx->st_out, ctx->st_A, ctx->st_z, s1, L);
       C(L.err, L.where);
       if (wv.last_layer_seg >= 0) {
@@ -882,6 +968,7 @@ armt_status forward_host_overlapped(armt_ctx* ctx, const void* emb_host, int S, 
                           cudaMemcpyDeviceToHost, s3), "copy out");
       }
     }
+    C(join_write(ov, s1), "join the memory write");
     C(cudaMemcpyAsync(A_host, ctx->st_A, (size_t)dm.L * dm.d * dm.P * 4, cudaMemcpyDeviceToHost, s1), "copy A");
     C(cudaMemcpyAsync(z_host, ctx->st_z, (size_t)dm.L * dm.P * 4, cudaMemcpyDeviceToHost, s1), "copy z");
     C(cudaEventRecord(ev_join_in, s2), "join");

@@ -164,6 +164,11 @@ struct armt_ctx {
   GraphKey host_key;
   cudaStream_t copy_in_stream = nullptr, copy_out_stream = nullptr;
   std::vector<cudaEvent_t> host_events;
+  // each wave's memory write on a second stream, overlapping the next wave's
+  // first kernels (tensor-core path); ARMT_OVERLAP_WRITE=0 turns it off
+  bool overlap_write = true;
+  cudaStream_t ov_stream = nullptr;
+  cudaEvent_t ov_ev[4] = {nullptr, nullptr, nullptr, nullptr};
 };
 
 namespace armt {
