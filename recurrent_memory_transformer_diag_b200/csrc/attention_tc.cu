@@ -8,10 +8,13 @@
 // attention).  Each node attends only over the T' rows of its own segment
 // plus memory tokens, causally.
 //
-// Two softmax warpgroups (A: warps 2..5, B: warps 6..9; one thread per query
+// Two softmax warpgroups (A: warps 4..7, B: warps 8..11; one thread per query
 // row) take the even and the odd query heads of the group, so two heads are
 // in flight and share every K/V tile; each has its own MMA-issuer warp (1 for
-// A, 10 for B).  Per key tile j and warpgroup w:
+// A, 2 for B) in the control warpgroup (warp 0 TMA, warp 3 idle), which hands
+// most of its registers to the softmax warpgroups (setmaxnreg: 232 registers
+// per softmax thread, 40 per control thread; with 168 each, the softmax
+// spilled and ran 7.5 % slower).  Per key tile j and warpgroup w:
 //   MMA  S_w = Q_w K_j^T          (M=128 queries, N=128 keys, K=hd) -> TMEM
 //   softmax: row max, p = exp2(s - m) and its fp32 row sum in registers; P_w
 //            (fp16 pairs) written to TMEM
@@ -45,7 +48,14 @@ using namespace tc;
 
 constexpr int BQ = 128;                 // query rows per tile
 constexpr int BKEY = 128;               // keys per tile
-constexpr int NUM_THREADS = 352;        // warp 0 TMA, warps 1 / 10 MMA for warpgroup A / B, warps 2..9 softmax
+// Warpgroup 0: warp 0 TMA, warps 1 / 2 MMA issue for softmax warpgroup A / B,
+// warp 3 idle; warpgroups 1 and 2 (warps 4..7, 8..11): softmax A and B.  The
+// control warpgroup gives registers to the softmax ones (setmaxnreg): of the
+// 384 x 168 registers the block is launched with, 128 x 40 + 256 x 232; on
+// each SM sub-partition (one control and two softmax warps) 40 + 2 x 232 = 3 x 168.
+constexpr int NUM_THREADS = 384;
+constexpr int CTRL_REGS = 40, SOFTMAX_REGS = 232;
+static_assert(128 * CTRL_REGS + 256 * SOFTMAX_REGS <= NUM_THREADS * 168, "register split");
 constexpr int HALF_BYTES = 128 * 128;   // 128 rows x 64 dims (fp16): one 128-byte-swizzled operand block
 constexpr int TMEM_COLS = 512;
 
@@ -272,6 +282,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     return true;
   };
 
+  if (warp < 4) {
+  // control warpgroup: hands registers to the softmax warpgroups
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(CTRL_REGS));
   if (warp == 0) {
     {
       // ---------------- TMA producer (the whole warp runs the loop; one elected lane issues) ----------------
@@ -378,12 +391,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             while (!mbar_try_wait(&v_full[b], 0) && !mbar_try_wait(&v_full[b], 1) && global_ns() - t0 < WAIT_LIMIT_NS) {}
       }
     }
-  } else if (warp == 1 || warp == 10) {
-    // ---------------- MMA issuers: warp 1 for warpgroup A, warp 10 for B ----------------
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: warp 1 for warpgroup A, warp 2 for B ----------------
     // Each runs the step sequence on the whole warp; one elected lane issues.
     // Two issuers halve the per-step issue chain (waits, descriptors, MMAs);
     // the K/V stages are released by both (count 2).
-    const int w = warp == 1 ? 0 : 1;
+    const int w = warp - 1;
     const bool issuer = elect_one();
     const uint32_t idesc_s = idesc_f16(BKEY, 0);   // 128 x 128 x 16
     const uint32_t idesc_o = idesc_f16(HD, 0);     // 128 x hd x 16
@@ -487,9 +500,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     while (!mbar_try_wait(&drain[w], 0)) {
       if (global_ns() - t0 > WAIT_LIMIT_NS) break;
     }
+  }   // warp 3: nothing to do
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(SOFTMAX_REGS));
     // ---------------- softmax (warpgroup w, one thread per query row) ----------------
-    const int w = (warp - 2) >> 2;
+    const int w = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int rloc = quarter * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
