@@ -4,7 +4,7 @@ Not collected by pytest (the oracle needs about an hour of host time for the
 128 segments).  Three steps, each writing an .npz:
 
     python tests/long_drift.py oracle  --out ORACLE.npz          # host, fp64 oracle
-    python tests/long_drift.py gpu     --out GPU.npz [--dtype bf16|fp32]   # B200, the library
+    python tests/long_drift.py gpu     --out GPU.npz [--dtype bf16|fp32] [--ref ORACLE.npz]   # B200
     python tests/long_drift.py compare ORACLE.npz GPU.npz [GPU2.npz ...]
 
 Both sides use the seeded inputs of the 131072-token workload (128 segments
@@ -64,7 +64,7 @@ def run_oracle(out, S):
             np.savez(out, rows=rows[:s + 1], A=A.astype(np.float32), z=z.astype(np.float32), segments=s + 1)
 
 
-def run_gpu(out, S, dtype):
+def run_gpu(out, S, dtype, ref=None):
     import torch
     from recurrent_memory_transformer_diag_b200 import Armt
     from recurrent_memory_transformer_diag_b200.inputs import make_embeddings, make_weights
@@ -91,6 +91,11 @@ def run_gpu(out, S, dtype):
     np.savez(out, rows=rows, A=A_keep.cpu().numpy(), z=z.cpu().numpy(), segments=S, seconds=secs)
     m.close()
     print(f"{dtype}: {S} segments in {secs:.2f} s -> {out}")
+    if ref:   # compare right here and keep only the small summary
+        summary = compare(ref, [out])
+        os.remove(out)
+        with open(out.replace(".npz", ".json"), "w") as f:
+            json.dump(summary, f)
 
 
 def rel(a, b):
@@ -121,6 +126,7 @@ def compare(ref_path, paths):
     print(json.dumps({k: {"worst_segment": max(v["hidden_per_segment"]),
                           "worst_A": max(v.get("A_per_layer", [0])),
                           "worst_z": max(v.get("z_per_layer", [0]))} for k, v in out.items()}))
+    return out
 
 
 def main():
@@ -130,11 +136,12 @@ def main():
     ap.add_argument("--out")
     ap.add_argument("--segments", type=int, default=128)
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "fp32"])
+    ap.add_argument("--ref", default=None, help="gpu: oracle .npz to compare with on the spot")
     a = ap.parse_args()
     if a.mode == "oracle":
         run_oracle(a.out, a.segments)
     elif a.mode == "gpu":
-        run_gpu(a.out, a.segments, a.dtype)
+        run_gpu(a.out, a.segments, a.dtype, a.ref)
     else:
         compare(a.paths[0], a.paths[1:])
 
