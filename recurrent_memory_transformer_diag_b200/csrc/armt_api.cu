@@ -329,6 +329,18 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
 }
 
+// Column tile of the memory-write projection (16 rows per node, weight-read
+// bound: narrower tiles put more CTAs, so more weight loads, in flight);
+// ARMT_KVMEM_BN selects 64 / 128 / 256 for measurement.
+int kvmem_bn() {
+  static const int bn = [] {
+    const char* v = getenv("ARMT_KVMEM_BN");
+    const int b = v ? atoi(v) : 256;
+    return (b == 64 || b == 128) ? b : 256;
+  }();
+  return bn;
+}
+
 // The memory write of a wave (projection, features, update of A and z) runs on
 // a second stream, so that the next wave's first kernels overlap it: the
 // memory-read query of wave i+1 needs only the layer outputs of wave i; the
@@ -492,7 +504,7 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     p.C = ws.kv; p.c_slot_stride = (long long)dm.M * ldkv; p.ldc = ldkv;
     norm_partials(p);
     p.rsq_row0 = T;
-    return launch_tc_gemm(op, p, TC_EPI_F32, 256, sms, cs);
+    return launch_tc_gemm(op, p, TC_EPI_F32, kvmem_bn(), sms, cs);
   });
   if (ov) mark(ov->kv, cs);
   L("memw_phi", [&] {
