@@ -84,14 +84,24 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
     __syncwarp();
   }
   __syncthreads();   // phi rows visible block-wide
-  for (int pair = warp; pair < M * M; pair += nw) {
-    const int a = pair / M, b = pair - a * M;
-    if (b < a) continue;
+  // Gram matrix: the M (M + 1) / 2 pairs a <= b, dealt to the warps; each dot
+  // product keeps four partial sums (a short dependency chain)
+  for (int q = warp; q < M * (M + 1) / 2; q += nw) {
+    int a = 0, rest = q;
+    while (rest >= M - a) { rest -= M - a; ++a; }
+    const int b = a + rest;
     const float* pa = phs + a * P;
     const float* pb = phs + b * P;
-    float g = 0.f;
-    for (int p = lane; p < P; p += 32) g = fmaf(pa[p], pb[p], g);
-    g = warp_sum_m(g);
+    float g0 = 0.f, g1 = 0.f, g2 = 0.f, g3 = 0.f;
+    int p = lane;
+    for (; p + 96 < P; p += 128) {
+      g0 = fmaf(pa[p], pb[p], g0);
+      g1 = fmaf(pa[p + 32], pb[p + 32], g1);
+      g2 = fmaf(pa[p + 64], pb[p + 64], g2);
+      g3 = fmaf(pa[p + 96], pb[p + 96], g3);
+    }
+    for (; p < P; p += 32) g0 = fmaf(pa[p], pb[p], g0);
+    const float g = warp_sum_m((g0 + g1) + (g2 + g3));
     if (lane == 0) {
       G[a * M + b] = g;
       G[b * M + a] = g;
@@ -101,26 +111,43 @@ __global__ void memw_phi_kernel(const NodeEntry* nodes, int M, int dk, int d, in
   if (warp == 0) {
     // z_j . phi_j = z_0 . phi_j + sum_{j'<j} gamma_j' G[j'][j]: lane j (< M <= 32)
     // carries row j; at step j lane j's value is final, gamma_j is broadcast
-    // and the later lanes add its term
+    // and the later lanes add its term.  Lane j's denominator |phi_j|^2 + eps
+    // and its column of G are read once, before the steps.
+    const int jl = lane < M ? lane : 0;
+    const float den = G[jl * (M + 1)] + eps;
+    float gcol[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) gcol[j] = (j < M) ? G[j * M + jl] : 0.f;
     float zp = lane < M ? zp0[lane] : 0.f;
-    for (int j = 0; j < M; ++j) {
-      const float g_raw = 1.f - zp / (G[(lane < M ? lane : 0) * (M + 1)] + eps);
-      const float gm_l = clamp_gamma ? fminf(fmaxf(g_raw, 0.f), 1.f) : g_raw;
-      const float gm = __shfl_sync(0xffffffffu, gm_l, j);
-      if (lane == j) {
-        gam[j] = gm;
-        coef[(long long)slot * M + j] = 1.f / (zp + eps);
-        gamma[(long long)slot * M + j] = gm;
+    float gm_own = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j < M) {
+        const float g_raw = 1.f - zp / den;
+        const float gm_l = clamp_gamma ? fminf(fmaxf(g_raw, 0.f), 1.f) : g_raw;
+        const float gm = __shfl_sync(0xffffffffu, gm_l, j);
+        if (lane == j) gm_own = gm;
+        if (lane > j) zp = fmaf(gm, gcol[j], zp);
       }
-      if (lane > j && lane < M) zp = fmaf(gm, G[j * M + lane], zp);
+    }
+    // zp is lane j's final z_j . phi_j (no step after j changes it)
+    if (lane < M) {
+      gam[lane] = gm_own;
+      coef[(long long)slot * M + lane] = 1.f / (zp + eps);
+      gamma[(long long)slot * M + lane] = gm_own;
     }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < M * M; e += blockDim.x) gram[(long long)slot * M * M + e] = G[e];
   for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    float acc = zs[p];
-    for (int j = 0; j < M; ++j) acc = fmaf(gam[j], phs[j * P + p], acc);
-    z[p] = acc;
+    float a0 = zs[p], a1 = 0.f;
+    int j = 0;
+    for (; j + 1 < M; j += 2) {
+      a0 = fmaf(gam[j], phs[j * P + p], a0);
+      a1 = fmaf(gam[j + 1], phs[(j + 1) * P + p], a1);
+    }
+    if (j < M) a0 = fmaf(gam[j], phs[j * P + p], a0);
+    z[p] = a0 + a1;
   }
 }
 
@@ -500,11 +527,11 @@ cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, co
 #define ARMT_MEMWV_CASE(C, MT)                                                                                      \
   {                                                                                                                 \
     if (pf)                                                                                                         \
-      e = launch_pdl(memw_update_vec_kernel<C, MT, true>, grid, dim3(256), sh_pf, st, nodes, dm.M, dm.dk, dm.d,   \
-                     dm.P, ldkv, kv, phik, gram, coef, beta, A_state);                                              \
+      e = launch_pdl(memw_update_vec_kernel<C, MT, true>, grid, dim3(256), sh_pf, st, nodes, dm.M, dm.dk,     \
+                     dm.d, dm.P, ldkv, kv, phik, gram, coef, beta, A_state);                                        \
     else                                                                                                            \
-      e = launch_pdl(memw_update_vec_kernel<C, MT, false>, grid, dim3(256), sh, st, nodes, dm.M, dm.dk, dm.d, dm.P, \
-                     ldkv, kv, phik, gram, coef, beta, A_state);                                                    \
+      e = launch_pdl(memw_update_vec_kernel<C, MT, false>, grid, dim3(256), sh, st, nodes, dm.M, dm.dk, dm.d,   \
+                     dm.P, ldkv, kv, phik, gram, coef, beta, A_state);                                              \
   }
 #define ARMT_MEMWV_M(C)                  \
   {                                      \
