@@ -88,9 +88,10 @@ struct AttnShape {
 };
 constexpr float RESCALE_THRESHOLD = 8.f;
 // Share of the exponentials taken off the MUFU unit (every POLY_EVERY-th
-// pair by polynomial; 0 = none).  A quarter measured 3 % faster than none on
-// the 1B wave (the softmax is mostly issue-bound, so more would cost).
-constexpr int POLY_EVERY = 4;
+// pair by polynomial; 0 = none).  An eighth measured fastest on the 1B wave,
+// about 3 % ahead of none and 5 % ahead of a quarter (the softmax is mostly
+// issue-bound, so a larger share costs more FMA issue than it saves).
+constexpr int POLY_EVERY = 8;
 
 struct AttnParams {
   const NodeEntry* nodes;
