@@ -27,6 +27,15 @@
 // Two TMEM accumulators (2 x BN columns) let the epilogue of tile t overlap
 // the main loop of tile t+1.  Tiles never straddle nodes: a node's rows are
 // the middle TMA coordinate with extent M, rows past M read as zeros.
+//
+// Ragged last row tile (swap_tail).  When a node's last row tile holds at
+// most SWAP_ROWS rows (1040 = 8 x 128 + 16 at 1B), it is computed transposed:
+// D^T = B_tile A_rows^T with the weight rows as the 128-row operand and the
+// SWAP_ROWS activation rows as N, one M = 128, N = SWAP_ROWS instruction per
+// 128 weight rows and K step, instead of a 128 x BN product of which 7/8 are
+// padding.  The epilogue warps move D^T through shared memory (a row per
+// activation row) and the warps of TMEM quarter 0 run the ordinary epilogue
+// on those rows.
 // Every mbarrier wait is bounded (about one second); on timeout the kernel
 // sets the device error word, drains its own outstanding copies and MMAs,
 // frees TMEM and returns.
@@ -49,6 +58,7 @@ constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
 constexpr int EPI_WARPS = 8;           // two warps per TMEM lane quarter, each half of the columns
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
+constexpr int SWAP_ROWS = 32;          // transposed ragged tile: rows (= MMA N) it covers
 
 __device__ __forceinline__ void store_f16x32(f16* dst, const float* v) {
   // 32 values = 64 bytes: four 16-byte stores (dst 16-byte aligned)
@@ -72,7 +82,16 @@ struct Smem {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN >= 256 ? 4 : (BN >= 128 ? 6 : 8);
   static constexpr int BAR_OFFSET = STAGES * STAGE_BYTES;
-  static constexpr int TOTAL = BAR_OFFSET + 256 + 1024;   // + barriers + alignment slack
+  // transposed ragged tile (BN a multiple of 128): A box of SWAP_ROWS rows and
+  // the staging area of D^T, one row of BN (+4 against bank conflicts) fp32
+  // per activation row
+  static constexpr bool SWAP = BN % 128 == 0;
+  static constexpr int SWAP_A_BYTES = SWAP_ROWS * BK * 2;
+  static constexpr int STG_PITCH = BN + 4;
+  static constexpr int STG_OFFSET = BAR_OFFSET + 256;
+  static constexpr int STG_BYTES = SWAP ? SWAP_ROWS * STG_PITCH * 4 : 0;
+  static constexpr int TOTAL = STG_OFFSET + STG_BYTES + 1024;   // + barriers, staging, alignment slack
+  static_assert(TOTAL + 64 <= 227 * 1024, "shared memory per CTA");
 };
 
 __device__ __forceinline__ void store_f32x32(float* dst, const float* v, int valid_cols) {
@@ -160,6 +179,22 @@ __device__ __forceinline__ void load_h8(const float* Hs, int row, int col, int d
 // Epilogue of one accumulator tile for this thread's row.  Every tcgen05.ld
 // is executed by the whole warp (warp-uniform loops); only the stores are
 // guarded by the row/column bounds.
+// 32 consecutive accumulator columns (col .. col+31) of this thread's row:
+// from TMEM (warp-collective), or, for the transposed ragged tile, from the
+// thread's row of the shared-memory staging area.
+__device__ __forceinline__ void acc_ld32(uint32_t tbase, const float* srow, int col, float* v) {
+  if (srow) {
+    const float4* s4 = reinterpret_cast<const float4*>(srow + col);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 x = s4[q];
+      v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+    }
+  } else {
+    tmem_ld32(tbase + (uint32_t)col, v);
+  }
+}
+
 // RMSNorm row scale from the per-tile partial sums of squares.
 __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot, int row) {
   const float* part = p.rsq + (long long)slot * p.rsq_slot_stride + row;
@@ -170,10 +205,12 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
 
 // hpre: residual epilogues only, the tile's first 32-column chunk of this
 // thread's row, loaded by the caller before it waited for the accumulator
-// (so that load's latency hides behind the main loop)
+// (so that load's latency hides behind the main loop).  srow: null, or this
+// row of the transposed ragged tile's staging area (then tbase is unused).
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
-                                             bool valid, int nb, int half, const float4* hpre) {
+                                             bool valid, int nb, int half, const float4* hpre,
+                                             const float* srow) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
   if constexpr (EPI == TC_EPI_F32) {
@@ -182,7 +219,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
 #pragma unroll 1
     for (int c = half * (BN / 64); c < (half + 1) * (BN / 64); ++c) {
       float v[32];
-      tmem_ld32(tbase + c * 32, v);
+      acc_ld32(tbase, srow, c * 32, v);
       const int col = nb * BN + c * 32;
       if (!valid || col >= p.N) continue;
       float* C = reinterpret_cast<float*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
@@ -215,7 +252,7 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       for (int q = 0; q < 8; ++q) hc[q] = hn[q];
       if (k + 1 < NCH && full_chunk(c + 1)) load_h8(Hs, row, nb * BN + (c + 1) * 32, p.ldh, hn);
       float v[32];
-      tmem_ld32(tbase + c * 32, v);
+      acc_ld32(tbase, srow, c * 32, v);
       const int col = nb * BN + c * 32;
       if (!valid || col >= p.N) continue;
       const int nv = p.N - col;
@@ -264,8 +301,8 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       for (int pc = 0; pc < pairs; ++pc) {
         const int c1 = hh * cph + pc, c2 = c1 + pairs;
         float v1[32], v2[32];
-        tmem_ld32(tbase + c1 * 32, v1);
-        tmem_ld32(tbase + c2 * 32, v2);
+        acc_ld32(tbase, srow, c1 * 32, v1);
+        acc_ld32(tbase, srow, c2 * 32, v2);
         const int col1 = nb * BN + c1 * 32, col2 = nb * BN + c2 * 32;
         if (!valid || col1 >= p.N) continue;
         if (rot) {
@@ -311,8 +348,8 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
 #pragma unroll 1
     for (int c = half * (HALF / 64); c < (half + 1) * (HALF / 64); ++c) {
       float g[32], u[32];
-      tmem_ld32(tbase + c * 32, g);
-      tmem_ld32(tbase + HALF + c * 32, u);
+      acc_ld32(tbase, srow, c * 32, g);
+      acc_ld32(tbase, srow, HALF + c * 32, u);
       const int f = f0 + c * 32;
       if (!valid || f >= p.f_out) continue;
 #pragma unroll
@@ -329,7 +366,8 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
 template <int BN, int EPI, bool TF32 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const TcGemmParams p) {
+                   const __grid_constant__ CUtensorMap tmAs, const TcGemmParams p) {
+  // tmAs: A with a SWAP_ROWS-row box (transposed ragged tile; unused otherwise)
   constexpr int BKE = TF32 ? BK / 2 : BK;   // elements per 128-byte k-block
   using SM = Smem<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -339,7 +377,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tfull = empty + SM::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* stg_full = drain + 1;    // transposed ragged tile: D^T staged (all epilogue threads arrive)
+  uint64_t* stg_empty = drain + 2;   // ... and read (the 64 threads of TMEM quarter 0 arrive)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   grid_dependency_sync();
@@ -362,6 +402,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(&tempty[b], EPI_WARPS);
     }
     mbar_init(drain, 1);
+    mbar_init(stg_full, 32 * EPI_WARPS);
+    mbar_init(stg_empty, 64);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -392,13 +434,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
         const NodeEntry nd = p.nodes[node];
         const int a_outer = p.a_by_layer ? nd.y : nd.z;
+        const bool swapped = SM::SWAP && p.swap_tail && mb == p.m_tiles - 1;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
           armed &= ~(1u << stage);
           uint8_t* sa = smem + stage * SM::STAGE_BYTES;
           if (!p.debug_no_loads) {
-            if (issuer) mbar_expect_tx(&full[stage], SM::STAGE_BYTES);
-            if (issuer) tma_load_3d(&tmA, &full[stage], sa, kb * BKE, p.row0 + mb * BM, a_outer);
+            if (issuer) mbar_expect_tx(&full[stage], swapped ? SM::SWAP_A_BYTES + SM::B_BYTES : SM::STAGE_BYTES);
+            if (issuer)
+              tma_load_3d(swapped ? &tmAs : &tmA, &full[stage], sa, kb * BKE, p.row0 + mb * BM, a_outer);
             if (issuer) tma_load_3d(&tmB, &full[stage], sa + SM::A_BYTES, kb * BKE, nb * BN, nd.y);
             armed |= 1u << stage;
           }
@@ -426,12 +470,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
       const bool issuer = elect_one();
       const uint32_t IDESC = TF32 ? idesc_tf32(BN) : idesc_f16(BN, p.ab_bf16);
+      // transposed ragged tile: M = 128 weight rows, N = SWAP_ROWS activation rows
+      const uint32_t IDESC_SW = TF32 ? idesc_tf32(SWAP_ROWS) : idesc_f16(SWAP_ROWS, p.ab_bf16);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const int mb = (t % tiles_per_node) % p.m_tiles;
+        const bool swapped = SM::SWAP && p.swap_tail && mb == p.m_tiles - 1;
         if (!mbar_wait_warp(&tempty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
@@ -440,6 +488,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * SM::STAGE_BYTES);
           const uint32_t sb = sa + SM::A_BYTES;
+          if (swapped) {
+            // D^T[128 j + f][r] (TMEM columns j SWAP_ROWS + r) = B rows 128 j + f times A rows r
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j) {
+                const uint32_t dj = d_tmem + (uint32_t)(j * SWAP_ROWS);
+                const uint64_t wdesc = sw128_desc(sb + j * 128 * 128 + kk * 32);
+                const uint64_t xdesc = sw128_desc(sa + kk * 32);
+                if constexpr (TF32) {
+                  if (issuer) mma_tf32(dj, wdesc, xdesc, IDESC_SW, (kb > 0 || kk > 0) ? 1u : 0u);
+                } else {
+                  if (issuer) mma_f16(dj, wdesc, xdesc, IDESC_SW, (kb > 0 || kk > 0) ? 1u : 0u);
+                }
+              }
+            }
+          } else {
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {   // 32 bytes of the k-block per instruction
             if constexpr (TF32) {
@@ -449,6 +514,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (issuer) mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32), IDESC,
                                   (kb > 0 || kk > 0) ? 1u : 0u);
             }
+          }
           }
           if (issuer) mma_commit(&empty[stage]);
           if (++stage == SM::STAGES) { stage = 0; phase ^= 1; }
@@ -475,9 +541,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int row_in_tile = quarter * 32 + lane;
     int buf = 0;
     uint32_t acc_phase = 0;
+    uint32_t stg_phase = 0;   // transposed ragged tiles seen so far, mod 2
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const int node = t / tiles_per_node, r = t - node * tiles_per_node;
       const int nb = r / p.m_tiles, mb = r - nb * p.m_tiles;
+      const bool swapped = SM::SWAP && p.swap_tail && mb == p.m_tiles - 1;
       const NodeEntry nd = p.nodes[node];
       const int row = p.row0 + mb * BM + row_in_tile;
       const bool valid = row < p.M;
@@ -495,10 +563,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hpre);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[buf]);
+      if (swapped) {
+        if constexpr (SM::SWAP) {
+          // D^T: this warp's TMEM lanes are weight rows 128 half + 32 quarter + lane of the
+          // tile, its columns half * SWAP_ROWS .. the activation rows; staged as
+          // stg[row][column] once the previous transposed tile's rows have been read
+          float* stg = reinterpret_cast<float*>(smem + SM::STG_OFFSET);
+          if (!__all_sync(0xffffffffu, mbar_wait(stg_empty, stg_phase ^ 1, abort_flag))) {
+            if (lane == 0) atomicOr(p.err, 4u);
+            *abort_flag = 1;
+            break;
+          }
+          if (half < BN / 128) {
+            float v[32];
+            tmem_ld32(tbase + (uint32_t)(half * SWAP_ROWS), v);
+            const int col = half * 128 + quarter * 32 + lane;
+#pragma unroll
+            for (int i = 0; i < SWAP_ROWS; ++i) stg[i * SM::STG_PITCH + col] = v[i];
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[buf]);   // TMEM buffer free for the next tile
+          mbar_arrive(stg_full);
+          if (quarter == 0) {
+            if (!__all_sync(0xffffffffu, mbar_wait(stg_full, stg_phase, abort_flag))) {
+              if (lane == 0) atomicOr(p.err, 4u);
+              *abort_flag = 1;
+              break;
+            }
+            run_epilogue<BN, EPI>(p, 0u, nd, row, valid, nb, half, hpre, stg + lane * SM::STG_PITCH);
+            mbar_arrive(stg_empty);
+          }
+          stg_phase ^= 1;
+        }
+      } else {
+        run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[buf]);
+      }
       if (++buf == 2) { buf = 0; acc_phase ^= 1; }
     }
   }
@@ -705,7 +808,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
-      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half, hpre);
+      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + (uint32_t)(buf * sizeof(uint64_t)));
@@ -738,12 +841,12 @@ PFN_cuTensorMapEncodeTiled_v12000 get_tensor_map_encoder() {
 namespace {
 
 template <int BN, int EPI, bool TF32 = false>
-cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const TcGemmParams& p, int sm_count,
-                          cudaStream_t st) {
+cudaError_t launch_kernel(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tas,
+                          const TcGemmParams& p, int sm_count, cudaStream_t st) {
   using SM = Smem<BN>;
   const int total = p.n_nodes * p.m_tiles * p.n_tiles;
   const int grid = total < sm_count ? total : sm_count;
-  return launch_pdl(tc_gemm_kernel<BN, EPI, TF32>, dim3(grid), dim3(NUM_THREADS), SM::TOTAL, st, ta, tb, p);
+  return launch_pdl(tc_gemm_kernel<BN, EPI, TF32>, dim3(grid), dim3(NUM_THREADS), SM::TOTAL, st, ta, tb, tas, p);
 }
 
 template <int BN, int EPI, bool TF32 = false>
@@ -865,12 +968,35 @@ bool tc_gemm_pairs_enabled() {
   return on;
 }
 
+// The transposed ragged row tile is on unless the environment sets
+// ARMT_GEMM_SWAP_TAIL=0 (for A/B measurement).
+bool tc_gemm_swap_enabled() {
+  static const bool on = [] {
+    const char* v = getenv("ARMT_GEMM_SWAP_TAIL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
+}
+
 bool tc_gemm_supported(int m, int n, int k) {
   (void)m;
   return k % 8 == 0 && n % 16 == 0 && get_tensor_map_encoder() != nullptr;
 }
 
 namespace {
+
+// Decide whether the last row tile runs transposed and, if so, build the A
+// map with a SWAP_ROWS-row box (otherwise tas is a copy of ta, never read).
+cudaError_t setup_swap_tail(const TcGemmOperands& op, TcGemmParams& p, int bn, int box_inner, int ty,
+                            const CUtensorMap& ta, CUtensorMap* tas) {
+  const int last_rows = p.M - p.row0 - (p.m_tiles - 1) * BM;
+  p.swap_tail = (bn % 128 == 0 && last_rows <= SWAP_ROWS && tc_gemm_swap_enabled()) ? 1 : 0;
+  if (!p.swap_tail) {
+    *tas = ta;
+    return cudaSuccess;
+  }
+  return make_tmap_3d(tas, op.A, p.K, op.a_rows, op.a_outer, box_inner, SWAP_ROWS, op.a_pitch, ty);
+}
 
 // fp32 operands on kind::tf32: k-blocks of 32 words; one-CTA kernel only
 cudaError_t launch_tc_gemm_tf32(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
@@ -884,10 +1010,14 @@ cudaError_t launch_tc_gemm_tf32(const TcGemmOperands& op, TcGemmParams p, int ep
   p.row0 = 0;
   p.m_tiles = (p.M + BM - 1) / BM;
   p.n_tiles = (p.N + bn - 1) / bn;
-  if (bn == 256 && epi == TC_EPI_RESID_ACT) return launch_kernel<256, TC_EPI_RESID_ACT, true>(ta, tb, p, sm_count, st);
-  if (bn == 256 && epi == TC_EPI_F32) return launch_kernel<256, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
-  if (bn == 128 && epi == TC_EPI_F32) return launch_kernel<128, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
-  if (bn == 64 && epi == TC_EPI_F32) return launch_kernel<64, TC_EPI_F32, true>(ta, tb, p, sm_count, st);
+  CUtensorMap tas;
+  e = setup_swap_tail(op, p, bn, BKE, 2, ta, &tas);
+  if (e != cudaSuccess) return e;
+  if (bn == 256 && epi == TC_EPI_RESID_ACT)
+    return launch_kernel<256, TC_EPI_RESID_ACT, true>(ta, tb, tas, p, sm_count, st);
+  if (bn == 256 && epi == TC_EPI_F32) return launch_kernel<256, TC_EPI_F32, true>(ta, tb, tas, p, sm_count, st);
+  if (bn == 128 && epi == TC_EPI_F32) return launch_kernel<128, TC_EPI_F32, true>(ta, tb, tas, p, sm_count, st);
+  if (bn == 64 && epi == TC_EPI_F32) return launch_kernel<64, TC_EPI_F32, true>(ta, tb, tas, p, sm_count, st);
   return cudaErrorInvalidValue;
 }
 
@@ -928,8 +1058,11 @@ cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, in
   if (e != cudaSuccess) return e;
   p.m_tiles = (p.M - p.row0 + BM - 1) / BM;
   p.n_tiles = (p.N + bn - 1) / bn;
+  CUtensorMap tas;
+  e = setup_swap_tail(op, p, bn, BK, p.ab_bf16 != 0, ta, &tas);
+  if (e != cudaSuccess) return e;
 #define ARMT_TC_CASE(BNV, E) \
-  if (bn == BNV && epi == E) return launch_kernel<BNV, E>(ta, tb, p, sm_count, st);
+  if (bn == BNV && epi == E) return launch_kernel<BNV, E>(ta, tb, tas, p, sm_count, st);
   ARMT_TC_CASE(256, TC_EPI_F32)
   ARMT_TC_CASE(128, TC_EPI_F32)
   ARMT_TC_CASE(64, TC_EPI_F32)

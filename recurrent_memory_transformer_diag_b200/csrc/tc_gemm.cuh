@@ -44,6 +44,7 @@ struct TcGemmParams {
   // final hidden states (down-projection epilogue of last-layer nodes)
   void* out; int out_layer; int seg_len;
   unsigned* err;            // device error word (bounded waits)
+  int swap_tail;            // 1: the last row tile (at most 32 rows) is computed transposed (set by the launcher)
   int debug_no_loads;       // test hook: the producer issues no copies, so the first wait for a stage
                             // cannot complete and the bounded-wait error path runs (never set by the forward)
 };
@@ -57,6 +58,7 @@ struct TcGemmOperands {
 cudaError_t setup_tc_gemm();
 int tc_pick_bn(int n);
 bool tc_gemm_pairs_enabled();
+bool tc_gemm_swap_enabled();
 bool tc_gemm_supported(int m, int n, int k);
 cudaError_t launch_tc_gemm(const TcGemmOperands& op, TcGemmParams p, int epi, int bn, int sm_count,
                            cudaStream_t st);

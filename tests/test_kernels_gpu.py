@@ -19,6 +19,12 @@ pytestmark = pytest.mark.gpu
     (16, 1040, 3072, 2048, 16), # a full 1B wave of QKV shapes
     (2, 512, 256, 128, 2),      # rows in whole 256-row CTA-pair tiles only
     (1, 300, 304, 200, 1),      # one pair tile + a 44-row one-CTA rest, ragged N and K
+    # transposed ragged row tile (last tile of <= 32 rows, N a multiple of 128):
+    (2, 150, 128, 256, 2),      # N = 128 tile, 22-row tail
+    (1, 129, 256, 128, 1),      # a 1-row tail
+    (2, 32, 256, 64, 1),        # a node of exactly 32 rows: its only tile transposed
+    (3, 16, 2128, 2048, 3),     # the gated memory-write projection: 16 rows, N = 64 + 2048 + 16
+    (40, 20, 2048, 128, 7),     # several transposed tiles per CTA (staging area reused)
 ])
 def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b, dtype):
     import torch
@@ -89,6 +95,7 @@ def test_memory_write_matches_oracle(M, d, dk, nu):
     (3, 144, 256, 96, 2),       # ragged M, K of 3 k-blocks of 32 words
     (2, 77, 64, 40, 1),         # N = 64 tile, ragged K (1.25 k-blocks)
     (1, 300, 128, 768, 1),      # N = 128, the 3B P
+    (2, 20, 128, 96, 1),        # N = 128, a 20-row node (transposed tile)
 ])
 def test_tc_grouped_gemm_tf32_matches_fp64(G, m, n, k, num_b):
     """fp32 operands on kind::tf32: each operand enters at tf32 precision
@@ -109,3 +116,40 @@ def test_tc_grouped_gemm_tf32_matches_fp64(G, m, n, k, num_b):
         ref = A[i].double().numpy() @ B[bidx[i]].double().numpy().T
         err = rel_l2(got[i], ref)
         assert 0 < err < 2e-3, (i, err)     # > 0: the product really ran at reduced precision
+
+
+SWAP_OFF_CHILD = """
+import numpy as np, torch
+from recurrent_memory_transformer_diag_b200 import grouped_gemm
+for G, m, n, k, num_b, tf32 in [(3, 1040, 512, 2048, 5, False), (3, 16, 2128, 2048, 3, False),
+                                (2, 1040, 2048, 384, 16, True)]:
+    g = torch.Generator().manual_seed(G * 1000 + m + n + k)
+    A = torch.randn(G, m, k, generator=g)
+    B = torch.randn(num_b, n, k, generator=g) * 0.05
+    if not tf32:
+        A, B = A.to(torch.bfloat16), B.to(torch.bfloat16)
+    bidx = [(3 * i + 1) % num_b for i in range(G)]
+    C = torch.full((G, m, n), float("nan"), device="cuda")
+    grouped_gemm(A.cuda(), B.cuda(), bidx, C, tf32=tf32)
+    torch.cuda.synchronize()
+    got = C.cpu().double().numpy()
+    An = A.double().numpy(); Bn = B.double().numpy()
+    for i in range(G):
+        ref = An[i] @ Bn[bidx[i]].T
+        err = np.linalg.norm(got[i] - ref) / np.linalg.norm(ref)
+        assert err < (2e-3 if tf32 else 1e-5), (G, m, n, k, i, err)
+print("SWAP_OFF_OK")
+"""
+
+
+def test_tc_grouped_gemm_without_transposed_tail():
+    """ARMT_GEMM_SWAP_TAIL=0 (the A/B switch) keeps the ragged last row tile
+    on the ordinary 128-row product; both layouts match the fp64 product."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, ARMT_GEMM_SWAP_TAIL="0")
+    r = subprocess.run([sys.executable, "-c", SWAP_OFF_CHILD], cwd=root, env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "SWAP_OFF_OK" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
