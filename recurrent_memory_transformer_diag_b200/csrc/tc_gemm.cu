@@ -36,10 +36,17 @@
 // padding.  The epilogue warps move D^T through shared memory (a row per
 // activation row) and the warps of TMEM quarter 0 run the ordinary epilogue
 // on those rows.
+//
+// 16-bit outputs (the next GEMM's operand copy, SwiGLU and QKV results) are
+// written through a 2 KB shared-memory slot per epilogue warp: a lane owns a
+// row, so a direct 16-byte store instruction touches 32 rows; through the
+// slot (16-byte pieces XOR-swizzled by row, conflict-free both ways) every
+// store instruction writes whole 64-byte row pieces of 8 rows.
 // Every mbarrier wait is bounded (about one second); on timeout the kernel
 // sets the device error word, drains its own outstanding copies and MMAs,
 // frees TMEM and returns.
 #include <cstdlib>
+#include <type_traits>
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -58,7 +65,8 @@ constexpr int BM = 128;
 constexpr int BK = 64;                 // 64 bf16 = 128 bytes = one swizzle row
 constexpr int EPI_WARPS = 8;           // two warps per TMEM lane quarter, each half of the columns
 constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;
-constexpr int SWAP_ROWS = 32;          // transposed ragged tile: rows (= MMA N) it covers
+constexpr int SWAP_ROWS = 16;          // transposed ragged tile: rows (= MMA N) it covers
+constexpr int XS_SLOT = 2048;          // per epilogue warp: 32 rows x 64 bytes of 16-bit output
 
 __device__ __forceinline__ void store_f16x32(f16* dst, const float* v) {
   // 32 values = 64 bytes: four 16-byte stores (dst 16-byte aligned)
@@ -90,7 +98,8 @@ struct Smem {
   static constexpr int STG_PITCH = BN + 4;
   static constexpr int STG_OFFSET = BAR_OFFSET + 256;
   static constexpr int STG_BYTES = SWAP ? SWAP_ROWS * STG_PITCH * 4 : 0;
-  static constexpr int TOTAL = STG_OFFSET + STG_BYTES + 1024;   // + barriers, staging, alignment slack
+  static constexpr int XS_OFFSET = STG_OFFSET + STG_BYTES;      // 16-byte aligned
+  static constexpr int TOTAL = XS_OFFSET + EPI_WARPS * XS_SLOT + 1024;   // + alignment slack
   static_assert(TOTAL + 64 <= 227 * 1024, "shared memory per CTA");
 };
 
@@ -134,6 +143,42 @@ __device__ __forceinline__ void store_bf16_32(bf16* dst, const float* v, int val
     for (int i = 0; i < 32; ++i)
       if (i < valid_cols) dst[i] = __float2bfloat16_rn(v[i]);
   }
+}
+
+// Warp-cooperative store of 32 16-bit values per lane: lane l's row is
+// dst0 + l * ld (the warp's rows; rows >= nrows and columns >= nv are not
+// written).  Every lane of the warp calls it (warp-uniform arguments except v).
+// xs: the warp's slot; the 16-byte piece q of row r sits at r * 64 + 16 (q ^
+// ((r >> 1) & 3)), so 8 consecutive lanes hit 8 different bank groups both
+// when a lane writes its row and when 4 lanes read one row.
+template <typename T>
+__device__ __forceinline__ void store16_warp(uint8_t* xs, T* dst0, long long ld, const float* v, int nv,
+                                             int nrows, int lane) {
+  static_assert(sizeof(T) == 2, "16-bit output");
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 pk;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if constexpr (std::is_same<T, bf16>::value) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+      } else {
+        __half2 h2 = __floats2half2_rn(v[q * 8 + 2 * i], v[q * 8 + 2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&h2);
+      }
+    }
+    *reinterpret_cast<uint4*>(xs + lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4)) = pk;
+  }
+  __syncwarp();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = 8 * k + (lane >> 2), q = lane & 3;
+    const uint4 x = *reinterpret_cast<const uint4*>(xs + r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+    if (r < nrows && 8 * q < nv) *reinterpret_cast<uint4*>(dst0 + (long long)r * ld + 8 * q) = x;
+  }
+  __syncwarp();
 }
 
 // h += v * rs on 32 columns (col % 4 == 0) of this thread's row of the
@@ -207,12 +252,22 @@ __device__ __forceinline__ float norm_row_scale(const TcGemmParams& p, int slot,
 // thread's row, loaded by the caller before it waited for the accumulator
 // (so that load's latency hides behind the main loop).  srow: null, or this
 // row of the transposed ragged tile's staging area (then tbase is unused).
+// xs: this warp's output slot, or null for direct 16-bit stores.
 template <int BN, int EPI>
 __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tbase, const NodeEntry& nd, int row,
                                              bool valid, int nb, int half, const float4* hpre,
-                                             const float* srow) {
+                                             const float* srow, uint8_t* xs) {
   const int slot = nd.z;
   const long long rofs = (long long)row;
+  // the warp's rows: lanes own consecutive rows; rows >= M are not stored
+  const int lane = threadIdx.x & 31;
+  const int wrow0 = row - lane;
+  const int nrows = min(32, p.M - wrow0);
+  // slot stores write 8-column pieces: 16-byte aligned rows and a column count
+  // that is a multiple of 8 (warp-uniform decision)
+  const int out_cols = EPI == TC_EPI_SWIGLU ? p.f_out : p.N;
+  const bool via_slot = xs != nullptr && (p.ldc & 7) == 0 && (out_cols & 7) == 0 &&
+                        (reinterpret_cast<uintptr_t>(p.C) & 15) == 0;
   if constexpr (EPI == TC_EPI_F32) {
     float rs = 1.f;
     if (p.rsq && valid) rs = norm_row_scale(p, slot, p.rsq_row0 + row);
@@ -254,30 +309,35 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       float v[32];
       acc_ld32(tbase, srow, c * 32, v);
       const int col = nb * BN + c * 32;
-      if (!valid || col >= p.N) continue;
+      if (col >= p.N) continue;   // warp-uniform; rows past M skip the residual below
       const int nv = p.N - col;
-      if (nv >= 32) {
-        float4* H4 = reinterpret_cast<float4*>(Hs + h_blocked_offset(row, col, p.ldh));
+      if (valid) {
+        if (nv >= 32) {
+          float4* H4 = reinterpret_cast<float4*>(Hs + h_blocked_offset(row, col, p.ldh));
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float4 o = hc[q];
-          o.x = fmaf(v[4 * q], rs, o.x);
-          o.y = fmaf(v[4 * q + 1], rs, o.y);
-          o.z = fmaf(v[4 * q + 2], rs, o.z);
-          o.w = fmaf(v[4 * q + 3], rs, o.w);
-          H4[q * 32] = o;
-          v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+          for (int q = 0; q < 8; ++q) {
+            float4 o = hc[q];
+            o.x = fmaf(v[4 * q], rs, o.x);
+            o.y = fmaf(v[4 * q + 1], rs, o.y);
+            o.z = fmaf(v[4 * q + 2], rs, o.z);
+            o.w = fmaf(v[4 * q + 3], rs, o.w);
+            H4[q * 32] = o;
+            v[4 * q] = o.x; v[4 * q + 1] = o.y; v[4 * q + 2] = o.z; v[4 * q + 3] = o.w;
+          }
+        } else {
+          resid_add32(Hs, row, col, p.ldh, v, rs, nv);
         }
-      } else {
-        resid_add32(Hs, row, col, p.ldh, v, rs, nv);
-      }
-      if (p.rsq) {
+        if (p.rsq) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
+          for (int i = 0; i < 32; ++i) ss = (i < nv) ? fmaf(v[i], v[i], ss) : ss;
+        }
       }
       if (EPI == TC_EPI_RESID_ACT) {
         f16* X = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + col;
-        store_act32(X, v, nv);
+        if (via_slot)
+          store16_warp(xs, X - (long long)lane * p.ldc, p.ldc, v, nv, nrows, lane);
+        else if (valid)
+          store_act32(X, v, nv);
         if (to_out) {
           bf16* O = reinterpret_cast<bf16*>(p.out) + ((long long)nd.x * p.seg_len + row) * p.N + col;
           store_bf16_32(O, v, nv);
@@ -304,10 +364,11 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         acc_ld32(tbase, srow, c1 * 32, v1);
         acc_ld32(tbase, srow, c2 * 32, v2);
         const int col1 = nb * BN + c1 * 32, col2 = nb * BN + c2 * 32;
-        if (!valid || col1 >= p.N) continue;
+        if (col1 >= p.N) continue;   // warp-uniform; rows past M are computed but not stored
         if (rot) {
           // frequency-major table: the warp's 32 rows read 32 consecutive entries
-          const float2* cs = p.rope + (long long)(pc * 32) * p.rope_pitch + row;
+          // (rows past M read row 0's)
+          const float2* cs = p.rope + (long long)(pc * 32) * p.rope_pitch + (valid ? row : 0);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const float2 a = cs[(long long)i * p.rope_pitch];
@@ -325,10 +386,16 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
         // value heads go only to V^T when it is requested (its reader takes V^T)
         if (!(p.vt && !rot)) {
           f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc;
-          store_act32(C + col1, v1, p.N - col1);
-          if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+          if (via_slot) {
+            f16* C0 = C - (long long)lane * p.ldc;
+            store16_warp(xs, C0 + col1, p.ldc, v1, p.N - col1, nrows, lane);
+            if (col2 < p.N) store16_warp(xs, C0 + col2, p.ldc, v2, p.N - col2, nrows, lane);
+          } else if (valid) {
+            store_act32(C + col1, v1, p.N - col1);
+            if (col2 < p.N) store_act32(C + col2, v2, p.N - col2);
+          }
         }
-        if (p.vt && !rot) {
+        if (p.vt && !rot && valid) {
           // value head: dims pc*32.. and hd/2 + pc*32.. of this row, transposed
           const int vh = head - p.rope_heads;
           f16* vt = p.vt + (((long long)slot * p.n_vheads + vh) * hd) * p.vt_pitch + row;
@@ -351,14 +418,17 @@ __device__ __forceinline__ void run_epilogue(const TcGemmParams& p, uint32_t tba
       acc_ld32(tbase, srow, c * 32, g);
       acc_ld32(tbase, srow, HALF + c * 32, u);
       const int f = f0 + c * 32;
-      if (!valid || f >= p.f_out) continue;
+      if (f >= p.f_out) continue;   // warp-uniform; rows past M are computed but not stored
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float gi = g[i] * rs;
         g[i] = gi / (1.f + __expf(-gi)) * (u[i] * rs);
       }
       f16* C = reinterpret_cast<f16*>(p.C) + (long long)slot * p.c_slot_stride + rofs * p.ldc + f;
-      store_act32(C, g, p.f_out - f);
+      if (via_slot)
+        store16_warp(xs, C - (long long)lane * p.ldc, p.ldc, g, p.f_out - f, nrows, lane);
+      else if (valid)
+        store_act32(C, g, p.f_out - f);
     }
   }
 }
@@ -539,6 +609,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int half = (warp - 2) >> 2;        // which half of the tile's columns
     const int row_in_tile = quarter * 32 + lane;
+    uint8_t* xs = smem + SM::XS_OFFSET + (warp - 2) * XS_SLOT;   // this warp's 16-bit output slot
     int buf = 0;
     uint32_t acc_phase = 0;
     uint32_t stg_phase = 0;   // transposed ragged tiles seen so far, mod 2
@@ -575,8 +646,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             break;
           }
           if (half < BN / 128) {
-            float v[32];
-            tmem_ld32(tbase + (uint32_t)(half * SWAP_ROWS), v);
+            float v[SWAP_ROWS];
+            tmem_ld16(tbase + (uint32_t)(half * SWAP_ROWS), v);
             const int col = half * 128 + quarter * 32 + lane;
 #pragma unroll
             for (int i = 0; i < SWAP_ROWS; ++i) stg[i * SM::STG_PITCH + col] = v[i];
@@ -591,13 +662,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               *abort_flag = 1;
               break;
             }
-            run_epilogue<BN, EPI>(p, 0u, nd, row, valid, nb, half, hpre, stg + lane * SM::STG_PITCH);
+            // lanes >= SWAP_ROWS own rows past M (nothing is stored for them): they
+            // read staged row 0, so every read stays inside the SWAP_ROWS-row area
+            const float* srow = stg + (lane < SWAP_ROWS ? lane : 0) * SM::STG_PITCH;
+            run_epilogue<BN, EPI>(p, 0u, nd, row, valid, nb, half, hpre, srow, xs);
             mbar_arrive(stg_empty);
           }
           stg_phase ^= 1;
         }
       } else {
-        run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr);
+        run_epilogue<BN, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr, xs);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -808,7 +882,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
-      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr);
+      run_epilogue<256, EPI>(p, tbase, nd, row, valid, nb, half, hpre, nullptr, nullptr);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty0 + (uint32_t)(buf * sizeof(uint64_t)));

@@ -19,12 +19,13 @@ pytestmark = pytest.mark.gpu
     (16, 1040, 3072, 2048, 16), # a full 1B wave of QKV shapes
     (2, 512, 256, 128, 2),      # rows in whole 256-row CTA-pair tiles only
     (1, 300, 304, 200, 1),      # one pair tile + a 44-row one-CTA rest, ragged N and K
-    # transposed ragged row tile (last tile of <= 32 rows, N a multiple of 128):
-    (2, 150, 128, 256, 2),      # N = 128 tile, 22-row tail
+    # transposed ragged row tile (last tile of <= 16 rows, N a multiple of 128):
+    (2, 144, 128, 256, 2),      # N = 128 tile, 16-row tail
     (1, 129, 256, 128, 1),      # a 1-row tail
-    (2, 32, 256, 64, 1),        # a node of exactly 32 rows: its only tile transposed
+    (2, 16, 256, 64, 1),        # a node of exactly 16 rows: its only tile transposed
     (3, 16, 2128, 2048, 3),     # the gated memory-write projection: 16 rows, N = 64 + 2048 + 16
-    (40, 20, 2048, 128, 7),     # several transposed tiles per CTA (staging area reused)
+    (40, 12, 2048, 128, 7),     # several transposed tiles per CTA (staging area reused)
+    (2, 150, 256, 256, 2),      # a 22-row tail: an ordinary (partly filled) row tile
 ])
 def test_tc_grouped_gemm_matches_fp64(G, m, n, k, num_b, dtype):
     import torch
@@ -95,7 +96,7 @@ def test_memory_write_matches_oracle(M, d, dk, nu):
     (3, 144, 256, 96, 2),       # ragged M, K of 3 k-blocks of 32 words
     (2, 77, 64, 40, 1),         # N = 64 tile, ragged K (1.25 k-blocks)
     (1, 300, 128, 768, 1),      # N = 128, the 3B P
-    (2, 20, 128, 96, 1),        # N = 128, a 20-row node (transposed tile)
+    (2, 10, 128, 96, 1),        # N = 128, a 10-row node (transposed tile)
 ])
 def test_tc_grouped_gemm_tf32_matches_fp64(G, m, n, k, num_b):
     """fp32 operands on kind::tf32: each operand enters at tf32 precision
