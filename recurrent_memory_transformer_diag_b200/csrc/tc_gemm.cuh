@@ -44,7 +44,7 @@ struct TcGemmParams {
   // final hidden states (down-projection epilogue of last-layer nodes)
   void* out; int out_layer; int seg_len;
   unsigned* err;            // device error word (bounded waits)
-  int swap_tail;            // 1: the last row tile (at most 32 rows) is computed transposed (set by the launcher)
+  int swap_tail;            // 1: the last row tile (at most 16 rows) is computed transposed (set by the launcher)
   int debug_no_loads;       // test hook: the producer issues no copies, so the first wait for a stage
                             // cannot complete and the bounded-wait error path runs (never set by the forward)
 };
