@@ -68,6 +68,14 @@ def kind_flops(cfg, n_nodes: int, T: int):
     return {k: v * n_nodes for k, v in per.items()}
 
 
+def weight_bytes(cfg) -> int:
+    """Bytes of the stacked 16-bit layer weights (attention, MLP, memory projections)."""
+    d, hd = cfg.d_model, cfg.head_dim
+    per_layer = ((cfg.n_heads + 2 * cfg.n_kv_heads) * hd * d + d * cfg.n_heads * hd + 3 * cfg.d_ffn * d
+                 + (cfg.d_key + cfg.d_key + d) * d)
+    return 2 * cfg.n_layers * per_layer
+
+
 def kind_bytes(cfg, n_nodes: int, T: int):
     """Algorithmic HBM bytes of the memory-bound kinds over n_nodes nodes."""
     Tp = T + cfg.n_mem
@@ -318,7 +326,7 @@ def run_ours(args, cfg, S):
     dms, dcnt = prof[dominant]
     d_flops_launch = flops.get(dominant, 0) / max(dcnt, 1)
     achieved = d_flops_launch / (dms / dcnt / 1e3) / 1e12
-    traffic = read_traffic(dominant)
+    traffic = read_traffic(dominant, cfg.name, T)
     if traffic is not None:
         traffic = round(traffic * n_nodes / dcnt)   # bytes per node x nodes per launch (average over launches)
     roofline = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1), "peak": peak_tf,
@@ -377,7 +385,8 @@ def run_ours(args, cfg, S):
         "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
         "config": {"workload": workload_name(cfg, S, args.schedule), "segments": S, "seg_len": T,
                    "batch": 1, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs (emb 512 MB at 1B) and weights exceed the 126 MB L2; no flush needed",
+                   "l2": (f"inputs (emb {S * T * cfg.d_model * 2 / 1e6:.0f} MB) and weights "
+                          f"({weight_bytes(cfg) / 1e9:.1f} GB) exceed the 126 MB L2; no flush needed"),
                    "weights": "random init N(0,0.02) (bf16-rounded), embeddings N(0,1)",
                    "precision": ("bf16 weights held exactly in fp16, fp16 MMA operands, fp32 accumulate, "
                                  "fp32 residual stream and memory state; bf16 embeddings in, bf16 hidden out"
@@ -483,11 +492,12 @@ def full_attention(cfg, weights, emb, tokens, ms_armt, stream):
                         f"(no memory tokens, one segment), same kernels"}
 
 
-def read_traffic(kernel: str):
+def read_traffic(kernel: str, config: str, seg_len: int):
     """DRAM bytes per node of `kernel` from the committed ncu summary
     (profiles/traffic.txt: dram__bytes_read.sum + dram__bytes_write.sum of one
     captured full wave, divided by its nodes), if it was taken on the current
-    kernel source (the source hash is recorded there); else None."""
+    kernel source (the source hash is recorded there) and on this model shape
+    and segment length; else None."""
     import hashlib
     summ = os.path.join(ROOT, "profiles", "traffic.txt")
     src = os.path.join(ROOT, "recurrent_memory_transformer_diag_b200", "csrc", "tc_gemm.cu")
@@ -496,7 +506,8 @@ def read_traffic(kernel: str):
     h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     for line in open(summ):
         parts = line.split()
-        if len(parts) >= 3 and parts[0] == kernel and parts[2] == h:
+        if (len(parts) >= 5 and parts[0] == kernel and parts[2] == h and parts[3] == config
+                and parts[4] == str(seg_len)):
             return float(parts[1])
     return None
 
