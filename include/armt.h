@@ -195,6 +195,43 @@ armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int se
                               void* out_hidden_host, float* out_A_host, float* out_z_host,
                               void* stream);
 
+/* One wave of a layer-pipelined forward (the layer-pipeline split of the
+ * diagonal schedule: the diagonal wave is a pipeline wavefront, Pith review of
+ * arXiv 2506.05229, "What carries the argument"; skill page "Diagonal
+ * Batching for Recurrent Memory Transformers", "Practical Guidance").  A model
+ * of total_layers layers is cut into contiguous layer blocks, one per stage
+ * (one GPU each); a stage's context is created with n_layers = its block's
+ * layer count and loaded with those layers' weights (mem_emb too).  Every
+ * stage calls this for every global wave i = 0 .. S + total_layers - 2, in
+ * order; the call enqueues, on `stream`, the nodes (s, l) with s + l = i,
+ * 0 <= s < S and layer_offset <= l < layer_offset + n_layers (nothing when
+ * there are none).  With first = layer_offset and last = layer_offset +
+ * n_layers - 1:
+ *   emb        device [S*seg_len, d] context dtype; read when first == 0
+ *   in_rows    device [seg_len + n_mem, d] fp32: when first > 0 and the wave
+ *              holds node (i - first, first), that segment's residual rows
+ *              after layer first - 1 (the previous stage's out_rows of wave
+ *              i - 1); otherwise unused (may be null)
+ *   out_rows   device [seg_len + n_mem, d] fp32: when last < total_layers - 1
+ *              and the wave holds node (i - last, last), receives that node's
+ *              residual rows after layer `last`; otherwise unused (may be null)
+ *   out_hidden device [S*seg_len, d] context dtype: when last ==
+ *              total_layers - 1, the final hidden states as armt_forward
+ *   A, z       device [n_layers, d, P] / [n_layers, P] fp32: this stage's
+ *              layers' state; the wave-0 call zeroes them unless carry_state
+ *              is 1
+ * Each wave is enqueued directly (no graph); the memory write runs on
+ * `stream` (no second stream), so consecutive calls need no other
+ * synchronisation.  The result equals armt_forward over all layers bit for
+ * bit when the model has memory tokens (n_mem > 0); without them the
+ * RMSNorm sums of a stage's first layer are recomputed and match to rounding.
+ * Errors: INVALID_ARG (a buffer the wave needs is null, wave or layer range
+ * out of bounds), NOT_LOADED, SHAPE (S > max_segments or seg_len >
+ * max_seg_len), CUDA. */
+armt_status armt_stage_wave(armt_ctx* ctx, int S, int seg_len, int wave, int layer_offset, int total_layers,
+                            const void* emb, const float* in_rows, float* out_rows, void* out_hidden,
+                            float* A, float* z, int carry_state, void* stream);
+
 /* Wait for `stream`, then report and clear the device-side error word that
  * kernels set when a bounded wait runs out (ARMT_ERR_DEVICE_TIMEOUT);
  * ARMT_OK otherwise (ARMT_ERR_CUDA if the stream itself failed). */

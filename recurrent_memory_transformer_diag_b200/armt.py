@@ -34,7 +34,7 @@ EXPORTS = (
     "armt_forward_host", "armt_device_status", "armt_launch_count", "armt_destroy",
     "armt_status_string", "armt_last_error", "armt_grouped_gemm", "armt_memory_write",
     "armt_kernel_kinds", "armt_kernel_kind_name", "armt_profile_forward", "armt_memory_write_static",
-    "armt_forward_ex", "armt_test_bounded_wait",
+    "armt_forward_ex", "armt_test_bounded_wait", "armt_stage_wave",
 )
 
 
@@ -94,6 +94,7 @@ def lib() -> ctypes.CDLL:
     L.armt_memory_write.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
     L.armt_memory_write_static.argtypes = [c_int, c_int, c_int, c_int, c_float, vp, vp, vp, vp, vp, vp]
     L.armt_test_bounded_wait.argtypes = [vp]
+    L.armt_stage_wave.argtypes = [vp, c_int, c_int, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, c_int, vp]
     L.armt_kernel_kinds.argtypes = []
     L.armt_kernel_kind_name.argtypes = [c_int]
     L.armt_kernel_kind_name.restype = ctypes.c_char_p
@@ -123,7 +124,9 @@ def _stream_handle(stream) -> Optional[int]:
     return stream.cuda_stream
 
 
-def _ptr(t) -> int:
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None   # NULL
     return t.data_ptr() if hasattr(t, "data_ptr") else t.ctypes.data
 
 
@@ -195,6 +198,15 @@ class Armt:
         _check(lib().armt_forward_ex(self._h, _ptr(emb), n_segments, seg_len, _ptr(out_hidden), _ptr(A),
                                      _ptr(z), int(bool(carry_state)), _stream_handle(stream)),
                "armt_forward_ex", self._h)
+
+    def stage_wave(self, n_segments: int, seg_len: int, wave: int, layer_offset: int, total_layers: int,
+                   emb, in_rows, out_rows, out_hidden, A, z, carry_state: bool = False, stream=None):
+        """armt_stage_wave: one global wave of a layer-pipelined forward for this
+        context's layer block (device buffers; None where the wave needs none)."""
+        _check(lib().armt_stage_wave(self._h, n_segments, seg_len, wave, layer_offset, total_layers,
+                                     _ptr(emb), _ptr(in_rows), _ptr(out_rows), _ptr(out_hidden), _ptr(A),
+                                     _ptr(z), int(bool(carry_state)), _stream_handle(stream)),
+               "armt_stage_wave", self._h)
 
     def forward_host(self, emb, n_segments: int, seg_len: int, out_hidden, out_A, out_z, stream=None):
         """Host buffers (numpy arrays or pinned CPU tensors): see armt_forward_host."""

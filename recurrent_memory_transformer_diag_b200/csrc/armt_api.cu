@@ -126,30 +126,33 @@ armt_status validate_config(const armt_config* c, const char** why) {
 }
 
 // Node table for (S, schedule): entries in launch order, grouped into waves.
+// The wave made of table entries first .. end (layers 0 .. L-1 of the context).
+Wave summarize_wave(const std::vector<NodeEntry>& tab, int first, int L) {
+  Wave w;
+  w.first = first;
+  w.count = (int)tab.size() - first;
+  w.any_first_layer = false;
+  w.any_last_layer = false;
+  w.first_layer_pos = -1;
+  w.first_layer_seg = -1;
+  w.last_layer_seg = -1;
+  for (int k = first; k < (int)tab.size(); ++k) {
+    if (tab[k].y == 0) {   // a wave holds at most one layer-0 node
+      w.first_layer_pos = k - first;
+      w.first_layer_seg = tab[k].x;
+    }
+    if (tab[k].y == L - 1) w.last_layer_seg = tab[k].x;   // and at most one last-layer node
+    w.any_first_layer |= tab[k].y == 0;
+    w.any_last_layer |= tab[k].y == L - 1;
+  }
+  return w;
+}
+
 void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeEntry>& tab,
                  std::vector<Wave>& waves) {
   tab.clear();
   waves.clear();
-  auto push_wave = [&](int first) {
-    Wave w;
-    w.first = first;
-    w.count = (int)tab.size() - first;
-    w.any_first_layer = false;
-    w.any_last_layer = false;
-    w.first_layer_pos = -1;
-    w.first_layer_seg = -1;
-    w.last_layer_seg = -1;
-    for (int k = first; k < (int)tab.size(); ++k) {
-      if (tab[k].y == 0) {   // a wave holds at most one layer-0 node
-        w.first_layer_pos = k - first;
-        w.first_layer_seg = tab[k].x;
-      }
-      if (tab[k].y == L - 1) w.last_layer_seg = tab[k].x;   // and at most one last-layer node
-      w.any_first_layer |= tab[k].y == 0;
-      w.any_last_layer |= tab[k].y == L - 1;
-    }
-    waves.push_back(w);
-  };
+  auto push_wave = [&](int first) { waves.push_back(summarize_wave(tab, first, L)); };
   if (sched == ARMT_SCHED_DIAGONAL) {
     for (int i = 0; i < S + L - 1; ++i) {
       const int first = (int)tab.size();
@@ -166,6 +169,24 @@ void build_table(int S, int L, int slots, armt_schedule sched, std::vector<NodeE
         tab.push_back(make_int4(s, l, s % slots, 0));
         push_wave(first);
       }
+  }
+}
+
+// Layer-pipeline stage holding global layers offset .. offset + L - 1 of a
+// model of `total` layers: one entry per global wave i = 0 .. S + total - 2
+// (possibly empty), with the nodes (s, j) of local layer j = l - offset,
+// s = i - l, 0 <= s < S.
+void build_stage_table(int S, int L, int offset, int total, int slots, std::vector<NodeEntry>& tab,
+                       std::vector<Wave>& waves) {
+  tab.clear();
+  waves.clear();
+  for (int i = 0; i < S + total - 1; ++i) {
+    const int first = (int)tab.size();
+    for (int j = 0; j < L; ++j) {
+      const int s = i - offset - j;
+      if (s >= 0 && s < S) tab.push_back(make_int4(s, j, s % slots, 0));
+    }
+    waves.push_back(summarize_wave(tab, first, L));
   }
 }
 
@@ -220,8 +241,9 @@ struct Launcher {
 
 // fp32 path: enqueue every kernel of one wave (SIMT kernels, fp32 throughout).
 // T = seg_len, Tp = T + M rows per node.
+// stage_in / stage_out: layer-pipeline hand-off rows (null in a whole forward).
 void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
-                  cudaStream_t st, Launcher& L) {
+                  cudaStream_t st, Launcher& L, const float* stage_in = nullptr, float* stage_out = nullptr) {
   const Dims& dm = ctx->dm;
   Workspace& ws = ctx->ws;
   const Weights& w = ctx->w;
@@ -233,6 +255,8 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
 
   if (wv.any_first_layer)
     L("init", [&] {   // only the wave's layer-0 node
+      if (stage_in)
+        return launch_stage_rows_in(dm, nodes + wv.first_layer_pos, 1, 0, Tp, stage_in, ws.h, nullptr, st);
       return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, nullptr, st);
     });
 
@@ -325,7 +349,9 @@ void enqueue_wave(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* o
     });
   }
 
-  if (wv.any_last_layer)
+  if (wv.any_last_layer && stage_out)
+    L("output", [&] { return launch_stage_rows_out(dm, nodes, n, dm.L - 1, Tp, ws.h, stage_out, st); });
+  else if (wv.any_last_layer)
     L("output", [&] { return launch_output(dm, nodes, n, T, Tp, ws.h, out, st); });
 }
 
@@ -364,7 +390,8 @@ struct WriteOverlap {
 // A itself at tf32 precision (fp16's mantissa, fp32's range), so no copy of
 // A is kept.  Residual stream, accumulation and the memory state are fp32.
 void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void* out, float* A, float* z,
-                     cudaStream_t st, Launcher& L, WriteOverlap* ov = nullptr) {
+                     cudaStream_t st, Launcher& L, WriteOverlap* ov = nullptr, const float* stage_in = nullptr,
+                     float* stage_out = nullptr) {
   const Dims& dm = ctx->dm;
   Workspace& ws = ctx->ws;
   const Weights& w = ctx->w;
@@ -404,6 +431,8 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
   if (wv.any_first_layer) {
     if (ov) after(st, ov->kv);
     L("init", [&] {   // only the wave's layer-0 node
+      if (stage_in)
+        return launch_stage_rows_in(dm, nodes + wv.first_layer_pos, 1, 0, Tp, stage_in, ws.h, ws.xb, st);
       return launch_init_first_layer(dm, nodes + wv.first_layer_pos, 1, T, Tp, emb, w.mem_emb, ws.h, (f16*)ws.xb, st);
     });
   }
@@ -482,6 +511,9 @@ void enqueue_wave_tc(armt_ctx* ctx, const Wave& wv, int T, const void* emb, void
     norm_partials(p);   // for the memory-write rows
     return launch_tc_gemm(op, p, TC_EPI_RESID_ACT, 256, sms, st);
   });
+  // layer pipeline: this stage's last layer hands its rows to the next stage
+  if (stage_out && wv.any_last_layer)
+    L("output", [&] { return launch_stage_rows_out(dm, nodes, n, dm.L - 1, Tp, ws.h, stage_out, st); });
 
   // ---- memory write: [k | v] = RMSNorm(m) [Wk_mem; Wv_mem]^T for the M memory
   // rows (rows T..T'-1 of the fp16 copy of the layer output the down GEMM
@@ -538,6 +570,7 @@ armt_status ensure_table(armt_ctx* ctx, int S, cudaStream_t st) {
   ARMT_TRY(cudaStreamSynchronize(st), "upload node table");
   ctx->table_S = S;
   ctx->table_sched = (int)sched;
+  ctx->stage_S = -1;   // the stage table (same device buffer) is gone
   return ARMT_OK;
 }
 
@@ -901,6 +934,59 @@ extern "C" armt_status armt_forward_ex(armt_ctx* ctx, const void* emb, int S, in
   if (s != ARMT_OK) return s;
   if (carry_state != 0 && carry_state != 1) return fail(ctx, ARMT_ERR_INVALID_ARG, "carry_state must be 0 or 1");
   return forward_impl(ctx, emb, S, seg_len, out_hidden, A, z, (cudaStream_t)stream, carry_state == 1);
+}
+
+extern "C" armt_status armt_stage_wave(armt_ctx* ctx, int S, int seg_len, int wave, int layer_offset,
+                                       int total_layers, const void* emb, const float* in_rows, float* out_rows,
+                                       void* out_hidden, float* A, float* z, int carry_state, void* stream) {
+  if (!ctx) return ARMT_ERR_INVALID_ARG;
+  if (!A || !z) return fail(ctx, ARMT_ERR_INVALID_ARG, "null state buffer");
+  if (S < 1 || seg_len < 1) return fail(ctx, ARMT_ERR_INVALID_ARG, "S and seg_len must be >= 1");
+  if (carry_state != 0 && carry_state != 1) return fail(ctx, ARMT_ERR_INVALID_ARG, "carry_state must be 0 or 1");
+  if (!ctx->w.loaded) return fail(ctx, ARMT_ERR_NOT_LOADED, "weights not loaded");
+  if (S > ctx->cfg.max_segments) return fail(ctx, ARMT_ERR_SHAPE, "S > max_segments");
+  if (seg_len > ctx->cfg.max_seg_len) return fail(ctx, ARMT_ERR_SHAPE, "seg_len > max_seg_len");
+  const int nl = ctx->dm.L;
+  if (layer_offset < 0 || total_layers < 1 || layer_offset + nl > total_layers)
+    return fail(ctx, ARMT_ERR_INVALID_ARG, "layer block outside the model");
+  if (wave < 0 || wave >= S + total_layers - 1) return fail(ctx, ARMT_ERR_INVALID_ARG, "wave out of range");
+  const int first = layer_offset, last = layer_offset + nl - 1;
+  const bool has_first = wave - first >= 0 && wave - first < S;
+  const bool has_last = wave - last >= 0 && wave - last < S;
+  const bool final_stage = last == total_layers - 1;
+  if (has_first && first == 0 && !emb) return fail(ctx, ARMT_ERR_INVALID_ARG, "null emb");
+  if (has_first && first > 0 && !in_rows) return fail(ctx, ARMT_ERR_INVALID_ARG, "null in_rows");
+  if (has_last && !final_stage && !out_rows) return fail(ctx, ARMT_ERR_INVALID_ARG, "null out_rows");
+  if (has_last && final_stage && !out_hidden) return fail(ctx, ARMT_ERR_INVALID_ARG, "null out_hidden");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (ctx->stage_S != S || ctx->stage_offset != layer_offset || ctx->stage_total != total_layers) {
+    std::vector<NodeEntry> tab;
+    build_stage_table(S, nl, layer_offset, total_layers, ctx->ws.slots, tab, ctx->stage_waves);
+    if ((int)tab.size() > ctx->ws.nodes_cap) return fail(ctx, ARMT_ERR_SHAPE, "node table too large");
+    // stream-ordered after the work that may still read the previous table
+    ARMT_TRY(cudaMemcpyAsync(ctx->ws.nodes, tab.data(), tab.size() * sizeof(NodeEntry), cudaMemcpyHostToDevice, st),
+             "upload stage table");
+    ARMT_TRY(cudaStreamSynchronize(st), "upload stage table");
+    ctx->table_S = -1;   // the forward's table is gone
+    ctx->stage_S = S;
+    ctx->stage_offset = layer_offset;
+    ctx->stage_total = total_layers;
+  }
+  const Dims& dm = ctx->dm;
+  if (wave == 0 && !carry_state) {
+    ARMT_TRY(cudaMemsetAsync(A, 0, (size_t)dm.L * dm.d * dm.P * sizeof(float), st), "zero A");
+    ARMT_TRY(cudaMemsetAsync(z, 0, (size_t)dm.L * dm.P * sizeof(float), st), "zero z");
+  }
+  const Wave& wv = ctx->stage_waves[wave];
+  if (wv.count == 0) return ARMT_OK;
+  Launcher L;
+  const float* sin = first > 0 ? in_rows : nullptr;
+  float* sout = final_stage ? nullptr : out_rows;
+  void* out = final_stage ? out_hidden : nullptr;
+  if (dm.bf16) enqueue_wave_tc(ctx, wv, seg_len, emb, out, A, z, st, L, nullptr, sin, sout);
+  else enqueue_wave(ctx, wv, seg_len, emb, out, A, z, st, L, sin, sout);
+  if (L.err != cudaSuccess) return cuda_fail(ctx, L.err, L.where);
+  return ARMT_OK;
 }
 
 namespace {

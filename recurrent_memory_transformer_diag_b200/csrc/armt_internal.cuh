@@ -155,6 +155,11 @@ struct armt_ctx {
   // node table of the last (S, schedule)
   int table_S = -1, table_sched = -1;
   std::vector<armt::Wave> waves;
+  // node table of the last layer-pipeline stage call (S, layer offset, total
+  // layers); it shares the device table with the forward, so uploading one
+  // invalidates the other
+  int stage_S = -1, stage_offset = -1, stage_total = -1;
+  std::vector<armt::Wave> stage_waves;
   // host-buffer forward staging
   void* st_emb = nullptr; void* st_out = nullptr; float* st_A = nullptr; float* st_z = nullptr;
   size_t st_tokens = 0;
@@ -220,6 +225,11 @@ cudaError_t launch_memw_phi(const Dims& dm, const NodeEntry* nodes, int n, const
 cudaError_t launch_memw_update(const Dims& dm, const NodeEntry* nodes, int n, const float* kv,
                                const float* phik, const float* gram, const float* coef, const float* beta,
                                float* A_state, cudaStream_t st);
+// layer-pipeline hand-off rows of the node at local layer `layer` (see simt_kernels.cu)
+cudaError_t launch_stage_rows_in(const Dims& dm, const NodeEntry* nodes, int n, int layer, int Tp, const float* in,
+                                 float* h, void* xb, cudaStream_t st);
+cudaError_t launch_stage_rows_out(const Dims& dm, const NodeEntry* nodes, int n, int layer, int Tp, const float* h,
+                                  float* out, cudaStream_t st);
 cudaError_t launch_output(const Dims& dm, const NodeEntry* nodes, int n, int T, int Tp,
                           const float* h, void* out, cudaStream_t st);
 

@@ -423,6 +423,98 @@ cudaError_t launch_swiglu(const Dims& dm, const NodeEntry* nodes, int n, int Tp,
 }
 
 // ---------------------------------------------------------------------------
+// Layer-pipeline hand-off: the residual rows [Tp][d] (fp32, row-major) after
+// the previous stage's last layer are loaded into the slot of this stage's
+// first-layer node, and those of this stage's last-layer node are stored.
+// Tensor-core path: the residual is row-blocked and the first layer's GEMMs
+// read its fp16 copy, which the load writes as the down-projection epilogue
+// would have (round to nearest); one block per 32 rows x 64 columns through a
+// shared tile, as for the layer-0 input.  fp32 path: row-major copies.
+// ---------------------------------------------------------------------------
+__global__ void stage_rows_in_blocked_kernel(const NodeEntry* nodes, int layer, int Tp, int d, const float* in,
+                                             float* h, f16* xb) {
+  __shared__ float tile[32][65];
+  const NodeEntry nd = nodes[blockIdx.z];
+  if (nd.y != layer) return;
+  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 64;
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int r = e >> 6, c = e & 63;
+    const int t = r0 + r, col = c0 + c;
+    float v = 0.f;
+    if (col < d && t < Tp) {
+      v = in[(long long)t * d + col];
+      xb[((long long)nd.z * Tp + t) * d + col] = __float2half_rn(v);
+    }
+    tile[r][c] = v;
+  }
+  __syncthreads();
+  float* hs = h + (long long)nd.z * rows_blocked(Tp) * d;
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int g = e >> 7, r = (e >> 2) & 31, cc = e & 3;   // column group, row, column in group
+    const int col = c0 + g * 4 + cc;
+    if (col < d) hs[h_blocked_offset(r0 + r, col, d)] = tile[r][g * 4 + cc];
+  }
+}
+
+__global__ void stage_rows_out_blocked_kernel(const NodeEntry* nodes, int layer, int Tp, int d, const float* h,
+                                              float* out) {
+  __shared__ float tile[32][65];
+  const NodeEntry nd = nodes[blockIdx.z];
+  if (nd.y != layer) return;
+  const int r0 = blockIdx.x * 32, c0 = blockIdx.y * 64;
+  const float* hs = h + (long long)nd.z * rows_blocked(Tp) * d;
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int g = e >> 7, r = (e >> 2) & 31, cc = e & 3;
+    const int col = c0 + g * 4 + cc;
+    tile[r][g * 4 + cc] = col < d ? hs[h_blocked_offset(r0 + r, col, d)] : 0.f;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 32 * 64; e += blockDim.x) {
+    const int r = e >> 6, c = e & 63;
+    const int t = r0 + r, col = c0 + c;
+    if (col < d && t < Tp) out[(long long)t * d + col] = tile[r][c];
+  }
+}
+
+// fp32 path: rows of the node's row-major slot <-> [Tp][d] (to_slot selects the direction)
+__global__ void stage_rows_copy_kernel(const NodeEntry* nodes, int layer, int Tp, int d, const float* src,
+                                       float* dst, int to_slot) {
+  const NodeEntry nd = nodes[blockIdx.y];
+  if (nd.y != layer) return;
+  const int t = blockIdx.x;
+  const long long slot_row = ((long long)nd.z * Tp + t) * d, flat_row = (long long)t * d;
+  const float* s = src + (to_slot ? flat_row : slot_row);
+  float* o = dst + (to_slot ? slot_row : flat_row);
+  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = s[c];
+}
+
+cudaError_t launch_stage_rows_in(const Dims& dm, const NodeEntry* nodes, int n, int layer, int Tp, const float* in,
+                                 float* h, void* xb, cudaStream_t st) {
+  if (dm.bf16) {
+    if (!xb || dm.d % 4) return cudaErrorInvalidValue;
+    dim3 grid(rows_blocked(Tp) / 32, (dm.d + 63) / 64, n);
+    stage_rows_in_blocked_kernel<<<grid, 256, 0, st>>>(nodes, layer, Tp, dm.d, in, h, (f16*)xb);
+  } else {
+    dim3 grid(Tp, n);
+    stage_rows_copy_kernel<<<grid, 256, 0, st>>>(nodes, layer, Tp, dm.d, in, h, 1);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage_rows_out(const Dims& dm, const NodeEntry* nodes, int n, int layer, int Tp, const float* h,
+                                  float* out, cudaStream_t st) {
+  if (dm.bf16) {
+    if (dm.d % 4) return cudaErrorInvalidValue;
+    dim3 grid(rows_blocked(Tp) / 32, (dm.d + 63) / 64, n);
+    stage_rows_out_blocked_kernel<<<grid, 256, 0, st>>>(nodes, layer, Tp, dm.d, h, out);
+  } else {
+    dim3 grid(Tp, n);
+    stage_rows_copy_kernel<<<grid, 256, 0, st>>>(nodes, layer, Tp, dm.d, h, out, 0);
+  }
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Final hidden states: node (s, L-1) writes rows 0..T-1 of its residual
 // stream to out[s*T + t].
 // ---------------------------------------------------------------------------
