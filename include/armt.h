@@ -222,7 +222,10 @@ armt_status armt_forward_host(armt_ctx* ctx, const void* emb_host, int S, int se
  *              is 1
  * Each wave is enqueued directly (no graph); the memory write runs on
  * `stream` (no second stream), so consecutive calls need no other
- * synchronisation.  The result equals armt_forward over all layers bit for
+ * synchronisation.  The stage's node table shares a device buffer with the
+ * whole forward's: a context used for both must issue them on one stream
+ * (or order them), and a change of (S, layer_offset, total_layers) waits for
+ * that stream while the new table is uploaded.  The result equals armt_forward over all layers bit for
  * bit when the model has memory tokens (n_mem > 0); without them the
  * RMSNorm sums of a stage's first layer are recomputed and match to rounding.
  * Errors: INVALID_ARG (a buffer the wave needs is null, wave or layer range
